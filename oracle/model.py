@@ -1,0 +1,417 @@
+"""Oracle: one masked block-diffusion denoising pass, written out plainly (TEST INFRASTRUCTURE).
+
+Only tests/, the smoke check and the benchmark's CPU-baseline leg use this module.
+
+What the pages fix (page titles abbreviated as "Distributed" = "Diffusion LLMs are
+not a good fit for distributed inference", "DiffusionGemma" = "DiffusionGemma: 4x
+Faster Text Generation via Parallel Diffusion", "What changes" = "Diffusion LLMs:
+what changes when you stop generating one token at a time"):
+
+* generation starts from an all-[MASK] block and repeatedly commits the positions
+  the model is most confident about until none is masked (What changes, section 2,
+  "Reverse (generation) process");
+* attention within the block is bidirectional (What changes, section 2, property 1;
+  DiffusionGemma, "Bi-directional Attention");
+* several positions may be committed per pass (What changes, section 2, property 2);
+* block decoding: a 256-token canvas is denoised in parallel, finished canvases are
+  appended to the KV cache, prefill is causal and denoising bidirectional (What
+  changes, section 4.2 "Block decoding"; section 4.1 Block Diffusion);
+* at most 48 denoising steps, about 12 with adaptive stopping (What changes,
+  section 4.2 "Few steps"; Distributed, canvas paragraph);
+* commit by confidence threshold (What changes, section 5 "Quality vs steps");
+* mask-to-token decoding: committed tokens are not revised (What changes,
+  section 4.3, M2T versus T2T);
+* a mixture-of-experts backbone (DiffusionGemma, "Memory Optimization"; What
+  changes, section 4.2).
+
+Readings where the pages are silent (all listed in the design notes):
+
+1. pre-norm blocks: x += Attn(RMSNorm(x)); x += FFN(RMSNorm(x)); no other extras;
+2. RMSNorm with eps 1e-6, gains from the weights (ones);
+3. RoPE, theta 1e4, rotate-half pairs (i, i + hd/2), absolute positions: prompt
+   0..P-1, canvas P..P+C-1;
+4. attention scale 1/sqrt(hd); query head h reads KV head floor(h * Hkv / H);
+5. router in fp32 on the un-rounded normalised activations, no bias; top-k by logit
+   with ties to the lower expert index; gate = softmax over the k selected logits;
+   expert = Wd (silu(Wg y) * (Wu y)); dense FFN = the same with one expert, gate 1;
+6. append = one more bidirectional pass over the finished canvas, whose K/V go to
+   the cache;
+7. [MASK] = vocab - 1, excluded from argmax and from the softmax sum;
+8. confidence = max softmax probability = 1 / sum_v exp(l_v - max); argmax ties go to
+   the lowest token id;
+9. commit: top-k: the min(k, R) most confident masked positions, ties to the lower
+   position; threshold: every masked position with conf > tau, and at least
+   n_min = max(1, ceil(R / (S_max - s))) of the most confident ones so that the
+   canvas completes within the step budget;
+10. precision: GEMM operands are bf16 ("bf16 operands, fp32 accumulation"); the
+   oracle accumulates in fp64 and rounds to bf16 exactly where a bf16 operand is
+   formed (normalised activations, Q/K/V after RoPE and the KV cache, attention
+   output, SwiGLU output); the residual stream, router and softmax statistics stay
+   in high precision; router logits and LM-head logits are rounded to fp32 before
+   the top-k / argmax decision, and conf is rounded to fp32 before commit ranking.
+
+Parity pins (tests/test_oracle_pins.py): attention against brute force and closed
+forms; RoPE relative-position invariance; KV-cache pass equal to an uncached
+block-causal sequence forward; MoE top-k against brute force over all subsets and
+the k = E / E = 1 reductions; LM-head confidence against a zero-gain closed form and
+log-sum-exp; commit schedule and sampler invariants. Values produced for random
+weights beyond those properties are "parity unpinned": no page prints a worked
+example.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Dict, List, Optional
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------------------
+# precision helpers
+
+def bf16(x) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), returned as float64."""
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    r = ((u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)) << np.uint64(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def f32(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# layer pieces
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """y = x / sqrt(mean(x^2) + eps) * g over the last axis (reading 2)."""
+    x = np.asarray(x, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * np.asarray(g, dtype=np.float64)
+
+
+def rope_cos_sin(positions: np.ndarray, head_dim: int, theta: float):
+    """cos/sin of pos * theta^(-2i/hd), i < hd/2 (reading 3)."""
+    half = head_dim // 2
+    inv = theta ** (-2.0 * np.arange(half, dtype=np.float64) / head_dim)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def apply_rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotate-half RoPE on x [T][heads][hd] with cos/sin [T][hd/2]."""
+    half = x.shape[-1] // 2
+    a, b = x[..., :half], x[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+              allowed: Optional[np.ndarray] = None) -> np.ndarray:
+    """softmax(q k^T / sqrt(hd)) v per query head; GQA by floor(h * Hkv / H) (reading 4).
+
+    q [Tq][H][hd], k/v [Tk][Hkv][hd]; allowed [Tq][Tk] (None = every key visible,
+    the bidirectional canvas case). Three-pass softmax: max, sum of exponentials,
+    normalise.
+    """
+    Tq, H, hd = q.shape
+    Hkv = k.shape[1]
+    out = np.zeros((Tq, H, v.shape[2]), dtype=np.float64)
+    scale = 1.0 / math.sqrt(hd)
+    for h in range(H):
+        g = (h * Hkv) // H
+        s = (q[:, h, :] @ k[:, g, :].T) * scale
+        if allowed is not None:
+            s = np.where(allowed, s, -np.inf)
+        m = np.max(s, axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = np.sum(e, axis=1, keepdims=True)
+        out[:, h, :] = (e / z) @ v[:, g, :]
+    return out
+
+
+def router_topk(y: np.ndarray, wr: np.ndarray, k: int):
+    """Router logits (fp32 decision), top-k experts and their gates (reading 5).
+
+    y [T][d] normalised activations (not rounded to bf16), wr [E][d].
+    Returns logits fp32-valued [T][E], idx [T][k] (descending logit, ties to the
+    lower expert), gates [T][k] = softmax of the selected logits.
+    """
+    logits = f32(np.asarray(y, np.float64) @ np.asarray(wr, np.float64).T)
+    T, E = logits.shape
+    # stable sort on -logit keeps the lower index first among equal logits
+    order = np.argsort(-logits, axis=1, kind="stable")
+    idx = order[:, :k]
+    sel = np.take_along_axis(logits, idx, axis=1)
+    ex = np.exp(sel - sel[:, :1])
+    gates = ex / np.sum(ex, axis=1, keepdims=True)
+    return logits, idx.astype(np.int64), gates
+
+
+def swiglu_expert(yb: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
+    """Wd (silu(Wg y) * (Wu y)); the SwiGLU product is a bf16 operand of the down GEMM."""
+    g = yb @ np.asarray(wg, np.float64).T
+    u = yb @ np.asarray(wu, np.float64).T
+    h = bf16(g / (1.0 + np.exp(-g)) * u)
+    return h @ np.asarray(wd, np.float64).T
+
+
+def moe_ffn(y: np.ndarray, experts, wr: Optional[np.ndarray], k: int):
+    """Mixture-of-experts FFN: sum_j gate_j * expert_{idx_j}(bf16(y)).
+
+    experts: list of (wg, wu, wd); wr None means the dense FFN (one expert, gate 1).
+    Returns (delta [T][d], logits or None, idx [T][k], gates [T][k]).
+    """
+    T = y.shape[0]
+    yb = bf16(y)
+    if wr is None:
+        logits = None
+        idx = np.zeros((T, 1), dtype=np.int64)
+        gates = np.ones((T, 1), dtype=np.float64)
+    else:
+        logits, idx, gates = router_topk(y, wr, k)
+    out = np.zeros((T, experts[0][2].shape[0]), dtype=np.float64)
+    for e in range(len(experts)):
+        tok, slot = np.nonzero(idx == e)
+        if tok.size == 0:
+            continue
+        o = swiglu_expert(yb[tok], *experts[e])
+        np.add.at(out, tok, gates[tok, slot][:, None] * o)
+    return out, logits, idx, gates
+
+
+def lm_head_conf(x: np.ndarray, final_norm: np.ndarray, head: np.ndarray, mask_id: int,
+                 eps: float, return_logits: bool = False):
+    """Per row: argmax token and conf = max softmax probability, [MASK] excluded (readings 7, 8)."""
+    yb = bf16(rmsnorm(x, final_norm, eps))
+    logits = f32(yb @ np.asarray(head, np.float64).T)
+    logits[:, mask_id] = -np.inf
+    m = np.max(logits, axis=1)
+    arg = np.argmax(logits, axis=1)          # first maximum = lowest token id
+    z = np.sum(np.exp(logits - m[:, None]), axis=1)
+    conf = np.asarray(1.0 / z, dtype=np.float32)
+    if return_logits:
+        return conf, arg.astype(np.int64), logits
+    return conf, arg.astype(np.int64)
+
+
+# --------------------------------------------------------------------------------------
+# sampler (commit)
+
+@dataclass(frozen=True)
+class Policy:
+    kind: str = "topk"       # "topk" or "threshold"
+    k: int = 1
+    tau: float = 0.9
+    floor: bool = True
+
+
+def commit_count(R: int, n_above: int, policy: Policy, step: int, s_max: int) -> int:
+    """How many masked positions step `step` commits (reading 9)."""
+    if policy.kind == "topk":
+        n = policy.k
+    else:
+        n = n_above
+        if policy.floor:
+            left = s_max - step
+            n_min = R if left <= 0 else max(1, -(-R // left))
+            n = max(n, n_min)
+    return max(0, min(n, R))
+
+
+def commit_select(conf: np.ndarray, mask: np.ndarray, policy: Policy, step: int,
+                  s_max: int) -> np.ndarray:
+    """Boolean [C]: the positions committed this step.
+
+    The n most confident masked positions (fp32 conf, ties to the lower position),
+    n from commit_count; for the threshold policy every masked position above tau
+    is among them.
+    """
+    conf32 = np.asarray(conf, dtype=np.float32)
+    masked = np.nonzero(np.asarray(mask, dtype=bool))[0]
+    R = masked.size
+    n_above = int(np.sum(conf32[masked] > np.float32(policy.tau))) if policy.kind != "topk" else 0
+    n = commit_count(R, n_above, policy, step, s_max)
+    order = masked[np.lexsort((masked, -conf32[masked].astype(np.float64)))]
+    sel = np.zeros(np.asarray(mask).shape[0], dtype=bool)
+    sel[order[:n]] = True
+    return sel
+
+
+# --------------------------------------------------------------------------------------
+# the model
+
+class _Request:
+    def __init__(self, n_layers: int):
+        self.k = [None] * n_layers      # per layer [P][Hkv][hd] (bf16 values)
+        self.v = [None] * n_layers
+        self.P = 0
+
+
+class OracleModel:
+    """The denoiser over named weights (float32 arrays, e.g. from synth.gen_weights)."""
+
+    def __init__(self, cfg, weights: Dict[str, np.ndarray]):
+        self.cfg = cfg
+        c = cfg
+        # every matrix is a bf16 operand (reading 10); norm gains stay as given
+        self.emb = bf16(weights["emb"])
+        self.layers = []
+        for l in range(c.n_layers):
+            p = f"layers.{l}."
+            lw = {
+                "attn_norm": np.asarray(weights[p + "attn_norm"], np.float64),
+                "wq": bf16(weights[p + "wq"]),
+                "wk": bf16(weights[p + "wk"]),
+                "wv": bf16(weights[p + "wv"]),
+                "wo": bf16(weights[p + "wo"]),
+                "ffn_norm": np.asarray(weights[p + "ffn_norm"], np.float64),
+            }
+            if c.dense:
+                lw["wr"] = None
+                lw["experts"] = [(bf16(weights[p + "wg"]), bf16(weights[p + "wu"]),
+                                  bf16(weights[p + "wd"]))]
+            else:
+                lw["wr"] = bf16(weights[p + "wr"])
+                lw["experts"] = [(bf16(weights[p + f"experts.{e}.wg"]),
+                                  bf16(weights[p + f"experts.{e}.wu"]),
+                                  bf16(weights[p + f"experts.{e}.wd"]))
+                                 for e in range(c.n_experts)]
+            self.layers.append(lw)
+        self.final_norm = np.asarray(weights["final_norm"], np.float64)
+        self.head = bf16(weights["head"])
+        self.requests: Dict[int, _Request] = {}
+
+    # ---- one transformer layer -------------------------------------------------------
+    def layer(self, l: int, x: np.ndarray, positions: np.ndarray, k_prev, v_prev,
+              allowed: Optional[np.ndarray], rec: Optional[dict] = None):
+        """x [T][d] -> x', plus the layer's new K/V [T][Hkv][hd] (bf16 values)."""
+        c, lw = self.cfg, self.layers[l]
+        T = x.shape[0]
+        y = bf16(rmsnorm(x, lw["attn_norm"], c.rms_eps))
+        q = (y @ lw["wq"].T).reshape(T, c.n_heads, c.head_dim)
+        k = (y @ lw["wk"].T).reshape(T, c.n_kv_heads, c.head_dim)
+        v = (y @ lw["wv"].T).reshape(T, c.n_kv_heads, c.head_dim)
+        cos, sin = rope_cos_sin(positions, c.head_dim, c.rope_theta)
+        q = bf16(apply_rope(q, cos, sin))
+        k = bf16(apply_rope(k, cos, sin))
+        v = bf16(v)
+        if k_prev is not None and k_prev.shape[0] > 0:
+            kk = np.concatenate([k_prev, k], axis=0)
+            vv = np.concatenate([v_prev, v], axis=0)
+        else:
+            kk, vv = k, v
+        o = bf16(attention(q, kk, vv, allowed)).reshape(T, c.q_dim)
+        x = x + o @ lw["wo"].T
+        y2 = rmsnorm(x, lw["ffn_norm"], c.rms_eps)
+        delta, logits, idx, gates = moe_ffn(y2, lw["experts"], lw["wr"], c.top_k)
+        x = x + delta
+        if rec is not None:
+            rec.setdefault("router_logits", []).append(logits)
+            rec.setdefault("topk_idx", []).append(idx)
+            rec.setdefault("gates", []).append(gates)
+            rec.setdefault("x", []).append(x.copy())
+        return x, k, v
+
+    # ---- request lifecycle ------------------------------------------------------------
+    def reset(self, req: int = 0):
+        self.requests[req] = _Request(self.cfg.n_layers)
+
+    def prefill(self, req: int, prompt: np.ndarray):
+        """Causal forward over the prompt; its K/V fill the cache at 0..n-1."""
+        c = self.cfg
+        prompt = np.asarray(prompt, dtype=np.int64)
+        n = prompt.size
+        st = _Request(c.n_layers)
+        x = self.emb[prompt].copy()
+        pos = np.arange(n)
+        allowed = pos[None, :] <= pos[:, None]
+        for l in range(c.n_layers):
+            x, k, v = self.layer(l, x, pos, None, None, allowed)
+            st.k[l], st.v[l] = k, v
+        st.P = n
+        self.requests[req] = st
+
+    def _canvas_forward(self, req: int, canvas: np.ndarray, mask: np.ndarray,
+                        rec: Optional[dict] = None):
+        c = self.cfg
+        st = self.requests[req]
+        tokens = np.where(np.asarray(mask, bool), c.mask_id, np.asarray(canvas, np.int64))
+        x = self.emb[tokens].copy()
+        C = tokens.size
+        pos = st.P + np.arange(C)
+        new_k, new_v = [], []
+        for l in range(c.n_layers):
+            x, k, v = self.layer(l, x, pos, st.k[l], st.v[l], None, rec)
+            new_k.append(k)
+            new_v.append(v)
+        return x, new_k, new_v
+
+    def denoise_pass(self, req: int, canvas: np.ndarray, mask: np.ndarray,
+                     rec: Optional[dict] = None):
+        """One pass: conf [C] (fp32) and argmax [C] for every canvas position."""
+        x, _, _ = self._canvas_forward(req, canvas, mask, rec)
+        out = lm_head_conf(x, self.final_norm, self.head, self.cfg.mask_id, self.cfg.rms_eps,
+                           return_logits=rec is not None)
+        if rec is not None:
+            conf, arg, logits = out
+            srt = np.sort(logits, axis=1)
+            rec["logit_margin"] = srt[:, -1] - srt[:, -2]
+            rec["final_x"] = x
+            return conf, arg
+        return out
+
+    def append(self, req: int, canvas: np.ndarray):
+        """Bidirectional pass over the finished canvas; its K/V join the cache (reading 6)."""
+        st = self.requests[req]
+        C = np.asarray(canvas).size
+        _, ks, vs = self._canvas_forward(req, canvas, np.zeros(C, dtype=bool))
+        for l in range(self.cfg.n_layers):
+            st.k[l] = np.concatenate([st.k[l], ks[l]], axis=0) if st.k[l] is not None else ks[l]
+            st.v[l] = np.concatenate([st.v[l], vs[l]], axis=0) if st.v[l] is not None else vs[l]
+        st.P += C
+
+    def generate_block(self, req: int, policy: Policy, s_max: int, trace: bool = False):
+        """Denoise one all-[MASK] canvas until no position is masked or S_max passes ran.
+
+        Returns (canvas, steps, trace list). Each trace entry holds the pass's input
+        canvas/mask, conf, argmax, the commit set and the masked count after it.
+        """
+        c = self.cfg
+        C = c.canvas
+        canvas = np.full(C, c.mask_id, dtype=np.int64)
+        mask = np.ones(C, dtype=bool)
+        steps, tr = 0, []
+        for s in range(s_max):
+            if not mask.any():
+                break
+            rec = {} if trace else None
+            conf, arg = self.denoise_pass(req, canvas, mask, rec)
+            sel = commit_select(conf, mask, policy, s, s_max)
+            if trace:
+                tr.append(dict(step=s, canvas=canvas.copy(), mask=mask.copy(), conf=conf,
+                               argmax=arg, commit=sel.copy(), rec=rec))
+            canvas = np.where(sel, arg, canvas)
+            mask = mask & ~sel
+            steps += 1
+            if trace:
+                tr[-1]["remaining"] = int(mask.sum())
+        return canvas, steps, tr
+
+
+def sequence_forward(model: OracleModel, tokens: np.ndarray, allowed: np.ndarray) -> np.ndarray:
+    """Uncached forward over a whole sequence with an explicit attention mask.
+
+    Positions are 0..n-1. Used only to pin the cached path: a canvas pass over a
+    cached prefix must equal this forward with a block-causal mask.
+    """
+    c = model.cfg
+    tokens = np.asarray(tokens, dtype=np.int64)
+    x = model.emb[tokens].copy()
+    pos = np.arange(tokens.size)
+    for l in range(c.n_layers):
+        x, _, _ = model.layer(l, x, pos, None, None, allowed)
+    return x

@@ -1,0 +1,341 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+No page prints a worked numeric example for this method, so every pin is a closed
+form, an invariant, a brute-force count on tiny inputs or a reduction to a library
+routine. A plausible mistake in the oracle (a dropped scale, a wrong GQA index, a
+swapped RoPE sign, a wrong tie rule, a missing mask) fails at least one of them;
+the planted-mistake tests at the end check that.
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+from oracle import (OracleModel, Policy, apply_rope, attention, commit_count, commit_select,
+                    lm_head_conf, moe_ffn, rope_cos_sin, router_topk, sequence_forward,
+                    swiglu_expert)
+from synth import gen_weights, prompt_tokens, uniform_f32
+from synth.configs import ModelConfig
+
+MICRO = ModelConfig("micro", n_layers=2, d_model=64, n_heads=4, n_kv_heads=2, head_dim=16,
+                    n_experts=4, top_k=2, ffn_dim=64, vocab=64, canvas=8,
+                    weight_dtype="bf16", weight_seed=77)
+MICRO_DENSE = ModelConfig("micro-dense", n_layers=2, d_model=64, n_heads=4, n_kv_heads=4,
+                          head_dim=16, n_experts=0, top_k=1, ffn_dim=64, vocab=64, canvas=8,
+                          weight_dtype="f32", weight_seed=78)
+
+
+def rnd(shape, tid, seed=5, scale=1.0):
+    n = int(np.prod(shape))
+    return (uniform_f32(seed, tid, n).astype(np.float64) * scale).reshape(shape)
+
+
+# ---------------------------------------------------------------- attention
+
+def brute_attention(q, k, v, allowed=None):
+    Tq, H, hd = q.shape
+    Tk, Hkv, _ = k.shape
+    out = np.zeros_like(q)
+    for i in range(Tq):
+        for h in range(H):
+            g = h // (H // Hkv)
+            w = []
+            for j in range(Tk):
+                if allowed is None or allowed[i, j]:
+                    w.append(math.exp(sum(q[i, h, t] * k[j, g, t] for t in range(hd)) / math.sqrt(hd)))
+                else:
+                    w.append(0.0)
+            z = sum(w)
+            for t in range(hd):
+                out[i, h, t] = sum(w[j] * v[j, g, t] for j in range(Tk)) / z
+    return out
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (4, 1)])
+def test_attention_matches_brute_force(H, Hkv):
+    q, k, v = rnd((5, H, 8), 1), rnd((7, Hkv, 8), 2), rnd((7, Hkv, 8), 3)
+    assert np.allclose(attention(q, k, v), brute_attention(q, k, v), rtol=1e-12, atol=1e-12)
+    causal = np.arange(7)[None, :] <= np.arange(5)[:, None] + 2
+    assert np.allclose(attention(q, k, v, causal), brute_attention(q, k, v, causal),
+                       rtol=1e-12, atol=1e-12)
+
+
+def test_attention_closed_forms():
+    q, v = rnd((3, 2, 8), 4), rnd((6, 1, 8), 5)
+    k_same = np.repeat(rnd((1, 1, 8), 6), 6, axis=0)
+    # identical keys: uniform weights, output = mean of V for every head
+    o = attention(q, k_same, v)
+    assert np.allclose(o, np.broadcast_to(v.mean(axis=0)[None], o.shape), atol=1e-14)
+    # one dominant score selects that value row
+    k = np.zeros((6, 1, 8))
+    k[4, 0, :] = 1e3 * np.sign(q[0, 0, :])
+    o = attention(q[:1, :1], k, v)
+    assert np.allclose(o[0, 0], v[4, 0], atol=1e-12)
+    # a causal row 0 sees only key 0
+    causal = np.arange(6)[None, :] <= np.arange(3)[:, None]
+    o = attention(q, rnd((6, 1, 8), 7), v, causal)
+    assert np.allclose(o[0, :, :], np.broadcast_to(v[0, 0], (2, 8)), atol=1e-14)
+
+
+def test_attention_gqa_head_mapping():
+    # Hkv = 2 with H = 4: heads 0,1 read KV head 0; heads 2,3 read KV head 1
+    q = np.zeros((1, 4, 4))
+    k = np.zeros((2, 2, 4))
+    v = np.zeros((2, 2, 4))
+    v[:, 0, :], v[:, 1, :] = 1.0, 2.0
+    o = attention(q, k, v)
+    assert np.allclose(o[0, :, 0], [1, 1, 2, 2])
+
+
+# ---------------------------------------------------------------- RoPE
+
+def test_rope_relative_position_and_norm():
+    hd = 16
+    q, k = rnd((1, 1, hd), 8), rnd((1, 1, hd), 9)
+    dots = []
+    for shift in (0, 5, 123, 4096):
+        cq, sq = rope_cos_sin(np.array([7 + shift]), hd, 1e4)
+        ck, sk = rope_cos_sin(np.array([3 + shift]), hd, 1e4)
+        dots.append(float(np.sum(apply_rope(q, cq, sq) * apply_rope(k, ck, sk))))
+    assert np.allclose(dots, dots[0], rtol=1e-10)
+    c, s = rope_cos_sin(np.array([11]), hd, 1e4)
+    assert np.isclose(np.linalg.norm(apply_rope(q, c, s)), np.linalg.norm(q), rtol=1e-12)
+    c0, s0 = rope_cos_sin(np.array([0]), hd, 1e4)
+    assert np.allclose(apply_rope(q, c0, s0), q)
+
+
+def test_rope_pairing_special_case():
+    # hd = 4, theta = 1e4: frequencies 1 and 1e-2; pair (0, 2) turns by pos radians
+    x = np.array([[[1.0, 0.0, 0.0, 0.0]]])
+    c, s = rope_cos_sin(np.array([1]), 4, 1e4)
+    assert np.allclose(apply_rope(x, c, s)[0, 0], [math.cos(1), 0, math.sin(1), 0])
+    y = np.array([[[0.0, 1.0, 0.0, 0.0]]])
+    assert np.allclose(apply_rope(y, c, s)[0, 0], [0, math.cos(0.01), 0, math.sin(0.01)])
+
+
+# ---------------------------------------------------------------- MoE
+
+def test_router_topk_brute_force_subsets():
+    E, k = 8, 2
+    y, wr = rnd((40, 16), 10), rnd((E, 16), 11)
+    logits, idx, gates = router_topk(y, wr, k)
+    for t in range(40):
+        best = max(itertools.combinations(range(E), k),
+                   key=lambda sub: (sum(logits[t, list(sub)]), [-e for e in sub]))
+        assert set(idx[t]) == set(best)
+        assert logits[t, idx[t, 0]] >= logits[t, idx[t, 1]]
+        sel = logits[t, idx[t]]
+        assert np.allclose(gates[t], scipy.special.softmax(sel))
+
+
+def test_router_ties_prefer_lower_expert():
+    y = np.ones((1, 4))
+    wr = np.array([[0.0] * 4, [1.0] * 4, [1.0] * 4, [1.0] * 4])
+    _, idx, gates = router_topk(y, wr, 2)
+    assert list(idx[0]) == [1, 2]
+    assert np.allclose(gates[0], [0.5, 0.5])
+
+
+def test_moe_reductions():
+    d, F, T = 16, 32, 6
+    y = rnd((T, d), 12)
+    experts = [(rnd((F, d), 20 + e, scale=0.3), rnd((F, d), 30 + e, scale=0.3),
+                rnd((d, F), 40 + e, scale=0.3)) for e in range(3)]
+    wr = rnd((3, d), 13)
+    # k = E: the softmax-weighted mixture of every expert
+    out, logits, idx, gates = moe_ffn(y, experts, wr, 3)
+    yb = oracle.bf16(y)
+    p = scipy.special.softmax(logits, axis=1)
+    ref = sum(p[:, e:e + 1] * swiglu_expert(yb, *experts[e]) for e in range(3))
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # dense = one expert with gate 1
+    dense, _, _, g = moe_ffn(y, experts[:1], None, 1)
+    assert np.allclose(g, 1.0)
+    wg, wu, wd = experts[0]
+    h = yb @ wg.T
+    ref_dense = oracle.bf16(h * scipy.special.expit(h) * (yb @ wu.T)) @ wd.T
+    assert np.allclose(dense, ref_dense, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- LM head and confidence
+
+def test_lm_head_zero_gain_closed_form():
+    V, d = 64, 16
+    x, head = rnd((5, d), 14), rnd((V, d), 15)
+    conf, arg = lm_head_conf(x, np.zeros(d), head, V - 1, 1e-6)
+    assert np.all(conf == np.float32(1.0 / (V - 1)))
+    assert np.all(arg == 0)
+
+
+def test_lm_head_logsumexp_and_mask_exclusion():
+    V, d = 64, 16
+    x, head = rnd((7, d), 16), rnd((V, d), 17)
+    head[V - 1] = 50.0 * oracle.bf16(x[0]) / np.linalg.norm(x[0])   # [MASK] would win row 0
+    head = oracle.bf16(head)
+    conf, arg, logits = lm_head_conf(x, np.ones(d), head, V - 1, 1e-6, return_logits=True)
+    y = oracle.bf16(oracle.rmsnorm(x, np.ones(d), 1e-6))
+    raw = (y @ head.T)[:, : V - 1]
+    assert np.all(arg != V - 1)
+    assert np.array_equal(arg, np.argmax(raw, axis=1))
+    lse = scipy.special.logsumexp(raw, axis=1)
+    assert np.allclose(conf, np.exp(raw.max(axis=1) - lse), rtol=1e-6)
+
+
+# ---------------------------------------------------------------- commit / sampler
+
+def test_threshold_floor_schedule_twelve_steps():
+    # flat confidences never pass tau = 0.9: the floor alone sets the schedule
+    R, sched = 256, []
+    for s in range(12):
+        n = commit_count(R, 0, Policy("threshold", tau=0.9, floor=True), s, 12)
+        sched.append(n)
+        R -= n
+    assert sched == [22] * 4 + [21] * 8 and R == 0
+
+
+def test_threshold_commits_everything_above_tau():
+    conf = np.array([0.95, 0.2, 0.91, 0.99, 0.5, 0.92], np.float32)
+    mask = np.array([1, 1, 1, 0, 1, 1], bool)
+    sel = commit_select(conf, mask, Policy("threshold", tau=0.9, floor=True), 0, 48)
+    assert list(np.nonzero(sel)[0]) == [0, 2, 5]          # 0.99 is already committed
+    sel = commit_select(conf, mask, Policy("threshold", tau=0.99, floor=False), 0, 48)
+    assert not sel.any()
+    # floor at the last step commits every remaining position
+    sel = commit_select(conf, mask, Policy("threshold", tau=0.99, floor=True), 47, 48)
+    assert sel.sum() == mask.sum()
+
+
+def test_topk_ties_go_to_lower_position():
+    conf = np.array([0.5, 0.7, 0.5, 0.7, 0.5], np.float32)
+    mask = np.ones(5, bool)
+    sel = commit_select(conf, mask, Policy("topk", k=3), 0, 8)
+    assert list(np.nonzero(sel)[0]) == [0, 1, 3]
+
+
+@pytest.mark.parametrize("cfg,policy,s_max", [
+    (MICRO, Policy("topk", k=2), 4),
+    (MICRO_DENSE, Policy("topk", k=1), 8),
+    (MICRO, Policy("threshold", tau=0.9, floor=True), 3),
+])
+def test_generate_block_invariants(cfg, policy, s_max):
+    m = OracleModel(cfg, gen_weights(cfg))
+    m.prefill(0, prompt_tokens(cfg.vocab, 2000, 12))
+    canvas, steps, tr = m.generate_block(0, policy, s_max, trace=True)
+    C = cfg.canvas
+    assert tr[0]["mask"].all()                                   # all-[MASK] start
+    assert steps <= s_max and not np.any(canvas == cfg.mask_id)  # full within budget
+    prev_R = C
+    for e in tr:
+        R = int(e["mask"].sum())
+        assert R == prev_R
+        committed = ~e["mask"]
+        nxt = np.where(e["commit"], e["argmax"], e["canvas"])
+        assert np.array_equal(nxt[committed], e["canvas"][committed])   # M2T: never revised
+        assert not np.any(e["commit"] & committed)
+        if policy.kind == "topk":
+            assert e["commit"].sum() == min(policy.k, R)
+        assert e["remaining"] < R                                # strictly decreasing
+        prev_R = e["remaining"]
+    assert prev_R == 0
+    if policy.kind == "topk":
+        assert steps == C // policy.k
+
+
+# ---------------------------------------------------------------- KV cache
+
+def block_causal(lengths):
+    n = sum(lengths)
+    blk = np.concatenate([[i] * L for i, L in enumerate(lengths)])
+    pos = np.arange(n)
+    allowed = blk[None, :] <= blk[:, None]
+    # block 0 (the prompt) is causal inside itself
+    allowed &= ~((blk[:, None] == 0) & (blk[None, :] == 0) & (pos[None, :] > pos[:, None]))
+    return allowed
+
+
+@pytest.mark.parametrize("cfg", [MICRO, MICRO_DENSE])
+def test_cached_passes_equal_block_causal_sequence(cfg):
+    m = OracleModel(cfg, gen_weights(cfg))
+    P, C = 10, cfg.canvas
+    prompt = prompt_tokens(cfg.vocab, 2001, P)
+    m.prefill(0, prompt)
+    c1 = prompt_tokens(cfg.vocab, 2002, C)
+    mask = np.zeros(C, bool)
+    mask[::3] = True
+    x_cached, _, _ = m._canvas_forward(0, c1, mask)
+    seq = np.concatenate([prompt, np.where(mask, cfg.mask_id, c1)])
+    x_full = sequence_forward(m, seq, block_causal([P, C]))
+    assert np.allclose(x_cached, x_full[P:], rtol=1e-9, atol=1e-9)
+    # append c1, then a second canvas sees [prompt | c1 | c2]
+    k0 = m.requests[0].k[0].copy()
+    m.append(0, c1)
+    assert m.requests[0].P == P + C
+    assert np.array_equal(m.requests[0].k[0][:P], k0)        # prefix K/V untouched
+    c2 = prompt_tokens(cfg.vocab, 2003, C)
+    x2, _, _ = m._canvas_forward(0, c2, np.ones(C, bool))
+    seq2 = np.concatenate([prompt, c1, np.full(C, cfg.mask_id)])
+    x2_full = sequence_forward(m, seq2, block_causal([P, C, C]))
+    assert np.allclose(x2, x2_full[P + C:], rtol=1e-9, atol=1e-9)
+
+
+def test_prefix_kv_is_causal():
+    cfg = MICRO
+    m = OracleModel(cfg, gen_weights(cfg))
+    p = prompt_tokens(cfg.vocab, 2004, 12)
+    m.prefill(0, p)
+    k_a = [a.copy() for a in m.requests[0].k]
+    p2 = p.copy()
+    p2[8:] = (p2[8:] + 1) % (cfg.vocab - 1)
+    m.prefill(1, p2)
+    for l in range(cfg.n_layers):
+        assert np.array_equal(k_a[l][:8], m.requests[1].k[l][:8])
+        assert not np.array_equal(k_a[l][8:], m.requests[1].k[l][8:])
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Each pin above must fail when a plausible mistake is planted in the oracle."""
+    q, k, v = rnd((5, 4, 8), 1), rnd((7, 2, 8), 2), rnd((7, 2, 8), 3)
+    good = brute_attention(q, k, v)
+
+    # dropped 1/sqrt(hd) scale
+    def attn_noscale(q, k, v, allowed=None):
+        return oracle.model.attention(q * math.sqrt(q.shape[2]), k, v, allowed)
+    assert not np.allclose(attn_noscale(q, k, v), good, atol=1e-6)
+
+    # wrong GQA mapping (h % Hkv instead of floor(h * Hkv / H))
+    def attn_mod(q, k, v):
+        out = np.zeros_like(q)
+        for h in range(q.shape[1]):
+            s = q[:, h] @ k[:, h % k.shape[1]].T / math.sqrt(q.shape[2])
+            p = scipy.special.softmax(s, axis=1)
+            out[:, h] = p @ v[:, h % k.shape[1]]
+        return out
+    assert not np.allclose(attn_mod(q, k, v), good, atol=1e-6)
+
+    # swapped RoPE sign breaks the pairing special case
+    x = np.array([[[1.0, 0.0, 0.0, 0.0]]])
+    c, s = rope_cos_sin(np.array([1]), 4, 1e4)
+    half = 2
+    bad = np.concatenate([x[..., :half] * c[:, None] + x[..., half:] * s[:, None],
+                          x[..., half:] * c[:, None] - x[..., :half] * s[:, None]], axis=-1)
+    assert not np.allclose(bad[0, 0], [math.cos(1), 0, math.sin(1), 0])
+
+    # [MASK] not excluded: the mask-exclusion pin would see argmax == V-1
+    V, d = 64, 16
+    xx, head = rnd((7, d), 16), rnd((V, d), 17)
+    head[V - 1] = 50.0 * oracle.bf16(xx[0]) / np.linalg.norm(xx[0])
+    monkeypatch.setattr(np, "argmax", np.argmax)
+    y = oracle.bf16(oracle.rmsnorm(xx, np.ones(d), 1e-6))
+    assert np.argmax(y @ oracle.bf16(head).T, axis=1)[0] == V - 1
+
+    # floor rule off: the 12-step schedule would not finish the canvas
+    R = 256
+    for s in range(12):
+        R -= commit_count(R, 0, Policy("threshold", tau=0.9, floor=False), s, 12)
+    assert R == 256
