@@ -1,0 +1,1061 @@
+// libdllm: the masked block-diffusion denoiser behind a C ABI (include/dllm.h).
+//
+// Per canvas pass (What changes, section 2 "Reverse (generation) process"; section 4.2
+// "Block decoding"), for T = B * C canvas tokens:
+//   embed -> per layer [ RMSNorm -> QKV GEMM (+RoPE, K/V into the cache at P..P+C-1)
+//   -> bidirectional attention over [prefix | canvas] -> O GEMM (+residual) -> RMSNorm
+//   -> fp32 router + top-k -> permute -> gather -> grouped gate/up GEMM (+SwiGLU)
+//   -> grouped down GEMM -> combine (+residual) ] -> final RMSNorm -> LM-head GEMM with
+//   fused max / argmax / sum-exp -> merge -> commit.
+// The same layer pipeline runs the causal prefill and the append pass. A canvas pass
+// is captured once per batch size into a CUDA graph and replayed every step.
+
+#include "dllm.h"
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace dllm;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][cols] matrix, box = 64 columns x box_rows,
+// 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
+bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (cols * 2) % 16 || box_rows == 0 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMoeBN[4] = {32, 64, 128, 256};
+
+struct LayerW {
+  float* attn_norm = nullptr;
+  float* ffn_norm = nullptr;
+  bf16_t* wqkv = nullptr;   // [(H + 2 Hkv) * hd][d]: Q heads, K heads, V heads
+  bf16_t* wo = nullptr;     // [d][H * hd]
+  bf16_t* wr = nullptr;     // [E][d]
+  bf16_t* wgu = nullptr;    // [E][2F][d]: per 128-row block, 64 gate rows then the 64 matching up rows
+  bf16_t* wd = nullptr;     // [E][d][F]
+  CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd;
+};
+
+struct Graph {
+  cudaGraphExec_t exec = nullptr;
+  long long kernels = 0;
+};
+
+}  // namespace
+
+struct dllm_handle {
+  dllm_config c{};
+  cudaStream_t st = nullptr;
+  bool own_stream = false;
+  std::string err;
+  int E = 1, k = 1;          // experts and top-k as run (dense: 1, 1)
+  bool dense = true;
+  int qkv_heads = 0;
+  long long launches = 0;
+  std::vector<void*> allocs;
+
+  bf16_t* emb = nullptr;
+  bf16_t* head = nullptr;
+  float* final_norm = nullptr;
+  CUtensorMap tm_head;
+  std::vector<LayerW> L;
+  float* rope_cos = nullptr;
+  float* rope_sin = nullptr;
+
+  bf16_t* kcache = nullptr;
+  bf16_t* vcache = nullptr;
+  size_t kv_layer = 0;      // elements per layer: max_batch * Hkv * max_ctx * hd
+
+  int T_max = 0, N_max = 0, T_canvas_max = 0;
+  float* x = nullptr;
+  bf16_t* y = nullptr;
+  float* rstd = nullptr;
+  bf16_t* q = nullptr;
+  bf16_t* ao = nullptr;
+  float* apart = nullptr;
+  float* alse = nullptr;
+  float* rlogits = nullptr;
+  int32_t* tk_idx = nullptr;
+  float* tk_w = nullptr;
+  int32_t* offsets = nullptr;
+  int32_t* slot_of = nullptr;
+  int32_t* row_token = nullptr;
+  bf16_t* xg = nullptr;
+  bf16_t* hbuf = nullptr;
+  float* obuf = nullptr;
+  float* lm_m = nullptr;
+  float* lm_s = nullptr;
+  int32_t* lm_i = nullptr;
+  float* conf = nullptr;
+  int32_t* argmax = nullptr;
+  // lo halves of the activation operands carried as (hi, lo) bf16 pairs
+  bf16_t* y_lo = nullptr;
+  bf16_t* ao_lo = nullptr;
+  bf16_t* xg_lo = nullptr;
+  bf16_t* hbuf_lo = nullptr;
+  CUtensorMap tm_y, tm_ao, tm_xg[4], tm_h[4];
+  CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
+
+  std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
+  int32_t* d_P = nullptr;    // [max_batch]
+  int32_t* d_slot = nullptr; // [max_batch] = 0..max_batch-1
+  int32_t* d_pre_pos = nullptr;   // [1] = 0
+  int32_t* d_pre_slot = nullptr;  // [1]
+  int32_t* d_tokens = nullptr;    // prompt staging [T_max]
+  int32_t* canvas = nullptr;      // [max_batch][C]
+  uint8_t* mask = nullptr;
+  int32_t* d_step = nullptr;
+  int32_t* d_remaining = nullptr;
+  PolicyDev* d_policy = nullptr;
+  int32_t* h_remaining = nullptr; // pinned [max_batch]
+  int* d_err = nullptr;
+  int last_B = 0;
+
+  bool debug = false;
+  float* dbg_logits = nullptr;   // [L][T_canvas_max][E]
+  int32_t* dbg_idx = nullptr;    // [L][T_canvas_max][k]
+  float* dbg_x = nullptr;        // [T_canvas_max][d]
+  float* dbg_xl = nullptr;       // [L][T_canvas_max][d] residual after each layer
+  int32_t* dbg_force = nullptr;  // [L][T_canvas_max][k] experts to use instead of the router's
+  bool force_routing = false;
+
+  std::map<int, Graph> graphs;   // key: B * 2 + mode
+};
+
+namespace {
+
+int fail(dllm_handle* h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  return code;
+}
+
+int cuda_fail(dllm_handle* h, cudaError_t e, const char* what) {
+  return fail(h, DLLM_E_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(call)                                              \
+  do {                                                        \
+    cudaError_t e_ = (call);                                  \
+    if (e_ != cudaSuccess) return cuda_fail(h, e_, #call);    \
+  } while (0)
+
+long g_alloc_count = 0;
+
+// Device allocation tracked by the handle. DLLM_FAULT_ALLOC_AT=n makes the n-th
+// allocation of the process fail (host-side fault injection for the error paths).
+template <class T>
+int dalloc(dllm_handle* h, T** p, size_t count) {
+  *p = nullptr;
+  ++g_alloc_count;
+  const char* f = getenv("DLLM_FAULT_ALLOC_AT");
+  if (f && atol(f) == g_alloc_count) return fail(h, DLLM_E_OOM, "injected allocation failure");
+  size_t bytes = count * sizeof(T);
+  if (bytes == 0) bytes = 16;
+  void* v = nullptr;
+  cudaError_t e = cudaMalloc(&v, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(h, DLLM_E_OOM, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  h->allocs.push_back(v);
+  *p = reinterpret_cast<T*>(v);
+  return DLLM_OK;
+}
+
+#define DA(ptr, n)                           \
+  do {                                       \
+    int r_ = dalloc(h, &(ptr), (size_t)(n)); \
+    if (r_) return r_;                       \
+  } while (0)
+
+int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
+
+int moe_bn_index(int N, int E) {
+  // token chunk width: the smallest width holding 1.5x the mean tokens per expert
+  const double mean = (double)N / (double)E;
+  for (int i = 0; i < 3; ++i)
+    if (mean * 1.5 <= kMoeBN[i]) return i;
+  return 3;
+}
+
+int attn_splits(const dllm_handle* h, int B) {
+  const int qblocks = ceil_div(h->c.canvas, 64);
+  const int ctas = qblocks * h->c.n_heads * B;
+  int s = ceil_div(2 * 148, ctas);
+  if (s < 1) s = 1;
+  if (s > 16) s = 16;
+  return s;
+}
+
+int attn_split_keys(const dllm_handle* h, int splits) {
+  return ceil_div(ceil_div(h->c.max_ctx, splits), 64) * 64;
+}
+
+// ------------------------------------------------------------------ GEMM launch helpers
+
+template <int BN, int STAGES, int ACC, int SPLIT, class Sched, class Epi>
+cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const CUtensorMap& tb, int kblocks,
+                        int a_first, const Sched& s, const Epi& e, const CUtensorMap* ta2 = nullptr,
+                        const CUtensorMap* tb2 = nullptr) {
+  auto kern = gemm_tc_kernel<BN, STAGES, ACC, SPLIT, Sched, Epi>;
+  constexpr int smem = GemmSmem<BN, STAGES, SPLIT, Epi>::kTotal;
+  static_assert(smem <= 232448, "shared memory per CTA");
+  cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (r != cudaSuccess) return r;
+  kern<<<grid, 192, smem, h->st>>>(ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e, h->d_err);
+  h->launches++;
+  return cudaGetLastError();
+}
+
+template <int HD>
+cudaError_t qkv_gemm_hd(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, int T, const int* pos0,
+                        const int* slot, int tok_per_req) {
+  const auto& c = h->c;
+  EpiQKV<HD> e{h->q, kc, vc, h->rope_cos, h->rope_sin, pos0, slot, tok_per_req, c.n_heads, c.n_kv_heads, c.max_ctx};
+  const int mt = ceil_div(T, 128);
+  DenseSched s{T, mt, HD};
+  dim3 grid(mt * h->qkv_heads);
+  constexpr int STAGES = HD > 128 ? 4 : 5;
+  return launch_gemm<HD, STAGES, 1, kSplitA>(h, grid, h->tm_y, L.tm_wqkv, c.d_model / 64, 0, s, e, &h->tm_y_lo);
+}
+
+cudaError_t qkv_gemm(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, int T, const int* pos0,
+                     const int* slot, int tok_per_req) {
+  if (h->c.head_dim == 176) return qkv_gemm_hd<176>(h, L, kc, vc, T, pos0, slot, tok_per_req);
+  return qkv_gemm_hd<64>(h, L, kc, vc, T, pos0, slot, tok_per_req);
+}
+
+template <int HD, int BK>
+cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
+                         const int* slot, int causal, int splits, int split_keys) {
+  const auto& c = h->c;
+  AttnParams p;
+  p.q = h->q;
+  p.kc = kc;
+  p.vc = vc;
+  p.out = h->ao;
+  p.out_lo = h->ao_lo;
+  p.part_o = h->apart;
+  p.part_lse = h->alse;
+  p.pos0 = pos0;
+  p.slot = slot;
+  p.tok_per_req = tok_per_req;
+  p.T = T;
+  p.H = c.n_heads;
+  p.Hkv = c.n_kv_heads;
+  p.max_ctx = c.max_ctx;
+  p.causal = causal;
+  p.n_splits = splits;
+  p.split_keys = split_keys;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  constexpr int smem = AttnSmem<HD, BK>::kTotal;
+  cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_kernel<HD, BK>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (r != cudaSuccess) return r;
+  dim3 grid(ceil_div(tok_per_req, 64), c.n_heads, nreq * splits);
+  attn_kernel<HD, BK><<<grid, 128, smem, h->st>>>(p);
+  h->launches++;
+  if (splits > 1) {
+    attn_merge_kernel<HD><<<ceil_div((long)T * c.n_heads * 32, 256), 256, 0, h->st>>>(p);
+    h->launches++;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
+                      const int* slot, int causal, int splits, int split_keys) {
+  if (h->c.head_dim == 176)
+    return attention_hd<176, 32>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
+  return attention_hd<64, 64>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
+}
+
+template <int BN>
+cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi) {
+  const auto& c = h->c;
+  const int F = c.ffn_dim, d = c.d_model;
+  constexpr int STAGES = BN <= 64 ? 6 : BN <= 128 ? 4 : 2;
+  {
+    GroupedSched s{h->offsets, 2 * F, BN};
+    EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
+    cudaError_t r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(2 * F / 128, h->E), L.tm_wgu, h->tm_xg[bi], d / 64,
+                                                        1, s, e, nullptr, &h->tm_xg_lo[bi]);
+    if (r != cudaSuccess) return r;
+  }
+  GroupedSched s{h->offsets, d, BN};
+  EpiDown<BN> e{h->obuf, d};
+  return launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(d / 128, h->E), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
+                                             &h->tm_h_lo[bi]);
+}
+
+cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N) {
+  const int bi = moe_bn_index(N, h->E);
+  switch (bi) {
+    case 0: return moe_gemms_bn<32>(h, L, bi);
+    case 1: return moe_gemms_bn<64>(h, L, bi);
+    case 2: return moe_gemms_bn<128>(h, L, bi);
+    default: return moe_gemms_bn<256>(h, L, bi);
+  }
+}
+
+// ------------------------------------------------------------------ the pass
+
+int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0, const int* slot, int causal,
+               int splits, int split_keys, bool record) {
+  const auto& c = h->c;
+  const int d = c.d_model;
+  const int N = T * h->k;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const LayerW& L = h->L[l];
+    bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
+    bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
+    rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
+    h->launches++;
+    CK(qkv_gemm(h, L, kc, vc, T, pos0, slot, tok_per_req));
+    CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys));
+    {
+      EpiResidual<64> e{h->x, d};
+      const int mt = ceil_div(T, 128);
+      DenseSched s{T, mt, 64};
+      CK((launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, c.n_heads * c.head_dim / 64, 0,
+                                         s, e, &h->tm_ao_lo)));
+    }
+    rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
+    h->launches++;
+    if (!h->dense) {
+      router_kernel<<<ceil_div(T, kRouterTok), 256, kRouterTok * d * sizeof(float), h->st>>>(
+          h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits);
+      topk_kernel<<<ceil_div((long)T * 32, 256), 256, 0, h->st>>>(h->rlogits, T, h->E, h->k, h->tk_idx, h->tk_w);
+      h->launches += 2;
+      if (record) {
+        CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
+                           sizeof(float) * T * h->E, cudaMemcpyDeviceToDevice, h->st));
+        CK(cudaMemcpyAsync(h->dbg_idx + (size_t)l * h->T_canvas_max * h->k, h->tk_idx, sizeof(int32_t) * T * h->k,
+                           cudaMemcpyDeviceToDevice, h->st));
+        if (h->force_routing) {
+          force_route_kernel<<<ceil_div(T, 128), 128, 0, h->st>>>(
+              h->rlogits, h->dbg_force + (size_t)l * h->T_canvas_max * h->k, T, h->E, h->k, h->tk_idx, h->tk_w);
+          h->launches++;
+        }
+      }
+    } else {
+      dense_route_kernel<<<ceil_div(T, 256), 256, 0, h->st>>>(T, h->tk_idx, h->tk_w);
+      h->launches++;
+    }
+    permute_kernel<<<1, 1024, 34 * h->E * sizeof(int), h->st>>>(h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
+                                                               h->row_token);
+    gather_rows_kernel<<<N, 128, 0, h->st>>>(h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo);
+    h->launches += 2;
+    CK(moe_gemms(h, L, N));
+    combine_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d);
+    h->launches++;
+    if (record)
+      CK(cudaMemcpyAsync(h->dbg_xl + (size_t)l * h->T_canvas_max * d, h->x, sizeof(float) * T * d,
+                         cudaMemcpyDeviceToDevice, h->st));
+  }
+  CK(cudaGetLastError());
+  return DLLM_OK;
+}
+
+// mode 0: denoise pass + commit; mode 1: append pass (K/V of the finished canvas kept).
+int run_canvas_pass(dllm_handle* h, int B, int mode) {
+  const auto& c = h->c;
+  const int C = c.canvas, T = B * C, d = c.d_model;
+  const int splits = attn_splits(h, B);
+  embed_kernel<<<T, 128, 0, h->st>>>(h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x);
+  h->launches++;
+  int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0);
+  if (r) return r;
+  if (mode == 1) return DLLM_OK;
+  if (h->debug) CK(cudaMemcpyAsync(h->dbg_x, h->x, sizeof(float) * T * d, cudaMemcpyDeviceToDevice, h->st));
+  rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, h->final_norm, d, c.rms_eps, h->y, h->y_lo, nullptr);
+  h->launches++;
+  const int nvt = c.vocab / 256;
+  {
+    EpiLMHead<256> e{h->lm_m, h->lm_s, h->lm_i, nvt, c.mask_id};
+    const int mt = ceil_div(T, 128);
+    DenseSched s{T, mt, 256};
+    CK((launch_gemm<256, 3, 1, kSplitA>(h, dim3(mt * nvt), h->tm_y, h->tm_head, d / 64, 0, s, e, &h->tm_y_lo)));
+  }
+  lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, h->st>>>(h->lm_m, h->lm_s, h->lm_i, T, nvt, h->conf,
+                                                                  h->argmax);
+  const int threads = ceil_div(C, 32) * 32;
+  commit_kernel<<<B, threads, C * (sizeof(float) + 1), h->st>>>(h->canvas, h->mask, h->conf, h->argmax, C,
+                                                                 h->d_policy, h->d_step, h->d_remaining, nullptr,
+                                                                 nullptr);
+  h->launches += 2;
+  CK(cudaGetLastError());
+  return DLLM_OK;
+}
+
+int replay_pass(dllm_handle* h, int B, int mode) {
+  const int key = B * 2 + mode;
+  auto it = h->graphs.find(key);
+  if (it == h->graphs.end()) {
+    // eager run first: loads modules and sets kernel attributes outside the capture
+    long long before = h->launches;
+    int r = run_canvas_pass(h, B, mode);
+    if (r) return r;
+    if (getenv("DLLM_NO_GRAPH")) return DLLM_OK;
+    cudaGraph_t g;
+    CK(cudaStreamBeginCapture(h->st, cudaStreamCaptureModeRelaxed));
+    before = h->launches;
+    r = run_canvas_pass(h, B, mode);
+    cudaError_t e = cudaStreamEndCapture(h->st, &g);
+    if (r) return r;
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamEndCapture");
+    Graph gr;
+    gr.kernels = h->launches - before;
+    h->launches = before;
+    e = cudaGraphInstantiate(&gr.exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaGraphInstantiate");
+    h->graphs[key] = gr;
+    return DLLM_OK;   // the eager run above did this call's work; the capture only recorded it
+  }
+  CK(cudaGraphLaunch(it->second.exec, h->st));
+  h->launches += it->second.kernels;
+  return DLLM_OK;
+}
+
+int check_requests(dllm_handle* h, int B) {
+  if (B < 1 || B > h->c.max_batch) return fail(h, DLLM_E_INVAL, "req_count out of range");
+  for (int b = 0; b < B; ++b) {
+    if (h->P[b] < 0) return fail(h, DLLM_E_STATE, "request slot " + std::to_string(b) + " has no prefill");
+    if (h->P[b] + h->c.canvas > h->c.max_ctx) return fail(h, DLLM_E_CTX_FULL, "KV cache full");
+  }
+  return DLLM_OK;
+}
+
+int upload_P(dllm_handle* h) {
+  std::vector<int32_t> v(h->P.size());
+  for (size_t i = 0; i < v.size(); ++i) v[i] = h->P[i] < 0 ? 0 : h->P[i];
+  CK(cudaMemcpyAsync(h->d_P, v.data(), sizeof(int32_t) * v.size(), cudaMemcpyHostToDevice, h->st));
+  CK(cudaStreamSynchronize(h->st));   // v is a local: keep the copy inside its lifetime
+  return DLLM_OK;
+}
+
+int upload_policy(dllm_handle* h, const dllm_policy* p, int max_steps) {
+  if (!p) return fail(h, DLLM_E_INVAL, "policy is NULL");
+  if (p->kind != DLLM_POLICY_TOPK && p->kind != DLLM_POLICY_THRESHOLD) return fail(h, DLLM_E_INVAL, "policy kind");
+  if (p->kind == DLLM_POLICY_TOPK && p->k < 1) return fail(h, DLLM_E_INVAL, "top-k policy needs k >= 1");
+  if (max_steps < 1) return fail(h, DLLM_E_INVAL, "max_steps < 1");
+  PolicyDev pd{p->kind == DLLM_POLICY_TOPK ? 0 : 1, p->k, p->tau, p->floor, max_steps};
+  CK(cudaMemcpyAsync(h->d_policy, &pd, sizeof(pd), cudaMemcpyHostToDevice, h->st));
+  CK(cudaStreamSynchronize(h->st));
+  return DLLM_OK;
+}
+
+int check_device_error(dllm_handle* h) {
+  int e = 0;
+  CK(cudaMemcpy(&e, h->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (e != 0) {
+    CK(cudaMemset(h->d_err, 0, sizeof(int)));
+    return fail(h, DLLM_E_TIMEOUT, "a kernel gave up a bounded wait (code " + std::to_string(e) + ")");
+  }
+  return DLLM_OK;
+}
+
+void drop_graphs(dllm_handle* h) {
+  for (auto& kv : h->graphs)
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+  h->graphs.clear();
+}
+
+int validate(const dllm_config* c, std::string* why) {
+  auto bad = [&](const char* m) { *why = m; return DLLM_E_INVAL; };
+  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256) return bad("d_model must be a multiple of 256");
+  if (c->head_dim != 64 && c->head_dim != 176) return bad("head_dim must be 64 or 176");
+  if (c->n_heads < 1 || c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads) return bad("n_heads % n_kv_heads != 0");
+  if ((c->n_heads * c->head_dim) % 64) return bad("n_heads * head_dim must be a multiple of 64");
+  if (c->ffn_dim < 64 || c->ffn_dim % 64) return bad("ffn_dim must be a multiple of 64");
+  if (c->vocab < 256 || c->vocab % 256) return bad("vocab must be a multiple of 256");
+  if (c->mask_id != c->vocab - 1) return bad("mask_id must be vocab - 1");
+  if (c->n_experts < 0 || c->n_experts > 256) return bad("n_experts in [0, 256]");
+  if (c->n_experts == 0 && c->top_k != 1) return bad("dense FFN needs top_k = 1");
+  if (c->n_experts > 0 && (c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts)) return bad("top_k in [1, 8]");
+  if (c->canvas < 1 || c->canvas > 1024) return bad("canvas in [1, 1024]");
+  if (c->max_batch < 1 || c->max_ctx < c->canvas + 1) return bad("max_batch >= 1 and max_ctx > canvas");
+  if (c->weight_dtype != DLLM_WEIGHTS_F32 && c->weight_dtype != DLLM_WEIGHTS_BF16) return bad("weight_dtype");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------ weight loading
+
+struct BlobReader {
+  const uint8_t* base;
+  size_t size;
+  size_t off = 0;
+  int esize;
+  bool on_device;
+  const uint8_t* next(size_t numel, bool* ok) {
+    size_t o = off;
+    size_t bytes = numel * esize;
+    if (o + bytes > size) {
+      *ok = false;
+      return nullptr;
+    }
+    off = (o + bytes + 255) / 256 * 256;
+    return base + o;
+  }
+};
+
+// Copies one blob tensor into bf16 rows of dst (see pack_rows_kernel for the row map).
+int pack_tensor(dllm_handle* h, BlobReader& br, void* staging, bf16_t* dst, long rows, int cols, long group,
+                long gstride, long goff) {
+  bool ok = true;
+  const uint8_t* src = br.next((size_t)rows * cols, &ok);
+  if (!ok) return fail(h, DLLM_E_INVAL, "weight blob too small");
+  const void* s = src;
+  if (!br.on_device) {
+    CK(cudaMemcpyAsync(staging, src, (size_t)rows * cols * br.esize, cudaMemcpyHostToDevice, h->st));
+    s = staging;
+  }
+  pack_rows_kernel<<<1184, 256, 0, h->st>>>(dst, s, br.esize == 4, rows, cols, group, gstride, goff);
+  CK(cudaGetLastError());
+  if (!br.on_device) CK(cudaStreamSynchronize(h->st));
+  return DLLM_OK;
+}
+
+int load_f32(dllm_handle* h, BlobReader& br, void* staging, float* dst, long n) {
+  bool ok = true;
+  const uint8_t* src = br.next((size_t)n, &ok);
+  if (!ok) return fail(h, DLLM_E_INVAL, "weight blob too small");
+  const void* s = src;
+  if (!br.on_device) {
+    CK(cudaMemcpyAsync(staging, src, (size_t)n * br.esize, cudaMemcpyHostToDevice, h->st));
+    s = staging;
+  }
+  to_f32_kernel<<<64, 256, 0, h->st>>>(dst, s, br.esize == 4, n);
+  CK(cudaGetLastError());
+  if (!br.on_device) CK(cudaStreamSynchronize(h->st));
+  return DLLM_OK;
+}
+
+int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on_device) {
+  const dllm_config& c = h->c;
+  const int d = c.d_model, F = c.ffn_dim, hd = c.head_dim, H = c.n_heads, Hkv = c.n_kv_heads, V = c.vocab;
+  h->dense = c.n_experts == 0;
+  h->E = h->dense ? 1 : c.n_experts;
+  h->k = h->dense ? 1 : c.top_k;
+  h->qkv_heads = H + 2 * Hkv;
+  const long qd = (long)H * hd, kvd = (long)Hkv * hd;
+
+  // ---- weights
+  DA(h->emb, (size_t)V * d);
+  DA(h->head, (size_t)V * d);
+  DA(h->final_norm, d);
+  h->L.resize(c.n_layers);
+  for (auto& L : h->L) {
+    DA(L.attn_norm, d);
+    DA(L.ffn_norm, d);
+    DA(L.wqkv, (size_t)(qd + 2 * kvd) * d);
+    DA(L.wo, (size_t)d * qd);
+    if (!h->dense) DA(L.wr, (size_t)h->E * d);
+    DA(L.wgu, (size_t)h->E * 2 * F * d);
+    DA(L.wd, (size_t)h->E * d * F);
+  }
+  uint8_t* staging = nullptr;
+  if (!on_device) {
+    const size_t sizes[] = {(size_t)V * d, (size_t)qd * d, (size_t)kvd * d, (size_t)F * d, (size_t)h->E * d};
+    size_t mx = 0;   // elements of the largest blob tensor
+    for (size_t s : sizes) mx = s > mx ? s : mx;
+    DA(staging, mx * 4 + 256);   // bytes, fp32 worst case
+  }
+  BlobReader br{reinterpret_cast<const uint8_t*>(weights), weight_bytes, 0,
+                c.weight_dtype == DLLM_WEIGHTS_F32 ? 4 : 2, on_device != 0};
+  const long BIG = 1L << 40;
+  int r;
+  if ((r = pack_tensor(h, br, staging, h->emb, V, d, BIG, 0, 0))) return r;
+  for (int l = 0; l < c.n_layers; ++l) {
+    LayerW& L = h->L[l];
+    if ((r = load_f32(h, br, staging, L.attn_norm, d))) return r;
+    if ((r = pack_tensor(h, br, staging, L.wqkv, qd, d, BIG, 0, 0))) return r;
+    if ((r = pack_tensor(h, br, staging, L.wqkv, kvd, d, BIG, 0, qd))) return r;
+    if ((r = pack_tensor(h, br, staging, L.wqkv, kvd, d, BIG, 0, qd + kvd))) return r;
+    if ((r = pack_tensor(h, br, staging, L.wo, d, (int)qd, BIG, 0, 0))) return r;
+    if ((r = load_f32(h, br, staging, L.ffn_norm, d))) return r;
+    if (!h->dense)
+      if ((r = pack_tensor(h, br, staging, L.wr, h->E, d, BIG, 0, 0))) return r;
+    for (int e = 0; e < h->E; ++e) {
+      const long gu0 = (long)e * 2 * F;
+      if ((r = pack_tensor(h, br, staging, L.wgu, F, d, 64, 128, gu0))) return r;        // gate rows
+      if ((r = pack_tensor(h, br, staging, L.wgu, F, d, 64, 128, gu0 + 64))) return r;   // up rows
+      if ((r = pack_tensor(h, br, staging, L.wd, d, F, BIG, 0, (long)e * d))) return r;
+    }
+  }
+  if ((r = load_f32(h, br, staging, h->final_norm, d))) return r;
+  if ((r = pack_tensor(h, br, staging, h->head, V, d, BIG, 0, 0))) return r;
+
+  // ---- RoPE tables (fp64 on the host, stored fp32)
+  const int half = hd / 2;
+  {
+    std::vector<float> cs((size_t)c.max_ctx * half), sn((size_t)c.max_ctx * half);
+    for (int p = 0; p < c.max_ctx; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double inv = pow((double)c.rope_theta, -2.0 * i / hd);
+        const double a = (double)p * inv;
+        cs[(size_t)p * half + i] = (float)cos(a);
+        sn[(size_t)p * half + i] = (float)sin(a);
+      }
+    DA(h->rope_cos, cs.size());
+    DA(h->rope_sin, sn.size());
+    CK(cudaMemcpy(h->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(h->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice));
+  }
+
+  // ---- KV cache
+  h->kv_layer = (size_t)c.max_batch * Hkv * c.max_ctx * hd;
+  DA(h->kcache, h->kv_layer * c.n_layers);
+  DA(h->vcache, h->kv_layer * c.n_layers);
+  CK(cudaMemsetAsync(h->kcache, 0, h->kv_layer * c.n_layers * 2, h->st));
+  CK(cudaMemsetAsync(h->vcache, 0, h->kv_layer * c.n_layers * 2, h->st));
+
+  // ---- activations
+  h->T_canvas_max = c.max_batch * c.canvas;
+  h->T_max = h->T_canvas_max > c.max_ctx - c.canvas ? h->T_canvas_max : c.max_ctx - c.canvas;
+  h->N_max = h->T_max * h->k;
+  const int T = h->T_max, N = h->N_max;
+  DA(h->x, (size_t)T * d);
+  DA(h->y, (size_t)T * d);
+  DA(h->y_lo, (size_t)T * d);
+  DA(h->rstd, T);
+  DA(h->q, (size_t)T * qd);
+  DA(h->ao, (size_t)T * qd);
+  DA(h->ao_lo, (size_t)T * qd);
+  {
+    size_t mx = 0;
+    for (int B = 1; B <= c.max_batch; ++B) {
+      const int s = attn_splits(h, B);
+      if (s > 1 && (size_t)s * B > mx) mx = (size_t)s * B;
+    }
+    DA(h->apart, mx * c.canvas * qd + 1);
+    DA(h->alse, mx * c.canvas * H + 1);
+  }
+  DA(h->rlogits, (size_t)T * h->E);
+  DA(h->tk_idx, (size_t)N);
+  DA(h->tk_w, (size_t)N);
+  DA(h->offsets, h->E + 1);
+  DA(h->slot_of, (size_t)N);
+  DA(h->row_token, (size_t)N);
+  DA(h->xg, (size_t)N * d);
+  DA(h->xg_lo, (size_t)N * d);
+  DA(h->hbuf, (size_t)N * F);
+  DA(h->hbuf_lo, (size_t)N * F);
+  DA(h->obuf, (size_t)N * d);
+  const int nvt = V / 256;
+  DA(h->lm_m, (size_t)h->T_canvas_max * nvt);
+  DA(h->lm_s, (size_t)h->T_canvas_max * nvt);
+  DA(h->lm_i, (size_t)h->T_canvas_max * nvt);
+  DA(h->conf, h->T_canvas_max);
+  DA(h->argmax, h->T_canvas_max);
+  CK(cudaMemsetAsync(h->xg, 0, (size_t)N * d * 2, h->st));
+  CK(cudaMemsetAsync(h->xg_lo, 0, (size_t)N * d * 2, h->st));
+  CK(cudaMemsetAsync(h->hbuf, 0, (size_t)N * F * 2, h->st));
+  CK(cudaMemsetAsync(h->hbuf_lo, 0, (size_t)N * F * 2, h->st));
+
+  // ---- request state
+  h->P.assign(c.max_batch, -1);
+  DA(h->d_P, c.max_batch);
+  DA(h->d_slot, c.max_batch);
+  DA(h->d_pre_pos, 1);
+  DA(h->d_pre_slot, 1);
+  DA(h->d_tokens, T);
+  DA(h->canvas, h->T_canvas_max);
+  DA(h->mask, h->T_canvas_max);
+  DA(h->d_step, c.max_batch);
+  DA(h->d_remaining, c.max_batch);
+  DA(h->d_policy, 1);
+  DA(h->d_err, 1);
+  {
+    std::vector<int32_t> s(c.max_batch);
+    for (int i = 0; i < c.max_batch; ++i) s[i] = i;
+    CK(cudaMemcpy(h->d_slot, s.data(), sizeof(int32_t) * s.size(), cudaMemcpyHostToDevice));
+  }
+  CK(cudaMemset(h->d_pre_pos, 0, sizeof(int32_t)));
+  CK(cudaMemset(h->d_err, 0, sizeof(int)));
+  CK(cudaMemset(h->d_P, 0, sizeof(int32_t) * c.max_batch));
+  CK(cudaMallocHost(&h->h_remaining, sizeof(int32_t) * c.max_batch));
+
+  // ---- tensor maps
+  bool ok = true;
+  ok &= make_tmap(&h->tm_y, h->y, T, d, 128);
+  ok &= make_tmap(&h->tm_y_lo, h->y_lo, T, d, 128);
+  ok &= make_tmap(&h->tm_ao, h->ao, T, qd, 128);
+  ok &= make_tmap(&h->tm_ao_lo, h->ao_lo, T, qd, 128);
+  ok &= make_tmap(&h->tm_head, h->head, V, d, 256);
+  for (int i = 0; i < 4; ++i) {
+    ok &= make_tmap(&h->tm_xg[i], h->xg, N, d, kMoeBN[i]);
+    ok &= make_tmap(&h->tm_xg_lo[i], h->xg_lo, N, d, kMoeBN[i]);
+    ok &= make_tmap(&h->tm_h[i], h->hbuf, N, F, kMoeBN[i]);
+    ok &= make_tmap(&h->tm_h_lo[i], h->hbuf_lo, N, F, kMoeBN[i]);
+  }
+  for (auto& L : h->L) {
+    ok &= make_tmap(&L.tm_wqkv, L.wqkv, qd + 2 * kvd, d, hd);
+    ok &= make_tmap(&L.tm_wo, L.wo, d, qd, 64);
+    ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
+    ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);
+  }
+  if (!ok) return fail(h, DLLM_E_CUDA, "cuTensorMapEncodeTiled failed");
+  CK(cudaFuncSetAttribute(reinterpret_cast<const void*>(router_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          kRouterTok * d * (int)sizeof(float)));
+  CK(cudaStreamSynchronize(h->st));
+  return DLLM_OK;
+}
+
+void free_all(dllm_handle* h) {
+  drop_graphs(h);
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+  if (h->h_remaining) cudaFreeHost(h->h_remaining);
+  h->h_remaining = nullptr;
+  if (h->own_stream && h->st) cudaStreamDestroy(h->st);
+  h->st = nullptr;
+}
+
+int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool prompt_on_host) {
+  const auto& c = h->c;
+  if (req < 0 || req >= c.max_batch) return fail(h, DLLM_E_INVAL, "req out of range");
+  if (n < 1 || !prompt) return fail(h, DLLM_E_INVAL, "empty prompt");
+  if (n + c.canvas > c.max_ctx) return fail(h, DLLM_E_CTX_FULL, "prompt + canvas exceeds max_ctx");
+  CK(cudaMemcpyAsync(h->d_tokens, prompt, sizeof(int32_t) * n,
+                     prompt_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, h->st));
+  const int32_t s = req;
+  CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
+  embed_kernel<<<n, 128, 0, h->st>>>(h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x);
+  h->launches++;
+  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false);
+  if (r) return r;
+  h->P[req] = n;
+  return upload_P(h);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+int dllm_create(const dllm_config* cfg, const void* weights, size_t weight_bytes, int weights_on_device,
+                void* cuda_stream, dllm_handle** out) {
+  if (!out) return DLLM_E_INVAL;
+  *out = nullptr;
+  if (!cfg || !weights) return DLLM_E_INVAL;
+  std::string why;
+  if (validate(cfg, &why)) {
+    fprintf(stderr, "dllm_create: %s\n", why.c_str());
+    return DLLM_E_INVAL;
+  }
+  dllm_handle* h = new dllm_handle();
+  h->c = *cfg;
+  if (cuda_stream) {
+    h->st = reinterpret_cast<cudaStream_t>(cuda_stream);
+  } else {
+    if (cudaStreamCreateWithFlags(&h->st, cudaStreamNonBlocking) != cudaSuccess) {
+      delete h;
+      return DLLM_E_CUDA;
+    }
+    h->own_stream = true;
+  }
+  int r = create_impl(h, weights, weight_bytes, weights_on_device);
+  if (r) {
+    fprintf(stderr, "dllm_create: %s\n", h->err.c_str());
+    free_all(h);
+    delete h;
+    return r;
+  }
+  *out = h;
+  return DLLM_OK;
+}
+
+int dllm_prefill(dllm_handle* h, int req, const int32_t* prompt, int n) {
+  if (!h) return DLLM_E_INVAL;
+  return prefill_impl(h, req, prompt, n, false);
+}
+
+int dllm_denoise_step(dllm_handle* h, int req_count, int32_t* canvas, uint8_t* mask, const dllm_policy* policy,
+                      int step, int max_steps, float* conf_out, int32_t* argmax_out, int32_t* remaining_out) {
+  if (!h) return DLLM_E_INVAL;
+  if (!canvas || !mask) return fail(h, DLLM_E_INVAL, "canvas/mask NULL");
+  int r = check_requests(h, req_count);
+  if (r) return r;
+  if (step < 0) return fail(h, DLLM_E_INVAL, "step < 0");
+  if ((r = upload_policy(h, policy, max_steps))) return r;
+  const int C = h->c.canvas, B = req_count;
+  std::vector<int32_t> steps(B, step);
+  CK(cudaMemcpyAsync(h->d_step, steps.data(), sizeof(int32_t) * B, cudaMemcpyHostToDevice, h->st));
+  CK(cudaMemcpyAsync(h->canvas, canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  CK(cudaMemcpyAsync(h->mask, mask, (size_t)B * C, cudaMemcpyDeviceToDevice, h->st));
+  CK(cudaStreamSynchronize(h->st));   // `steps` is a local
+  if ((r = replay_pass(h, B, 0))) return r;
+  h->last_B = B;
+  CK(cudaMemcpyAsync(canvas, h->canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  CK(cudaMemcpyAsync(mask, h->mask, (size_t)B * C, cudaMemcpyDeviceToDevice, h->st));
+  if (conf_out) CK(cudaMemcpyAsync(conf_out, h->conf, sizeof(float) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  if (argmax_out)
+    CK(cudaMemcpyAsync(argmax_out, h->argmax, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  if (remaining_out)
+    CK(cudaMemcpyAsync(remaining_out, h->d_remaining, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, h->st));
+  return DLLM_OK;
+}
+
+int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm_policy* policy, int32_t* canvas_out,
+                        int* steps_taken) {
+  if (!h) return DLLM_E_INVAL;
+  int r = check_requests(h, req_count);
+  if (r) return r;
+  if ((r = upload_policy(h, policy, max_steps))) return r;
+  const int C = h->c.canvas, B = req_count;
+  canvas_init_kernel<<<ceil_div((long)B * C, 256), 256, 0, h->st>>>(h->canvas, h->mask, B * C, h->c.mask_id,
+                                                                    h->d_step, B);
+  h->launches++;
+  std::vector<int> done_at(B, -1);
+  int s = 0;
+  bool all_done = false;
+  for (; s < max_steps && !all_done; ++s) {
+    if ((r = replay_pass(h, B, 0))) return r;
+    CK(cudaMemcpyAsync(h->h_remaining, h->d_remaining, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, h->st));
+    CK(cudaStreamSynchronize(h->st));
+    all_done = true;
+    for (int b = 0; b < B; ++b) {
+      if (h->h_remaining[b] == 0 && done_at[b] < 0) done_at[b] = s + 1;
+      if (h->h_remaining[b] != 0) all_done = false;
+    }
+  }
+  h->last_B = B;
+  if ((r = check_device_error(h))) return r;
+  if (steps_taken)
+    for (int b = 0; b < B; ++b) steps_taken[b] = done_at[b] < 0 ? s : done_at[b];
+  if (canvas_out)
+    CK(cudaMemcpyAsync(canvas_out, h->canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  if (!all_done) return fail(h, DLLM_E_BUDGET, "step budget spent with masked positions left");
+  return DLLM_OK;
+}
+
+int dllm_append_kv(dllm_handle* h, int req_count, const int32_t* canvas) {
+  if (!h) return DLLM_E_INVAL;
+  int r = check_requests(h, req_count);
+  if (r) return r;
+  const int C = h->c.canvas, B = req_count;
+  if (canvas) CK(cudaMemcpyAsync(h->canvas, canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
+  if ((r = replay_pass(h, B, 1))) return r;
+  for (int b = 0; b < B; ++b) h->P[b] += C;
+  return upload_P(h);
+}
+
+int dllm_generate(dllm_handle* h, int req_count, const int32_t* prompts, int n_prompt, int n_canvases, int max_steps,
+                  const dllm_policy* policy, int32_t* tokens_out, int* steps_out) {
+  if (!h) return DLLM_E_INVAL;
+  if (!prompts || !tokens_out || n_canvases < 1) return fail(h, DLLM_E_INVAL, "bad arguments");
+  if (req_count < 1 || req_count > h->c.max_batch) return fail(h, DLLM_E_INVAL, "req_count out of range");
+  const int C = h->c.canvas;
+  if (n_prompt + (long)n_canvases * C + C > (long)h->c.max_ctx + C)
+    return fail(h, DLLM_E_CTX_FULL, "prompt + canvases exceed max_ctx");
+  int r;
+  for (int b = 0; b < req_count; ++b)
+    if ((r = prefill_impl(h, b, prompts + (size_t)b * n_prompt, n_prompt, true))) return r;
+  std::vector<int> steps(req_count);
+  for (int ci = 0; ci < n_canvases; ++ci) {
+    if ((r = dllm_generate_block(h, req_count, max_steps, policy, nullptr, steps.data()))) return r;
+    for (int b = 0; b < req_count; ++b) {
+      CK(cudaMemcpyAsync(tokens_out + ((size_t)b * n_canvases + ci) * C, h->canvas + (size_t)b * C,
+                         sizeof(int32_t) * C, cudaMemcpyDeviceToHost, h->st));
+      if (steps_out) steps_out[(size_t)b * n_canvases + ci] = steps[b];
+    }
+    if ((r = dllm_append_kv(h, req_count, nullptr))) return r;
+  }
+  CK(cudaStreamSynchronize(h->st));
+  return check_device_error(h);
+}
+
+int dllm_reset(dllm_handle* h, int req) {
+  if (!h) return DLLM_E_INVAL;
+  if (req < 0 || req >= h->c.max_batch) return fail(h, DLLM_E_INVAL, "req out of range");
+  h->P[req] = -1;
+  return upload_P(h);
+}
+
+int dllm_prefix_len(const dllm_handle* h, int req) {
+  if (!h || req < 0 || req >= h->c.max_batch) return DLLM_E_INVAL;
+  return h->P[req] < 0 ? 0 : h->P[req];
+}
+
+int dllm_check(dllm_handle* h) {
+  if (!h) return DLLM_E_INVAL;
+  CK(cudaStreamSynchronize(h->st));
+  CK(cudaGetLastError());
+  return check_device_error(h);
+}
+
+long long dllm_launch_count(const dllm_handle* h) { return h ? h->launches : -1; }
+
+int dllm_set_debug(dllm_handle* h, int on) {
+  if (!h) return DLLM_E_INVAL;
+  if (on && !h->dbg_x) {
+    const size_t T = h->T_canvas_max;
+    DA(h->dbg_logits, (size_t)h->c.n_layers * T * h->E);
+    DA(h->dbg_idx, (size_t)h->c.n_layers * T * h->k);
+    DA(h->dbg_x, T * h->c.d_model);
+    DA(h->dbg_xl, (size_t)h->c.n_layers * T * h->c.d_model);
+  }
+  h->debug = on != 0;
+  drop_graphs(h);
+  return DLLM_OK;
+}
+
+int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T) {
+  if (!h) return DLLM_E_INVAL;
+  if (!h->debug) return fail(h, DLLM_E_STATE, "debug is off");
+  if (h->dense) return fail(h, DLLM_E_INVAL, "dense model has no routing");
+  drop_graphs(h);
+  if (!idx) {
+    h->force_routing = false;
+    return DLLM_OK;
+  }
+  if (T < 1 || T > h->T_canvas_max) return fail(h, DLLM_E_INVAL, "T out of range");
+  if (!h->dbg_force) DA(h->dbg_force, (size_t)h->c.n_layers * h->T_canvas_max * h->k);
+  for (int l = 0; l < h->c.n_layers; ++l) {
+    for (size_t i = 0; i < (size_t)T * h->k; ++i)
+      if (idx[(size_t)l * T * h->k + i] < 0 || idx[(size_t)l * T * h->k + i] >= h->E)
+        return fail(h, DLLM_E_INVAL, "expert index out of range");
+    CK(cudaMemcpy(h->dbg_force + (size_t)l * h->T_canvas_max * h->k, idx + (size_t)l * T * h->k,
+                  sizeof(int32_t) * T * h->k, cudaMemcpyHostToDevice));
+  }
+  h->force_routing = true;
+  return DLLM_OK;
+}
+
+int dllm_debug_read(dllm_handle* h, int what, int layer, void* dst, size_t bytes) {
+  if (!h || !dst) return DLLM_E_INVAL;
+  if (!h->debug) return fail(h, DLLM_E_STATE, "debug is off");
+  const size_t T = (size_t)h->last_B * h->c.canvas;
+  const void* src = nullptr;
+  size_t need = 0;
+  if (layer < 0 || layer >= h->c.n_layers) layer = 0;
+  switch (what) {
+    case 0: src = h->dbg_x; need = T * h->c.d_model * 4; break;
+    case 1: src = h->dbg_logits + (size_t)layer * h->T_canvas_max * h->E; need = T * h->E * 4; break;
+    case 2: src = h->dbg_idx + (size_t)layer * h->T_canvas_max * h->k; need = T * h->k * 4; break;
+    case 3: src = h->conf; need = T * 4; break;
+    case 4: src = h->argmax; need = T * 4; break;
+    case 5: src = h->dbg_xl + (size_t)layer * h->T_canvas_max * h->c.d_model; need = T * h->c.d_model * 4; break;
+    case 6:   // K cache of `layer`, slot 0: [Hkv][max_ctx][hd] bf16
+      src = h->kcache + (size_t)layer * h->kv_layer;
+      need = (size_t)h->c.n_kv_heads * h->c.max_ctx * h->c.head_dim * 2;
+      break;
+    case 7:   // V cache of `layer`, slot 0
+      src = h->vcache + (size_t)layer * h->kv_layer;
+      need = (size_t)h->c.n_kv_heads * h->c.max_ctx * h->c.head_dim * 2;
+      break;
+    default: return fail(h, DLLM_E_INVAL, "unknown debug buffer");
+  }
+  if (bytes < need) return fail(h, DLLM_E_INVAL, "debug buffer too small");
+  CK(cudaStreamSynchronize(h->st));
+  CK(cudaMemcpy(dst, src, need, cudaMemcpyDeviceToHost));
+  return DLLM_OK;
+}
+
+const char* dllm_last_error(const dllm_handle* h) { return h ? h->err.c_str() : "null handle"; }
+
+void dllm_destroy(dllm_handle* h) {
+  if (!h) return;
+  if (h->st) cudaStreamSynchronize(h->st);
+  free_all(h);
+  delete h;
+}
+
+// ---------------------------------------------------------------- single-operation entry points
+
+int dllm_op_gemm_bf16(const uint16_t* A, const uint16_t* B, float* D, int M, int N, int K, void* stream) {
+  if (!A || !B || !D || M < 1 || N < 128 || N % 128 || K < 64 || K % 64) return DLLM_E_INVAL;
+  dllm_handle tmp;
+  tmp.st = reinterpret_cast<cudaStream_t>(stream);
+  dllm_handle* h = &tmp;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, A, M, K, 128) || !make_tmap(&tb, B, N, K, 128)) return DLLM_E_INVAL;
+  int* err = nullptr;
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&err), sizeof(int), tmp.st));
+  CK(cudaMemsetAsync(err, 0, sizeof(int), tmp.st));
+  tmp.d_err = err;
+  const int mt = ceil_div(M, 128);
+  DenseSched s{M, mt, 128};
+  EpiStoreF32<128> e{D, N, N};
+  cudaError_t r = launch_gemm<128, 4, 1, kSplitNone>(h, dim3(mt * (N / 128)), ta, tb, K / 64, 0, s, e);
+  cudaFreeAsync(err, tmp.st);
+  tmp.d_err = nullptr;
+  if (r != cudaSuccess) return DLLM_E_CUDA;
+  return DLLM_OK;
+}
+
+int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, int V, int mask_id, float* conf,
+                         int32_t* argmax, void* stream) {
+  if (!y || !head || !conf || !argmax || T < 1 || d < 64 || d % 64 || V < 256 || V % 256) return DLLM_E_INVAL;
+  dllm_handle tmp;
+  tmp.st = reinterpret_cast<cudaStream_t>(stream);
+  dllm_handle* h = &tmp;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, y, T, d, 128) || !make_tmap(&tb, head, V, d, 256)) return DLLM_E_INVAL;
+  const int nvt = V / 256;
+  float *pm = nullptr, *ps = nullptr;
+  int32_t* pi = nullptr;
+  int* err = nullptr;
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&pm), sizeof(float) * T * nvt, tmp.st));
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&ps), sizeof(float) * T * nvt, tmp.st));
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&pi), sizeof(int32_t) * T * nvt, tmp.st));
+  CK(cudaMallocAsync(reinterpret_cast<void**>(&err), sizeof(int), tmp.st));
+  CK(cudaMemsetAsync(err, 0, sizeof(int), tmp.st));
+  tmp.d_err = err;
+  const int mt = ceil_div(T, 128);
+  DenseSched s{T, mt, 256};
+  EpiLMHead<256> e{pm, ps, pi, nvt, mask_id};
+  cudaError_t r = launch_gemm<256, 4, 1, kSplitNone>(h, dim3(mt * nvt), ta, tb, d / 64, 0, s, e);
+  if (r == cudaSuccess) {
+    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax);
+    r = cudaGetLastError();
+  }
+  cudaFreeAsync(pm, tmp.st);
+  cudaFreeAsync(ps, tmp.st);
+  cudaFreeAsync(pi, tmp.st);
+  cudaFreeAsync(err, tmp.st);
+  tmp.d_err = nullptr;
+  return r == cudaSuccess ? DLLM_OK : DLLM_E_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,497 @@
+// Tensor-core GEMM for sm_100a: D[128 x BN] = A[128 x K] * B[BN x K]^T per tile, bf16
+// operands staged by TMA into 128-byte-swizzled shared memory, tcgen05.mma issued by one
+// thread, fp32 accumulators in TMEM, and a fused epilogue that reads TMEM row by row.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 owns the TMEM allocation
+// and lane 0 issues the MMAs; warps 2..5 run the epilogue, warp w reading TMEM lanes
+// 32*(w%4)..32*(w%4)+31 (one accumulator row per thread). Stages are handed over with
+// mbarriers (full: TMA bytes landed; empty: the MMAs reading the stage completed), the
+// accumulator with acc_full / acc_empty so that, when a CTA owns several tiles, the
+// epilogue of one overlaps the main loop of the next. Every wait is bounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace dllm {
+
+struct Tile {
+  int a_row;     // A tensor-map row of the tile's first row
+  int b_row;     // B tensor-map row of the tile's first column
+  int m_valid;   // rows of the tile inside the problem
+  int n_valid;   // columns of the tile inside the problem
+  int mt, nt;    // dense: (m tile, n tile); grouped: (m tile inside the expert, expert)
+};
+
+// One output tile per CTA over an M x N problem; m tiles vary fastest so that the CTAs
+// sharing a weight tile run close together (the second read hits L2).
+struct DenseSched {
+  int M, n_mtiles, BN;
+  DLLM_DEV int count() const { return 1; }
+  DLLM_DEV Tile tile(int) const {
+    Tile t;
+    int id = blockIdx.x;
+    t.mt = id % n_mtiles;
+    t.nt = id / n_mtiles;
+    t.a_row = t.mt * 128;
+    t.b_row = t.nt * BN;
+    t.m_valid = min(128, M - t.a_row);
+    t.n_valid = BN;
+    return t;
+  }
+};
+
+// Grouped (one GEMM per expert), operands swapped so that the expert's weight rows fill
+// the 128-row M side and its few tokens form N. CTA (blockIdx.x, blockIdx.y) = (m tile,
+// expert); its tiles are the expert's token chunks of BN rows, taken from the
+// expert-sorted token buffer between offsets[e] and offsets[e+1].
+struct GroupedSched {
+  const int* offsets;
+  int rows_per_expert;
+  int BN;
+  DLLM_DEV int count() const {
+    int e = blockIdx.y;
+    int cnt = offsets[e + 1] - offsets[e];
+    return (cnt + BN - 1) / BN;
+  }
+  DLLM_DEV Tile tile(int j) const {
+    Tile t;
+    int e = blockIdx.y;
+    int off = offsets[e];
+    int cnt = offsets[e + 1] - off;
+    t.mt = blockIdx.x;
+    t.nt = e;
+    t.a_row = e * rows_per_expert + blockIdx.x * 128;
+    t.b_row = off + j * BN;
+    t.m_valid = 128;
+    t.n_valid = min(BN, cnt - j * BN);
+    return t;
+  }
+};
+
+__host__ __device__ constexpr int tmem_cols_for(int bn) {
+  return bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
+}
+
+// Operand splitting. Weights are bf16; an activation operand can be carried as a pair
+// of bf16 tensors (hi = bf16(v), lo = bf16(v - hi)) so that products keep about 16
+// mantissa bits of the activation: every k step then issues two MMAs into the same
+// accumulator. kSplitNone: plain; kSplitA: A is a (hi, lo) pair; kSplitB: B is.
+enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
+
+template <int BN, int STAGES, int SPLIT, class Epi>
+struct GemmSmem {
+  static constexpr int kA = 128 * 64 * 2;
+  static constexpr int kB = BN * 64 * 2;
+  static constexpr int kA2 = SPLIT == kSplitA ? kA : 0;
+  static constexpr int kB2 = SPLIT == kSplitB ? kB : 0;
+  static constexpr int kStageBytes = kA + kA2 + kB + kB2;   // TMA bytes per stage
+  static constexpr int kOffA2 = STAGES * kA;
+  static constexpr int kOffB = kOffA2 + STAGES * kA2;
+  static constexpr int kOffB2 = kOffB + STAGES * kB;
+  static constexpr int kBarOff = STAGES * kStageBytes;
+  static constexpr int kEpiOff = kBarOff + 256;
+  static constexpr int kTotal = kEpiOff + Epi::kSmemBytes + 1024;   // + alignment slack
+};
+
+DLLM_DEV void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// True on every epilogue thread iff it is true on all 128 of them (named barrier 1).
+DLLM_DEV bool epi_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+template <int BN, int STAGES, int ACC_BUFS, int SPLIT, class Sched, class Epi>
+__global__ void __launch_bounds__(192, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a2,
+               const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_b2,
+               int k_blocks, int a_stream_first, Sched sched, Epi epi, int* err) {
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
+  using L = GemmSmem<BN, STAGES, SPLIT, Epi>;
+  constexpr int kCols = tmem_cols_for(BN);
+  constexpr int kTmemCols = kCols * ACC_BUFS;
+  static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sA2 = smem + L::kOffA2;
+  uint8_t* sB = smem + L::kOffB;
+  uint8_t* sB2 = smem + L::kOffB2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + ACC_BUFS;
+  uint64_t* drain = acc_empty + ACC_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* epi_smem = smem + L::kEpiOff;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < ACC_BUFS; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tma_a);
+    tma_prefetch_desc(&tma_b);
+    if (SPLIT == kSplitA) tma_prefetch_desc(&tma_a2);
+    if (SPLIT == kSplitB) tma_prefetch_desc(&tma_b2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = sched.count();
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    const uint64_t pol_first = policy_evict_first();
+    const uint64_t pol_last = policy_evict_last();
+    const uint64_t pol_a = a_stream_first ? pol_first : pol_last;
+    const uint64_t pol_b = a_stream_first ? pol_last : pol_first;
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const Tile t = sched.tile(j);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+        tma_load_2d(sA + stage * L::kA, &tma_a, &full[stage], kb * 64, t.a_row, pol_a);
+        if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
+        tma_load_2d(sB + stage * L::kB, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
+        if (SPLIT == kSplitB) tma_load_2d(sB2 + stage * L::kB2, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok) {
+      atomicExch(err, kDevTimeoutProducer);
+      *abort_flag = 1;
+      // let the copies already in flight land before the CTA's shared memory goes away
+      int s = stage, p = phase;
+      for (int i = 0; i < min(issued, STAGES); ++i) {
+        s = (s + STAGES - 1) % STAGES;
+        if (s == STAGES - 1) p ^= 1;
+        unsigned long long t0 = global_ns();
+        while (!mbar_try_wait(&full[s], p) && global_ns() - t0 < kWaitLimitNs) {}
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int acc = j % ACC_BUFS;
+      const uint32_t acc_phase = (j / ACC_BUFS) & 1;
+      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kCols;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + stage * L::kA);
+        const uint32_t b0 = smem_u32(sB + stage * L::kB);
+        const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
+        const uint32_t b1 = smem_u32(sB2 + stage * L::kB2);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc,
+                    (kb | kk) != 0);
+          if (SPLIT == kSplitA)
+            umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc, 1);
+          if (SPLIT == kSplitB)
+            umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b1 + kk * 32), kIdesc, 1);
+        }
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok) umma_commit(&acc_full[acc]);
+    }
+    if (!ok) {
+      atomicExch(err, kDevTimeoutMma);
+      *abort_flag = 1;
+    }
+    // wait for every MMA issued by this thread before TMEM is released
+    umma_commit(drain);
+    unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;            // accumulator row owned by this thread
+    for (int j = 0; j < ntiles; ++j) {
+      const int acc = j % ACC_BUFS;
+      const uint32_t acc_phase = (j / ACC_BUFS) & 1;
+      const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
+      if (!epi_all(got)) {
+        if (!got) atomicExch(err, kDevTimeoutEpilogue);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const Tile t = sched.tile(j);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kCols;
+      epi(t, taddr, r, epi_smem);
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ======================================================================== epilogues
+
+// Plain fp32 store of D (used by the GEMM unit entry point).
+template <int BN>
+struct EpiStoreF32 {
+  static constexpr int kSmemBytes = 0;
+  float* out;
+  int ldo;
+  int N;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    const long row = t.a_row + r;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+      if (r < t.m_valid) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          int col = t.b_row + c + i;
+          if (col < N) out[row * ldo + col] = v[i];
+        }
+      }
+    }
+  }
+};
+
+// Fused QKV epilogue: tile = one head (BN = head_dim) of the concatenated [Q | K | V]
+// projection. Q and K get RoPE (rotate-half pairs (i, i + hd/2)); Q goes to the query
+// buffer, K and V to the layer's KV cache at the token's absolute position.
+template <int HD>
+struct EpiQKV {
+  static constexpr int kSmemBytes = 0;
+  bf16_t* q;            // [T][H][HD]
+  bf16_t* kc;           // layer cache [slots][Hkv][max_ctx][HD]
+  bf16_t* vc;
+  const float* rope_cos;   // [max_ctx][HD/2]
+  const float* rope_sin;
+  const int* pos0;      // per request: absolute position of its first token
+  const int* slot;      // per request: KV slot
+  int tok_per_req, H, Hkv, max_ctx;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    constexpr int HALF = HD / 2;
+    const int tok = t.a_row + r;
+    const bool valid = r < t.m_valid;
+    const int hh = t.nt;
+    int b = 0, pos = 0;
+    if (valid) {
+      b = tok / tok_per_req;
+      pos = pos0[b] + (tok - b * tok_per_req);
+    }
+    bf16_t* dst;
+    if (hh < H) dst = q + ((long)tok * H + hh) * HD;
+    else if (hh < H + Hkv) dst = kc + (((long)slot[b] * Hkv + (hh - H)) * max_ctx + pos) * HD;
+    else dst = vc + (((long)slot[b] * Hkv + (hh - H - Hkv)) * max_ctx + pos) * HD;
+    if (hh < H + Hkv) {
+#pragma unroll 1
+      for (int c = 0; c < HALF; c += 8) {
+        float a[8], bb[8];
+        tmem_ld8(taddr + c, a);
+        tmem_ld8(taddr + c + HALF, bb);
+        if (valid) {
+          const float* cs = rope_cos + (long)pos * HALF + c;
+          const float* sn = rope_sin + (long)pos * HALF + c;
+          uint32_t lo[4], hi[4];
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            float c0 = cs[i], c1 = cs[i + 1], s0 = sn[i], s1 = sn[i + 1];
+            lo[i / 2] = pack_bf16x2(a[i] * c0 - bb[i] * s0, a[i + 1] * c1 - bb[i + 1] * s1);
+            hi[i / 2] = pack_bf16x2(bb[i] * c0 + a[i] * s0, bb[i + 1] * c1 + a[i + 1] * s1);
+          }
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(dst + c + HALF) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < HD; c += 8) {
+        float a[8];
+        tmem_ld8(taddr + c, a);
+        if (valid) {
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                                                          pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+        }
+      }
+    }
+  }
+};
+
+// x[row][col] += D: the attention output projection with its residual add.
+template <int BN>
+struct EpiResidual {
+  static constexpr int kSmemBytes = 0;
+  float* x;
+  int ldx;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    float* row = x + (long)(t.a_row + r) * ldx + t.b_row;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+      if (r < t.m_valid) {
+        float4* p = reinterpret_cast<float4*>(row + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float4 o = p[i];
+          o.x += v[4 * i + 0];
+          o.y += v[4 * i + 1];
+          o.z += v[4 * i + 2];
+          o.w += v[4 * i + 3];
+          p[i] = o;
+        }
+      }
+    }
+  }
+};
+
+// Grouped gate/up epilogue: accumulator rows 0..63 are gate features 64*mt + r, rows
+// 64..127 the matching up features; columns are the chunk's tokens. The up half goes
+// through shared memory; h = silu(g) * u is written as the (hi, lo) bf16 pair that the
+// down GEMM consumes.
+template <int BN>
+struct EpiSwiGLU {
+  static constexpr int kSmemBytes = 16 * 65 * 4;
+  bf16_t* h;     // [slots][F], hi part
+  bf16_t* h_lo;  // [slots][F], lo part
+  int F;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t* smem) const {
+    float* us = reinterpret_cast<float*>(smem);
+    const int f = t.mt * 64 + (r & 63);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+      if (r >= 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) us[i * 65 + (r - 64)] = v[i];
+      }
+      epi_bar_sync();
+      if (r < 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int n = c + i;
+          if (n < t.n_valid) {
+            const float g = v[i];
+            const float u = us[i * 65 + r];
+            const float hv = g / (1.0f + __expf(-g)) * u;
+            const bf16_t hi = f32_to_bf16(hv);
+            const long o = (long)(t.b_row + n) * F + f;
+            h[o] = hi;
+            h_lo[o] = f32_to_bf16(hv - bf16_to_f32(hi));
+          }
+        }
+      }
+      epi_bar_sync();
+    }
+  }
+};
+
+// Grouped down epilogue: accumulator rows are output features 128*mt + r, columns the
+// chunk's tokens; o[slot][feature] in fp32 for the combine.
+template <int BN>
+struct EpiDown {
+  static constexpr int kSmemBytes = 0;
+  float* o;      // [slots][d]
+  int d;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    const int dd = t.mt * 128 + r;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int n = c + i;
+        if (n < t.n_valid) o[(long)(t.b_row + n) * d + dd] = v[i];
+      }
+    }
+  }
+};
+
+// LM-head epilogue: per row, over this tile's BN vocabulary columns, the running
+// maximum logit, its (lowest) token id and sum exp(l - max), with [MASK] left out.
+// Logits never leave the SM; a merge kernel combines the per-tile partials.
+template <int BN>
+struct EpiLMHead {
+  static constexpr int kSmemBytes = 0;
+  float* part_m;      // [rows][n_vtiles]
+  float* part_s;
+  int* part_i;
+  int n_vtiles;
+  int mask_id;
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    constexpr float kLog2e = 1.4426950408889634f;
+    float m = -INFINITY, s = 0.f;
+    int idx = 0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int col = t.b_row + c + i;
+        const float l = v[i];
+        if (col == mask_id) continue;
+        if (l > m) {
+          s = s * exp2f((m - l) * kLog2e) + 1.0f;
+          m = l;
+          idx = col;
+        } else {
+          s += exp2f((l - m) * kLog2e);
+        }
+      }
+    }
+    if (r < t.m_valid) {
+      const long o = (long)(t.a_row + r) * n_vtiles + t.nt;
+      part_m[o] = m;
+      part_s[o] = s;
+      part_i[o] = idx;
+    }
+  }
+};
+
+}  // namespace dllm

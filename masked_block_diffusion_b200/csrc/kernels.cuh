@@ -1,0 +1,431 @@
+// Bandwidth- and latency-bound kernels of the denoising pass: embedding gather,
+// RMSNorm, MoE router / top-k / permute / gather / combine, the LM-head partial merge,
+// and the commit (sampler) kernel.
+#pragma once
+
+#include "common.cuh"
+
+namespace dllm {
+
+// ---------------------------------------------------------------- a1: embedding
+
+// x[t] = Emb[token] as fp32; a masked canvas position reads the [MASK] row.
+__global__ void embed_kernel(const bf16_t* __restrict__ emb, const int32_t* __restrict__ tokens,
+                             const uint8_t* __restrict__ mask, int mask_id, int d, float* __restrict__ x) {
+  const int t = blockIdx.x;
+  int tok = tokens[t];
+  if (mask != nullptr && mask[t]) tok = mask_id;
+  const uint4* src = reinterpret_cast<const uint4*>(emb + (long)tok * d);
+  float4* dst = reinterpret_cast<float4*>(x + (long)t * d);
+  for (int c = threadIdx.x; c < d / 8; c += blockDim.x) {
+    uint4 v = src[c];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    dst[2 * c] = make_float4(f[0], f[1], f[2], f[3]);
+    dst[2 * c + 1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// ---------------------------------------------------------------- a2/a6/a12: RMSNorm
+
+// v = x * rsqrt(mean(x^2) + eps) * g, written as the bf16 pair y = bf16(v),
+// y_lo = bf16(v - y) (y_lo may be NULL); rstd[t] kept for the fp32 router.
+__global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
+                               bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo, float* __restrict__ rstd) {
+  const int t = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + (long)t * d);
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 v = xr[c];
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = rsqrtf(red[0] / (float)d + eps);
+  if (threadIdx.x == 0 && rstd != nullptr) rstd[t] = r;
+  const float4* gr = reinterpret_cast<const float4*>(g);
+  uint2* yr = reinterpret_cast<uint2*>(y + (long)t * d);
+  uint2* yl = y_lo ? reinterpret_cast<uint2*>(y_lo + (long)t * d) : nullptr;
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 v = xr[c], gg = gr[c];
+    uint32_t h0, l0, h1, l1;
+    split_bf16x2(v.x * r * gg.x, v.y * r * gg.y, h0, l0);
+    split_bf16x2(v.z * r * gg.z, v.w * r * gg.w, h1, l1);
+    yr[c] = make_uint2(h0, h1);
+    if (yl) yl[c] = make_uint2(l0, l1);
+  }
+}
+
+// ---------------------------------------------------------------- a7: router + top-k
+
+// logits[t][e] = sum_k (x[t][k] * rstd[t] * g[k]) * Wr[e][k], all in fp32. Each block
+// holds kRouterTok normalised rows in shared memory; each warp walks experts.
+constexpr int kRouterTok = 4;
+__global__ void router_kernel(const float* __restrict__ x, const float* __restrict__ rstd,
+                              const float* __restrict__ g, const bf16_t* __restrict__ wr, int T, int d, int E,
+                              float* __restrict__ logits) {
+  extern __shared__ float xs[];   // [kRouterTok][d]
+  const int t0 = blockIdx.x * kRouterTok;
+  for (int i = threadIdx.x; i < kRouterTok * d; i += blockDim.x) {
+    const int tk = i / d, k = i % d;
+    const int t = t0 + tk;
+    xs[i] = (t < T) ? x[(long)t * d + k] * rstd[t] * g[k] : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nw) {
+    float acc[kRouterTok];
+#pragma unroll
+    for (int i = 0; i < kRouterTok; ++i) acc[i] = 0.f;
+    const bf16_t* w = wr + (long)e * d;
+    for (int k = lane * 8; k < d; k += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(w + k);
+      const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+      float wf[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        wf[2 * i] = __uint_as_float(ww[i] << 16);
+        wf[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int tk = 0; tk < kRouterTok; ++tk) {
+        const float* xr = xs + tk * d + k;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[tk] = fmaf(wf[i], xr[i], acc[tk]);
+      }
+    }
+#pragma unroll
+    for (int tk = 0; tk < kRouterTok; ++tk) {
+      const float s = warp_sum(acc[tk]);
+      if (lane == 0 && t0 + tk < T) logits[(long)(t0 + tk) * E + e] = s;
+    }
+  }
+}
+
+// Top-k experts per token by logit (ties to the lower expert) and gates = softmax of
+// the k selected logits. One warp per token; E <= 256, k <= 32.
+__global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
+                            float* __restrict__ gate) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float v[8];
+  bool taken[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? logits[(long)t * E + e] : -INFINITY;
+    taken[j] = (e >= E);
+  }
+  float sel_v = 0.f, top = 0.f;
+  int sel_i = 0;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (!taken[j] && (v[j] > bv || (v[j] == bv && e < bi))) { bv = v[j]; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (lane + 32 * j == bi) taken[j] = true;
+    if (r == 0) top = bv;
+    if (lane == r) { sel_v = bv; sel_i = bi; }
+  }
+  const float ex = (lane < k) ? expf(sel_v - top) : 0.f;
+  const float z = warp_sum(ex);
+  if (lane < k) {
+    idx[(long)t * k + lane] = sel_i;
+    gate[(long)t * k + lane] = ex / z;
+  }
+}
+
+// Debug: replace the top-k experts with given ones (the oracle's), gates recomputed
+// from this pass's own logits at those experts. One thread per token.
+__global__ void force_route_kernel(const float* __restrict__ logits, const int32_t* __restrict__ forced, int T,
+                                   int E, int k, int32_t* __restrict__ idx, float* __restrict__ gate) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float mx = -INFINITY;
+  for (int j = 0; j < k; ++j) mx = fmaxf(mx, logits[(long)t * E + forced[(long)t * k + j]]);
+  float z = 0.f;
+  for (int j = 0; j < k; ++j) z += expf(logits[(long)t * E + forced[(long)t * k + j]] - mx);
+  for (int j = 0; j < k; ++j) {
+    const int e = forced[(long)t * k + j];
+    idx[(long)t * k + j] = e;
+    gate[(long)t * k + j] = expf(logits[(long)t * E + e] - mx) / z;
+  }
+}
+
+// Dense FFN as one expert with gate 1.
+__global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) { idx[t] = 0; gate[t] = 1.f; }
+}
+
+// ---------------------------------------------------------------- a8: permute
+
+// Stable counting sort of the N = T*k assignments by expert (one CTA of 1024 threads).
+// offsets[E+1]: expert ranges in the sorted order; slot_of[i]: sorted position of
+// assignment i = t*k + j; row_token[slot]: its token. Within an expert, assignments
+// keep their (t, j) order, so the permutation is deterministic.
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int N, int k, int E,
+                                                       int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
+                                                       int32_t* __restrict__ row_token) {
+  extern __shared__ int sh[];
+  int* cnt = sh;                 // [E]
+  int* base = sh + E;            // [E] running start of each expert
+  int* wcnt = sh + 2 * E;        // [32][E] per-warp counts -> per-warp prefix
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < N; i += blockDim.x) atomicAdd(&cnt[idx[i]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      base[e] = run;
+      offsets[e] = run;
+      run += cnt[e];
+    }
+    offsets[E] = run;
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const int i = c0 + tid;
+    const int e = (i < N) ? idx[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank_w == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int run = 0;
+      for (int w = 0; w < 32; ++w) {
+        const int v = wcnt[w * E + ee];
+        wcnt[w * E + ee] = run;
+        run += v;
+      }
+      cnt[ee] = run;   // this chunk's count of expert ee
+    }
+    __syncthreads();
+    if (e >= 0) {
+      const int s = base[e] + wcnt[warp * E + e] + rank_w;
+      slot_of[i] = s;
+      row_token[s] = i / k;
+    }
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) base[ee] += cnt[ee];
+    __syncthreads();
+  }
+}
+
+// xg[slot] = y[row_token[slot]] for the hi and lo bf16 rows: the B operand pair of the
+// grouped gate/up GEMM.
+__global__ void gather_rows_kernel(const bf16_t* __restrict__ y, const bf16_t* __restrict__ y_lo,
+                                   const int32_t* __restrict__ row_token, int N, int d, bf16_t* __restrict__ xg,
+                                   bf16_t* __restrict__ xg_lo) {
+  const int s = blockIdx.x;
+  if (s >= N) return;
+  const long src_row = (long)row_token[s] * d;
+  const uint4* src = reinterpret_cast<const uint4*>(y + src_row);
+  const uint4* src_lo = reinterpret_cast<const uint4*>(y_lo + src_row);
+  uint4* dst = reinterpret_cast<uint4*>(xg + (long)s * d);
+  uint4* dst_lo = reinterpret_cast<uint4*>(xg_lo + (long)s * d);
+  for (int c = threadIdx.x; c < d / 8; c += blockDim.x) {
+    dst[c] = src[c];
+    dst_lo[c] = src_lo[c];
+  }
+}
+
+// ---------------------------------------------------------------- a11: combine
+
+// x[t] += sum_j gate[t][j] * o[slot_of[t*k + j]], j in fixed order 0..k-1.
+__global__ void combine_kernel(float* __restrict__ x, const float* __restrict__ o, const int32_t* __restrict__ slot_of,
+                               const float* __restrict__ gate, int k, int d) {
+  const int t = blockIdx.x;
+  float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float w = gate[(long)t * k + j];
+      const float4 v = reinterpret_cast<const float4*>(o + (long)slot_of[(long)t * k + j] * d)[c];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    float4 xv = xr[c];
+    xv.x += acc.x;
+    xv.y += acc.y;
+    xv.z += acc.z;
+    xv.w += acc.w;
+    xr[c] = xv;
+  }
+}
+
+// ---------------------------------------------------------------- a13: LM-head merge
+
+DLLM_DEV void lse_combine(float& m, float& s, int& i, float m2, float s2, int i2) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (m2 > m) {
+    s = s2 + s * exp2f((m - m2) * kLog2e);
+    m = m2;
+    i = i2;
+  } else if (m2 < m) {
+    s += s2 * exp2f((m2 - m) * kLog2e);
+  } else {
+    s += s2;
+    i = min(i, i2);
+  }
+}
+
+// conf[t] = 1 / sum_v exp(l_v - max), argmax[t] = lowest id reaching the max.
+// One warp per row over the row's vocabulary-tile partials.
+__global__ void lm_merge_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
+                                const int32_t* __restrict__ pi, int rows, int n_tiles, float* __restrict__ conf,
+                                int32_t* __restrict__ argmax) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= rows) return;
+  float m = -INFINITY, s = 0.f;
+  int i = 0x7fffffff;
+  for (int j = lane; j < n_tiles; j += 32) {
+    const long o = (long)t * n_tiles + j;
+    lse_combine(m, s, i, pm[o], ps[o], pi[o]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+    const int i2 = __shfl_xor_sync(0xffffffffu, i, off);
+    lse_combine(m, s, i, m2, s2, i2);
+  }
+  if (lane == 0) {
+    conf[t] = 1.0f / s;
+    argmax[t] = i;
+  }
+}
+
+// ---------------------------------------------------------------- a14: commit
+
+struct PolicyDev {
+  int kind;       // 0 top-k, 1 threshold
+  int k;
+  float tau;
+  int floor;
+  int max_steps;
+};
+
+// One CTA per request (C <= 1024 positions). Commits the n most confident masked
+// positions (fp32 conf, ties to the lower position): top-k: n = min(k, R);
+// threshold: n = max(#{conf > tau}, n_min) with the step-budget floor
+// n_min = max(1, ceil(R / (S_max - s))), capped at R. Writes the committed token,
+// clears the mask bit, stores R - n and advances the request's step counter.
+__global__ void commit_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict__ mask, const float* __restrict__ conf,
+                              const int32_t* __restrict__ argmax, int C, const PolicyDev* __restrict__ pol,
+                              int32_t* __restrict__ step, int32_t* __restrict__ remaining, float* __restrict__ conf_out,
+                              int32_t* __restrict__ argmax_out) {
+  extern __shared__ uint8_t smc[];
+  float* sc = reinterpret_cast<float*>(smc);
+  uint8_t* sm = smc + C * sizeof(float);
+  const int b = blockIdx.x, i = threadIdx.x;
+  const long o = (long)b * C + i;
+  const PolicyDev P = *pol;
+  float ci = 0.f;
+  int mi = 0;
+  if (i < C) {
+    ci = conf[o];
+    mi = mask[o];
+    sc[i] = ci;
+    sm[i] = (uint8_t)mi;
+    if (conf_out) conf_out[o] = ci;
+    if (argmax_out) argmax_out[o] = argmax[o];
+  }
+  const int R = __syncthreads_count(i < C && mi);
+  const int above = __syncthreads_count(i < C && mi && ci > P.tau);
+  const int s = step[b];
+  int n;
+  if (P.kind == 0) {
+    n = P.k;
+  } else {
+    n = above;
+    if (P.floor) {
+      const int left = P.max_steps - s;
+      const int nmin = left <= 0 ? R : max(1, (R + left - 1) / left);
+      n = max(n, nmin);
+    }
+  }
+  n = max(0, min(n, R));
+  if (i < C && mi) {
+    int rank = 0;
+    for (int j = 0; j < C; ++j) {
+      const float cj = sc[j];
+      rank += (sm[j] && (cj > ci || (cj == ci && j < i))) ? 1 : 0;
+    }
+    if (rank < n) {
+      canvas[o] = argmax[o];
+      mask[o] = 0;
+    }
+  }
+  if (i == 0) {
+    remaining[b] = R - n;
+    step[b] = s + 1;
+  }
+}
+
+// Fresh all-[MASK] canvases and zeroed step counters.
+__global__ void canvas_init_kernel(int32_t* canvas, uint8_t* mask, int n, int mask_id, int32_t* step, int B) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    canvas[i] = mask_id;
+    mask[i] = 1;
+  }
+  if (i < B) step[i] = 0;
+}
+
+// ---------------------------------------------------------------- weight packing
+
+// dst row ((i / group) * group_stride + i % group + row_offset) = bf16(src row i).
+__global__ void pack_rows_kernel(bf16_t* __restrict__ dst, const void* __restrict__ src, int src_f32, long n_rows,
+                                 int d, long group, long group_stride, long row_offset) {
+  const long n = n_rows * d;
+  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long)gridDim.x * blockDim.x) {
+    const long i = e / d, c = e % d;
+    const long drow = (i / group) * group_stride + (i % group) + row_offset;
+    bf16_t v;
+    if (src_f32) v = f32_to_bf16(reinterpret_cast<const float*>(src)[e]);
+    else v = reinterpret_cast<const bf16_t*>(src)[e];
+    dst[drow * d + c] = v;
+  }
+}
+
+__global__ void to_f32_kernel(float* __restrict__ dst, const void* __restrict__ src, int src_f32, long n) {
+  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long)gridDim.x * blockDim.x) {
+    dst[e] = src_f32 ? reinterpret_cast<const float*>(src)[e]
+                     : bf16_to_f32(reinterpret_cast<const bf16_t*>(src)[e]);
+  }
+}
+
+}  // namespace dllm

@@ -43,12 +43,12 @@ Readings where the pages are silent (all listed in the design notes):
    position; threshold: every masked position with conf > tau, and at least
    n_min = max(1, ceil(R / (S_max - s))) of the most confident ones so that the
    canvas completes within the step budget;
-10. precision: GEMM operands are bf16 ("bf16 operands, fp32 accumulation"); the
-   oracle accumulates in fp64 and rounds to bf16 exactly where a bf16 operand is
-   formed (normalised activations, Q/K/V after RoPE and the KV cache, attention
-   output, SwiGLU output); the residual stream, router and softmax statistics stay
-   in high precision; router logits and LM-head logits are rounded to fp32 before
-   the top-k / argmax decision, and conf is rounded to fp32 before commit ranking.
+10. precision: the weights are bf16 values and the KV cache holds bf16 values, so
+   Q, K and V after RoPE are rounded to bf16 (Q too: it is formed once and read only
+   by attention); every other quantity (normalised activations, attention output,
+   SwiGLU output, residual stream, router, softmax statistics) is computed in fp64;
+   router and LM-head logits are rounded to fp32 before the top-k / argmax decision,
+   and conf to fp32 before commit ranking.
 
 Parity pins (tests/test_oracle_pins.py): attention against brute force and closed
 forms; RoPE relative-position invariance; KV-cache pass equal to an uncached
@@ -81,6 +81,15 @@ def bf16(x) -> np.ndarray:
 
 def f32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+def bf16_store(w) -> np.ndarray:
+    """A weight matrix as its bf16 values, kept in float32 (exact); matmuls upcast to fp64."""
+    w = np.asarray(w, dtype=np.float32)
+    u = w.view(np.uint32)
+    if not np.any(u & np.uint32(0xFFFF)):
+        return w                      # already bf16-exact: no copy
+    return bf16(w).astype(np.float32)
 
 
 # --------------------------------------------------------------------------------------
@@ -152,21 +161,21 @@ def router_topk(y: np.ndarray, wr: np.ndarray, k: int):
 
 
 def swiglu_expert(yb: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
-    """Wd (silu(Wg y) * (Wu y)); the SwiGLU product is a bf16 operand of the down GEMM."""
+    """Wd (silu(Wg y) * (Wu y)) in fp64."""
     g = yb @ np.asarray(wg, np.float64).T
     u = yb @ np.asarray(wu, np.float64).T
-    h = bf16(g / (1.0 + np.exp(-g)) * u)
+    h = g / (1.0 + np.exp(-g)) * u
     return h @ np.asarray(wd, np.float64).T
 
 
 def moe_ffn(y: np.ndarray, experts, wr: Optional[np.ndarray], k: int):
-    """Mixture-of-experts FFN: sum_j gate_j * expert_{idx_j}(bf16(y)).
+    """Mixture-of-experts FFN: sum_j gate_j * expert_{idx_j}(y).
 
     experts: list of (wg, wu, wd); wr None means the dense FFN (one expert, gate 1).
     Returns (delta [T][d], logits or None, idx [T][k], gates [T][k]).
     """
     T = y.shape[0]
-    yb = bf16(y)
+    yb = np.asarray(y, dtype=np.float64)
     if wr is None:
         logits = None
         idx = np.zeros((T, 1), dtype=np.int64)
@@ -186,7 +195,7 @@ def moe_ffn(y: np.ndarray, experts, wr: Optional[np.ndarray], k: int):
 def lm_head_conf(x: np.ndarray, final_norm: np.ndarray, head: np.ndarray, mask_id: int,
                  eps: float, return_logits: bool = False):
     """Per row: argmax token and conf = max softmax probability, [MASK] excluded (readings 7, 8)."""
-    yb = bf16(rmsnorm(x, final_norm, eps))
+    yb = rmsnorm(x, final_norm, eps)
     logits = f32(yb @ np.asarray(head, np.float64).T)
     logits[:, mask_id] = -np.inf
     m = np.max(logits, axis=1)
@@ -258,31 +267,31 @@ class OracleModel:
         self.cfg = cfg
         c = cfg
         # every matrix is a bf16 operand (reading 10); norm gains stay as given
-        self.emb = bf16(weights["emb"])
+        self.emb = bf16_store(weights["emb"])
         self.layers = []
         for l in range(c.n_layers):
             p = f"layers.{l}."
             lw = {
                 "attn_norm": np.asarray(weights[p + "attn_norm"], np.float64),
-                "wq": bf16(weights[p + "wq"]),
-                "wk": bf16(weights[p + "wk"]),
-                "wv": bf16(weights[p + "wv"]),
-                "wo": bf16(weights[p + "wo"]),
+                "wq": bf16_store(weights[p + "wq"]),
+                "wk": bf16_store(weights[p + "wk"]),
+                "wv": bf16_store(weights[p + "wv"]),
+                "wo": bf16_store(weights[p + "wo"]),
                 "ffn_norm": np.asarray(weights[p + "ffn_norm"], np.float64),
             }
             if c.dense:
                 lw["wr"] = None
-                lw["experts"] = [(bf16(weights[p + "wg"]), bf16(weights[p + "wu"]),
-                                  bf16(weights[p + "wd"]))]
+                lw["experts"] = [(bf16_store(weights[p + "wg"]), bf16_store(weights[p + "wu"]),
+                                  bf16_store(weights[p + "wd"]))]
             else:
-                lw["wr"] = bf16(weights[p + "wr"])
-                lw["experts"] = [(bf16(weights[p + f"experts.{e}.wg"]),
-                                  bf16(weights[p + f"experts.{e}.wu"]),
-                                  bf16(weights[p + f"experts.{e}.wd"]))
+                lw["wr"] = bf16_store(weights[p + "wr"])
+                lw["experts"] = [(bf16_store(weights[p + f"experts.{e}.wg"]),
+                                  bf16_store(weights[p + f"experts.{e}.wu"]),
+                                  bf16_store(weights[p + f"experts.{e}.wd"]))
                                  for e in range(c.n_experts)]
             self.layers.append(lw)
         self.final_norm = np.asarray(weights["final_norm"], np.float64)
-        self.head = bf16(weights["head"])
+        self.head = bf16_store(weights["head"])
         self.requests: Dict[int, _Request] = {}
 
     # ---- one transformer layer -------------------------------------------------------
@@ -291,7 +300,7 @@ class OracleModel:
         """x [T][d] -> x', plus the layer's new K/V [T][Hkv][hd] (bf16 values)."""
         c, lw = self.cfg, self.layers[l]
         T = x.shape[0]
-        y = bf16(rmsnorm(x, lw["attn_norm"], c.rms_eps))
+        y = rmsnorm(x, lw["attn_norm"], c.rms_eps)
         q = (y @ lw["wq"].T).reshape(T, c.n_heads, c.head_dim)
         k = (y @ lw["wk"].T).reshape(T, c.n_kv_heads, c.head_dim)
         v = (y @ lw["wv"].T).reshape(T, c.n_kv_heads, c.head_dim)
@@ -304,7 +313,7 @@ class OracleModel:
             vv = np.concatenate([v_prev, v], axis=0)
         else:
             kk, vv = k, v
-        o = bf16(attention(q, kk, vv, allowed)).reshape(T, c.q_dim)
+        o = attention(q, kk, vv, allowed).reshape(T, c.q_dim)
         x = x + o @ lw["wo"].T
         y2 = rmsnorm(x, lw["ffn_norm"], c.rms_eps)
         delta, logits, idx, gates = moe_ffn(y2, lw["experts"], lw["wr"], c.top_k)
@@ -326,7 +335,7 @@ class OracleModel:
         prompt = np.asarray(prompt, dtype=np.int64)
         n = prompt.size
         st = _Request(c.n_layers)
-        x = self.emb[prompt].copy()
+        x = self.emb[prompt].astype(np.float64)
         pos = np.arange(n)
         allowed = pos[None, :] <= pos[:, None]
         for l in range(c.n_layers):
@@ -340,7 +349,7 @@ class OracleModel:
         c = self.cfg
         st = self.requests[req]
         tokens = np.where(np.asarray(mask, bool), c.mask_id, np.asarray(canvas, np.int64))
-        x = self.emb[tokens].copy()
+        x = self.emb[tokens].astype(np.float64)
         C = tokens.size
         pos = st.P + np.arange(C)
         new_k, new_v = [], []
@@ -410,7 +419,7 @@ def sequence_forward(model: OracleModel, tokens: np.ndarray, allowed: np.ndarray
     """
     c = model.cfg
     tokens = np.asarray(tokens, dtype=np.int64)
-    x = model.emb[tokens].copy()
+    x = model.emb[tokens].astype(np.float64)
     pos = np.arange(tokens.size)
     for l in range(c.n_layers):
         x, _, _ = model.layer(l, x, pos, None, None, allowed)

@@ -15,6 +15,7 @@ from .gen import (
     gen_tensor,
     gen_weights,
     gen_blob,
+    blob_from_weights,
     prompt_tokens,
     normal_f32,
     f32_to_bf16_bits,
@@ -24,6 +25,6 @@ from .gen import (
 
 __all__ = [
     "ModelConfig", "Workload", "CONFIGS", "WORKLOADS", "get_config", "get_workload",
-    "splitmix64", "tensor_specs", "blob_layout", "gen_tensor", "gen_weights", "gen_blob",
+    "splitmix64", "tensor_specs", "blob_layout", "gen_tensor", "gen_weights", "gen_blob", "blob_from_weights",
     "prompt_tokens", "normal_f32", "f32_to_bf16_bits", "bf16_bits_to_f32", "uniform_f32",
 ]

@@ -199,3 +199,13 @@ def gen_blob(cfg: ModelConfig, seed: int | None = None) -> np.ndarray:
             raw = w.astype(np.float32).view(np.uint8)
         buf[ent.offset:ent.offset + raw.size] = raw
     return buf
+
+
+def blob_from_weights(cfg: ModelConfig, weights: Dict[str, np.ndarray]) -> np.ndarray:
+    """The blob holding already generated tensors (avoids generating them twice)."""
+    buf = np.zeros(blob_bytes(cfg), dtype=np.uint8)
+    for ent in blob_layout(cfg):
+        w = np.asarray(weights[ent.spec.name], dtype=np.float32).reshape(-1)
+        raw = f32_to_bf16_bits(w).view(np.uint8) if cfg.weight_dtype == "bf16" else w.view(np.uint8)
+        buf[ent.offset:ent.offset + raw.size] = raw
+    return buf

@@ -1,0 +1,134 @@
+"""Step-by-step parity of the CUDA path against the oracle (used by the GPU tests).
+
+Each denoising step of the oracle's trace is replayed on the GPU from the oracle's
+own (canvas, mask), so a near-tie decided differently at one step cannot compound.
+Tolerances (fixed for this path): routing sets, argmax tokens and commit sets equal
+wherever the oracle's margin at the decision exceeds 1e-3 (router logit units, LM
+logit units, log-confidence units); conf within 2e-2 relative; final hidden state
+within 2e-2 of the row's largest magnitude.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from masked_block_diffusion_b200 import Denoiser, make_policy
+from oracle import OracleModel, Policy
+from synth import blob_from_weights, gen_weights, prompt_tokens
+
+MARGIN = 1e-3
+REL = 2e-2
+
+
+def build_pair(cfg, prefix: int, prompt_seed: int, max_ctx: int, max_batch: int = 1):
+    W = gen_weights(cfg)
+    blob = blob_from_weights(cfg, W)
+    orc = OracleModel(cfg, W)
+    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=max_batch)
+    del blob
+    prompt = prompt_tokens(cfg.vocab, prompt_seed, prefix)
+    orc.prefill(0, prompt)
+    den.prefill(0, prompt)
+    return orc, den, prompt
+
+
+def commit_margin(conf: np.ndarray, mask: np.ndarray, n: int, policy: Policy) -> float:
+    """log-confidence gap at the commit boundary (and at tau for the threshold policy)."""
+    masked = np.nonzero(mask)[0]
+    c = np.asarray(conf, np.float64)[masked]
+    order = np.lexsort((masked, -c))
+    cs = c[order]
+    m = math.inf
+    if 0 < n < cs.size:
+        m = math.log(cs[n - 1]) - math.log(cs[n])
+    if policy.kind == "threshold" and math.isfinite(policy.tau):
+        m = min(m, float(np.min(np.abs(np.log(cs) - math.log(policy.tau)))))
+    return m
+
+
+def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, stats=None):
+    """Replays every oracle step on the GPU and checks the decisions and values."""
+    C = cfg.canvas
+    stats = stats if stats is not None else {"route_pinned": 0, "route_total": 0, "arg_pinned": 0,
+                                             "arg_total": 0, "commit_pinned": 0, "steps": 0}
+    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor)
+    den.set_debug(True)
+    for e in orc_trace:
+        rec = e["rec"]
+        canvas = torch.from_numpy(e["canvas"].astype(np.int32)[None]).cuda()
+        mask = torch.from_numpy(e["mask"].astype(np.uint8)[None]).cuda()
+        old_mask = e["mask"].copy()
+        if not cfg.dense:
+            # each layer runs on the oracle's experts, so a near-tie flip in one layer
+            # cannot move the inputs of the next; every layer's own choice is still checked
+            den.force_routing(np.stack(rec["topk_idx"]))
+        conf, arg, rem = den.denoise_step(canvas, mask, pol, e["step"], s_max)
+        conf = conf.cpu().numpy()[0]
+        arg = arg.cpu().numpy()[0]
+        new_mask = mask.cpu().numpy()[0].astype(bool)
+        new_canvas = canvas.cpu().numpy()[0]
+
+        # hidden state after the last layer
+        x_gpu = den.debug_read(0, 0, (C, cfg.d_model), np.float32).astype(np.float64)
+        x_ref = rec["final_x"]
+        row_err = np.abs(x_gpu - x_ref).max(axis=1) / np.abs(x_ref).max(axis=1)
+        assert row_err.max() <= REL, f"step {e['step']}: hidden rel err {row_err.max():.3g}"
+
+        # routing, layer by layer
+        if not cfg.dense:
+            k = cfg.top_k
+            for l in range(cfg.n_layers):
+                lg = rec["router_logits"][l]
+                srt = -np.sort(-lg, axis=1)
+                margin = srt[:, k - 1] - srt[:, k]
+                sel = margin > MARGIN
+                gi = den.debug_read(2, l, (C, k), np.int32)
+                ri = rec["topk_idx"][l]
+                same = np.array([set(gi[t]) == set(ri[t]) for t in range(C)])
+                bad = np.nonzero(sel & ~same)[0]
+                assert bad.size == 0, f"step {e['step']} layer {l}: routing differs at tokens {bad[:8]}"
+                stats["route_pinned"] += int(sel.sum())
+                stats["route_total"] += C
+                gl = den.debug_read(1, l, (C, cfg.n_experts), np.float32)
+                assert np.abs(gl - lg).max() <= REL * np.abs(lg).max()
+
+        # LM head: conf and argmax
+        assert np.all(np.abs(conf / e["conf"] - 1.0) <= REL), f"step {e['step']}: conf"
+        lm_sel = rec["logit_margin"] > MARGIN
+        bad = np.nonzero(lm_sel & (arg != e["argmax"]))[0]
+        assert bad.size == 0, f"step {e['step']}: argmax differs at {bad[:8]}"
+        stats["arg_pinned"] += int(lm_sel.sum())
+        stats["arg_total"] += C
+
+        # commit
+        gpu_commit = old_mask & ~new_mask
+        n = int(e["commit"].sum())
+        assert int(gpu_commit.sum()) == n, f"step {e['step']}: commit count {gpu_commit.sum()} vs {n}"
+        assert int(rem.cpu().numpy()[0]) == int(old_mask.sum()) - n
+        if commit_margin(e["conf"], old_mask, n, policy) > MARGIN:
+            assert np.array_equal(gpu_commit, e["commit"]), f"step {e['step']}: commit set differs"
+            stats["commit_pinned"] += 1
+        # committed positions hold the pass's argmax; earlier commits are untouched (M2T)
+        assert np.array_equal(new_canvas[gpu_commit], arg[gpu_commit])
+        assert np.array_equal(new_canvas[~old_mask], e["canvas"][~old_mask])
+        assert not np.any(new_mask & ~old_mask)
+        stats["steps"] += 1
+    if not cfg.dense:
+        den.force_routing(None)
+    den.set_debug(False)
+    return stats
+
+
+def check_generate_invariants(cfg, den: Denoiser, policy: Policy, s_max: int, expect_steps=None):
+    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor)
+    code, canvas, steps = den.generate_block(1, s_max, pol)
+    assert code == 0, code
+    c = canvas.cpu().numpy()[0]
+    assert np.all((c >= 0) & (c <= cfg.vocab - 2)), "a [MASK] or out-of-range token survived"
+    assert steps[0] <= s_max
+    if expect_steps is not None:
+        assert steps[0] == expect_steps
+    return c, steps[0]

@@ -148,7 +148,7 @@ def test_moe_reductions():
     wr = rnd((3, d), 13)
     # k = E: the softmax-weighted mixture of every expert
     out, logits, idx, gates = moe_ffn(y, experts, wr, 3)
-    yb = oracle.bf16(y)
+    yb = y
     p = scipy.special.softmax(logits, axis=1)
     ref = sum(p[:, e:e + 1] * swiglu_expert(yb, *experts[e]) for e in range(3))
     assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
@@ -157,7 +157,7 @@ def test_moe_reductions():
     assert np.allclose(g, 1.0)
     wg, wu, wd = experts[0]
     h = yb @ wg.T
-    ref_dense = oracle.bf16(h * scipy.special.expit(h) * (yb @ wu.T)) @ wd.T
+    ref_dense = (h * scipy.special.expit(h) * (yb @ wu.T)) @ wd.T
     assert np.allclose(dense, ref_dense, rtol=1e-12, atol=1e-12)
 
 
@@ -177,7 +177,7 @@ def test_lm_head_logsumexp_and_mask_exclusion():
     head[V - 1] = 50.0 * oracle.bf16(x[0]) / np.linalg.norm(x[0])   # [MASK] would win row 0
     head = oracle.bf16(head)
     conf, arg, logits = lm_head_conf(x, np.ones(d), head, V - 1, 1e-6, return_logits=True)
-    y = oracle.bf16(oracle.rmsnorm(x, np.ones(d), 1e-6))
+    y = oracle.rmsnorm(x, np.ones(d), 1e-6)
     raw = (y @ head.T)[:, : V - 1]
     assert np.all(arg != V - 1)
     assert np.array_equal(arg, np.argmax(raw, axis=1))
@@ -331,7 +331,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
     xx, head = rnd((7, d), 16), rnd((V, d), 17)
     head[V - 1] = 50.0 * oracle.bf16(xx[0]) / np.linalg.norm(xx[0])
     monkeypatch.setattr(np, "argmax", np.argmax)
-    y = oracle.bf16(oracle.rmsnorm(xx, np.ones(d), 1e-6))
+    y = oracle.rmsnorm(xx, np.ones(d), 1e-6)
     assert np.argmax(y @ oracle.bf16(head).T, axis=1)[0] == V - 1
 
     # floor rule off: the 12-step schedule would not finish the canvas
