@@ -156,14 +156,27 @@ long long dllm_launch_count(const dllm_handle* h);
 int dllm_set_debug(dllm_handle* h, int on);
 int dllm_debug_read(dllm_handle* h, int what, int layer, void* dst, size_t bytes);
 
-/* Debug (needs dllm_set_debug(h, 1)): later canvas passes over T tokens use the given
- * experts instead of their own top-k, layer by layer (idx: host int32 [n_layers][T][k]);
+/* Debug (needs dllm_set_debug(h, 1)): later passes over T tokens (canvas passes,
+ * prefill or append, whichever has exactly T tokens) use the given experts instead of
+ * their own top-k, layer by layer (idx: host int32 [n_layers][T][k]);
  * gates come from the pass's own router logits at those experts. The router's own
  * choice is still recorded for dllm_debug_read(what = 2). This isolates one layer's
  * routing decision from near-tie flips in earlier layers when comparing with a
  * reference. idx = NULL switches it off. Errors: DLLM_E_STATE (debug off),
  * DLLM_E_INVAL (dense model, T or an index out of range). */
 int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T);
+
+/* Kernel timing: with timing on, every later canvas pass brackets each layer's grouped
+ * gate/up GEMM and grouped down GEMM with CUDA events (recorded inside the pass's CUDA
+ * graph) and the elapsed times are summed per kind after each pass of
+ * dllm_generate_block. dllm_timing_read fills total_ms[kind] and launches[kind]
+ * (arrays of DLLM_TIMING_KINDS) and, if reset, zeroes the sums. Toggling timing drops
+ * captured graphs. */
+#define DLLM_TIMING_GATE_UP 0
+#define DLLM_TIMING_DOWN 1
+#define DLLM_TIMING_KINDS 2
+int dllm_set_timing(dllm_handle* h, int on);
+int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, int reset);
 
 const char* dllm_last_error(const dllm_handle* h);
 void dllm_destroy(dllm_handle* h);

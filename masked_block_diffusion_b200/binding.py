@@ -35,8 +35,11 @@ EXPORTS = [
     "dllm_create", "dllm_prefill", "dllm_denoise_step", "dllm_generate_block", "dllm_append_kv",
     "dllm_generate", "dllm_reset", "dllm_prefix_len", "dllm_check", "dllm_launch_count",
     "dllm_set_debug", "dllm_debug_read", "dllm_debug_force_routing", "dllm_last_error", "dllm_destroy",
-    "dllm_op_gemm_bf16", "dllm_op_lm_head_conf",
+    "dllm_op_gemm_bf16", "dllm_op_lm_head_conf", "dllm_set_timing", "dllm_timing_read",
 ]
+DLLM_TIMING_GATE_UP = 0
+DLLM_TIMING_DOWN = 1
+DLLM_TIMING_KINDS = 2
 
 
 class dllm_config(ctypes.Structure):
@@ -92,6 +95,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dllm_destroy": (None, [_vp]),
         "dllm_op_gemm_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
         "dllm_op_lm_head_conf": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+        "dllm_set_timing": (_i, [_vp, _i]),
+        "dllm_timing_read": (_i, [_vp, _vp, _vp, _i]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -209,3 +214,14 @@ def dllm_op_gemm_bf16(a_ptr, b_ptr, d_ptr, M, N, K, stream_ptr):
 def dllm_op_lm_head_conf(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, argmax_ptr, stream_ptr):
     _check(load().dllm_op_lm_head_conf(_vp(y_ptr), _vp(head_ptr), T, d, V, mask_id, _vp(conf_ptr),
                                        _vp(argmax_ptr), _vp(stream_ptr)), "dllm_op_lm_head_conf")
+
+
+def dllm_set_timing(h, on: bool):
+    _check(load().dllm_set_timing(h, 1 if on else 0), "dllm_set_timing", h)
+
+
+def dllm_timing_read(h, reset: bool = False):
+    ms = (ctypes.c_double * DLLM_TIMING_KINDS)()
+    n = (ctypes.c_longlong * DLLM_TIMING_KINDS)()
+    _check(load().dllm_timing_read(h, ms, n, 1 if reset else 0), "dllm_timing_read", h)
+    return list(ms), list(n)

@@ -153,10 +153,16 @@ struct dllm_handle {
   int32_t* dbg_idx = nullptr;    // [L][T_canvas_max][k]
   float* dbg_x = nullptr;        // [T_canvas_max][d]
   float* dbg_xl = nullptr;       // [L][T_canvas_max][d] residual after each layer
-  int32_t* dbg_force = nullptr;  // [L][T_canvas_max][k] experts to use instead of the router's
+  int32_t* dbg_force = nullptr;  // [L][force_T][k] experts to use instead of the router's
   bool force_routing = false;
+  int force_T = 0;               // token count of the passes the forced routing applies to
 
   std::map<int, Graph> graphs;   // key: B * 2 + mode
+
+  bool timing = false;
+  std::vector<cudaEvent_t> tev;  // [kind][layer][start, stop]
+  double t_ms[DLLM_TIMING_KINDS] = {0, 0};
+  long long t_n[DLLM_TIMING_KINDS] = {0, 0};
 };
 
 namespace {
@@ -307,38 +313,53 @@ cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, i
   return attention_hd<64, 64>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
 }
 
+// Event of (kind, layer, start|stop); recorded only when the pass is timed.
+cudaError_t tmark(dllm_handle* h, bool timed, int kind, int layer, int which) {
+  if (!timed) return cudaSuccess;
+  // External: under stream capture the record becomes an event node of the graph
+  // (a plain record would only express a dependency)
+  return cudaEventRecordWithFlags(h->tev[((size_t)kind * h->c.n_layers + layer) * 2 + which], h->st,
+                                  cudaEventRecordExternal);
+}
+
 template <int BN>
-cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi) {
+cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, bool timed) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
   constexpr int STAGES = BN <= 64 ? 6 : BN <= 128 ? 4 : 2;
+  cudaError_t r;
   {
     GroupedSched s{h->offsets, 2 * F, BN};
     EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-    cudaError_t r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(2 * F / 128, h->E), L.tm_wgu, h->tm_xg[bi], d / 64,
-                                                        1, s, e, nullptr, &h->tm_xg_lo[bi]);
+    if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
+    r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(2 * F / 128, h->E), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e,
+                                            nullptr, &h->tm_xg_lo[bi]);
     if (r != cudaSuccess) return r;
+    if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   }
   GroupedSched s{h->offsets, d, BN};
   EpiDown<BN> e{h->obuf, d};
-  return launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(d / 128, h->E), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
-                                             &h->tm_h_lo[bi]);
+  if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
+  r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(d / 128, h->E), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
+                                          &h->tm_h_lo[bi]);
+  if (r != cudaSuccess) return r;
+  return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
 
-cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N) {
+cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, bool timed) {
   const int bi = moe_bn_index(N, h->E);
   switch (bi) {
-    case 0: return moe_gemms_bn<32>(h, L, bi);
-    case 1: return moe_gemms_bn<64>(h, L, bi);
-    case 2: return moe_gemms_bn<128>(h, L, bi);
-    default: return moe_gemms_bn<256>(h, L, bi);
+    case 0: return moe_gemms_bn<32>(h, L, bi, l, timed);
+    case 1: return moe_gemms_bn<64>(h, L, bi, l, timed);
+    case 2: return moe_gemms_bn<128>(h, L, bi, l, timed);
+    default: return moe_gemms_bn<256>(h, L, bi, l, timed);
   }
 }
 
 // ------------------------------------------------------------------ the pass
 
 int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0, const int* slot, int causal,
-               int splits, int split_keys, bool record) {
+               int splits, int split_keys, bool record, bool timed) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int N = T * h->k;
@@ -369,11 +390,11 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                            sizeof(float) * T * h->E, cudaMemcpyDeviceToDevice, h->st));
         CK(cudaMemcpyAsync(h->dbg_idx + (size_t)l * h->T_canvas_max * h->k, h->tk_idx, sizeof(int32_t) * T * h->k,
                            cudaMemcpyDeviceToDevice, h->st));
-        if (h->force_routing) {
-          force_route_kernel<<<ceil_div(T, 128), 128, 0, h->st>>>(
-              h->rlogits, h->dbg_force + (size_t)l * h->T_canvas_max * h->k, T, h->E, h->k, h->tk_idx, h->tk_w);
-          h->launches++;
-        }
+      }
+      if (h->force_routing && T == h->force_T) {
+        force_route_kernel<<<ceil_div(T, 128), 128, 0, h->st>>>(
+            h->rlogits, h->dbg_force + (size_t)l * h->force_T * h->k, T, h->E, h->k, h->tk_idx, h->tk_w);
+        h->launches++;
       }
     } else {
       dense_route_kernel<<<ceil_div(T, 256), 256, 0, h->st>>>(T, h->tk_idx, h->tk_w);
@@ -383,7 +404,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                                                                h->row_token);
     gather_rows_kernel<<<N, 128, 0, h->st>>>(h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo);
     h->launches += 2;
-    CK(moe_gemms(h, L, N));
+    CK(moe_gemms(h, L, N, l, timed));
     combine_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d);
     h->launches++;
     if (record)
@@ -401,7 +422,8 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
   const int splits = attn_splits(h, B);
   embed_kernel<<<T, 128, 0, h->st>>>(h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x);
   h->launches++;
-  int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0);
+  int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0,
+                     h->timing && mode == 0);
   if (r) return r;
   if (mode == 1) return DLLM_OK;
   if (h->debug) CK(cudaMemcpyAsync(h->dbg_x, h->x, sizeof(float) * T * d, cudaMemcpyDeviceToDevice, h->st));
@@ -491,6 +513,20 @@ int check_device_error(dllm_handle* h) {
     return fail(h, DLLM_E_TIMEOUT, "a kernel gave up a bounded wait (code " + std::to_string(e) + ")");
   }
   return DLLM_OK;
+}
+
+void accumulate_timing(dllm_handle* h) {
+  for (int kind = 0; kind < DLLM_TIMING_KINDS; ++kind)
+    for (int l = 0; l < h->c.n_layers; ++l) {
+      float ms = 0.f;
+      const size_t i = ((size_t)kind * h->c.n_layers + l) * 2;
+      if (cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]) == cudaSuccess) {
+        h->t_ms[kind] += ms;
+        h->t_n[kind] += 1;
+      } else {
+        cudaGetLastError();
+      }
+    }
 }
 
 void drop_graphs(dllm_handle* h) {
@@ -742,6 +778,8 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
 
 void free_all(dllm_handle* h) {
   drop_graphs(h);
+  for (auto& e : h->tev) cudaEventDestroy(e);
+  h->tev.clear();
   for (void* p : h->allocs) cudaFree(p);
   h->allocs.clear();
   if (h->h_remaining) cudaFreeHost(h->h_remaining);
@@ -761,7 +799,7 @@ int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool pro
   CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
   embed_kernel<<<n, 128, 0, h->st>>>(h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x);
   h->launches++;
-  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false);
+  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false, false);
   if (r) return r;
   h->P[req] = n;
   return upload_P(h);
@@ -853,6 +891,7 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
     if ((r = replay_pass(h, B, 0))) return r;
     CK(cudaMemcpyAsync(h->h_remaining, h->d_remaining, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, h->st));
     CK(cudaStreamSynchronize(h->st));
+    if (h->timing) accumulate_timing(h);
     all_done = true;
     for (int b = 0; b < B; ++b) {
       if (h->h_remaining[b] == 0 && done_at[b] < 0) done_at[b] = s + 1;
@@ -949,15 +988,13 @@ int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T) {
     h->force_routing = false;
     return DLLM_OK;
   }
-  if (T < 1 || T > h->T_canvas_max) return fail(h, DLLM_E_INVAL, "T out of range");
-  if (!h->dbg_force) DA(h->dbg_force, (size_t)h->c.n_layers * h->T_canvas_max * h->k);
-  for (int l = 0; l < h->c.n_layers; ++l) {
-    for (size_t i = 0; i < (size_t)T * h->k; ++i)
-      if (idx[(size_t)l * T * h->k + i] < 0 || idx[(size_t)l * T * h->k + i] >= h->E)
-        return fail(h, DLLM_E_INVAL, "expert index out of range");
-    CK(cudaMemcpy(h->dbg_force + (size_t)l * h->T_canvas_max * h->k, idx + (size_t)l * T * h->k,
-                  sizeof(int32_t) * T * h->k, cudaMemcpyHostToDevice));
-  }
+  if (T < 1 || T > h->T_max) return fail(h, DLLM_E_INVAL, "T out of range");
+  const size_t n = (size_t)h->c.n_layers * T * h->k;
+  for (size_t i = 0; i < n; ++i)
+    if (idx[i] < 0 || idx[i] >= h->E) return fail(h, DLLM_E_INVAL, "expert index out of range");
+  if (!h->dbg_force) DA(h->dbg_force, (size_t)h->c.n_layers * h->T_max * h->k);
+  CK(cudaMemcpy(h->dbg_force, idx, sizeof(int32_t) * n, cudaMemcpyHostToDevice));
+  h->force_T = T;
   h->force_routing = true;
   return DLLM_OK;
 }
@@ -989,6 +1026,30 @@ int dllm_debug_read(dllm_handle* h, int what, int layer, void* dst, size_t bytes
   if (bytes < need) return fail(h, DLLM_E_INVAL, "debug buffer too small");
   CK(cudaStreamSynchronize(h->st));
   CK(cudaMemcpy(dst, src, need, cudaMemcpyDeviceToHost));
+  return DLLM_OK;
+}
+
+int dllm_set_timing(dllm_handle* h, int on) {
+  if (!h) return DLLM_E_INVAL;
+  if (on && h->tev.empty()) {
+    h->tev.resize((size_t)DLLM_TIMING_KINDS * h->c.n_layers * 2);
+    for (auto& e : h->tev) CK(cudaEventCreate(&e));
+  }
+  h->timing = on != 0;
+  drop_graphs(h);
+  return DLLM_OK;
+}
+
+int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, int reset) {
+  if (!h || !total_ms || !launches) return DLLM_E_INVAL;
+  for (int k = 0; k < DLLM_TIMING_KINDS; ++k) {
+    total_ms[k] = h->t_ms[k];
+    launches[k] = h->t_n[k];
+    if (reset) {
+      h->t_ms[k] = 0;
+      h->t_n[k] = 0;
+    }
+  }
   return DLLM_OK;
 }
 

@@ -329,7 +329,7 @@ class OracleModel:
     def reset(self, req: int = 0):
         self.requests[req] = _Request(self.cfg.n_layers)
 
-    def prefill(self, req: int, prompt: np.ndarray):
+    def prefill(self, req: int, prompt: np.ndarray, rec: Optional[dict] = None):
         """Causal forward over the prompt; its K/V fill the cache at 0..n-1."""
         c = self.cfg
         prompt = np.asarray(prompt, dtype=np.int64)
@@ -339,7 +339,7 @@ class OracleModel:
         pos = np.arange(n)
         allowed = pos[None, :] <= pos[:, None]
         for l in range(c.n_layers):
-            x, k, v = self.layer(l, x, pos, None, None, allowed)
+            x, k, v = self.layer(l, x, pos, None, None, allowed, rec)
             st.k[l], st.v[l] = k, v
         st.P = n
         self.requests[req] = st

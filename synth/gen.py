@@ -183,9 +183,16 @@ def gen_tensor(cfg: ModelConfig, spec: TensorSpec, seed: int | None = None) -> n
     return w.reshape(spec.shape)
 
 
-def gen_weights(cfg: ModelConfig, seed: int | None = None) -> Dict[str, np.ndarray]:
-    """All tensors by name (host memory; meant for the small configurations)."""
-    return {s.name: gen_tensor(cfg, s, seed) for s in tensor_specs(cfg)}
+def gen_weights(cfg: ModelConfig, seed: int | None = None, threads: int = 0) -> Dict[str, np.ndarray]:
+    """All tensors by name (host memory). threads > 1 generates tensors concurrently
+    (numpy releases the GIL inside its array loops); values do not depend on it."""
+    specs = tensor_specs(cfg)
+    if threads <= 1:
+        return {s.name: gen_tensor(cfg, s, seed) for s in specs}
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        arrays = list(ex.map(lambda s: gen_tensor(cfg, s, seed), specs))
+    return {s.name: a for s, a in zip(specs, arrays)}
 
 
 def gen_blob(cfg: ModelConfig, seed: int | None = None) -> np.ndarray:

@@ -30,8 +30,17 @@ def build_pair(cfg, prefix: int, prompt_seed: int, max_ctx: int, max_batch: int 
     den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=max_batch)
     del blob
     prompt = prompt_tokens(cfg.vocab, prompt_seed, prefix)
-    orc.prefill(0, prompt)
+    rec = {}
+    orc.prefill(0, prompt, rec)
+    if not cfg.dense:
+        # the prefix K/V feed every later pass: prefill on the oracle's experts too, so
+        # that a near-tie routed differently in the prompt cannot move the canvas passes
+        den.set_debug(True)
+        den.force_routing(np.stack(rec["topk_idx"]))
     den.prefill(0, prompt)
+    if not cfg.dense:
+        den.force_routing(None)
+        den.set_debug(False)
     return orc, den, prompt
 
 
