@@ -50,7 +50,21 @@ def parse_args():
     ap.add_argument("--workload", default="c3-moe26b-canvas")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    # profiling runs only (smaller captures); the reported workload never uses them
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling)")
+    ap.add_argument("--max-steps", type=int, default=0, help="override the step budget (profiling)")
     return ap.parse_args()
+
+
+def resolve_workload(args):
+    from dataclasses import replace
+    from synth import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.layers:
+        w = replace(w, model=w.model.with_layers(args.layers), name=f"{w.name}-{args.layers}L")
+    if args.max_steps:
+        w = replace(w, max_steps=args.max_steps, name=f"{w.name}-{args.max_steps}steps")
+    return w
 
 
 def load_peaks():
@@ -272,7 +286,7 @@ def run_ours(args):
     from synth.device import device_blob
 
     world, rank, local = dist_setup()
-    w = WORKLOADS[args.workload]
+    w = resolve_workload(args)
     cfg = w.model
     C = cfg.canvas
     max_ctx = w.prefix + w.n_canvases * C
@@ -423,7 +437,7 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = resolve_workload(args)
     C = w.model.canvas
     times, threads, sample = oracle_sample(w, expected_passes(w), reps=args.warmup + args.steps)
     steps = [t[0] for t in times[args.warmup:]]

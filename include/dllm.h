@@ -59,7 +59,7 @@ extern "C" {
 
 typedef struct dllm_handle dllm_handle;
 
-/* Model and capacity. Requirements of this build: d_model % 256 == 0,
+/* Model and capacity. Requirements of this build: d_model % 256 == 0, d_model <= 4096,
  * head_dim in {64, 176}, n_heads * head_dim % 64 == 0, ffn_dim % 64 == 0,
  * vocab % 256 == 0, n_experts <= 256, top_k <= 8 (dense: n_experts = 0, top_k = 1),
  * canvas <= 1024, mask_id = vocab - 1. */
@@ -196,6 +196,7 @@ int dllm_op_gemm_bf16(const uint16_t* A, const uint16_t* B, float* D, int M, int
  * and frees its own partial-result scratch (stream-ordered). */
 int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, int V, int mask_id, float* conf,
                          int32_t* argmax, void* stream);
+
 
 #ifdef __cplusplus
 }

@@ -225,3 +225,4 @@ def dllm_timing_read(h, reset: bool = False):
     n = (ctypes.c_longlong * DLLM_TIMING_KINDS)()
     _check(load().dllm_timing_read(h, ms, n, 1 if reset else 0), "dllm_timing_read", h)
     return list(ms), list(n)
+

@@ -316,10 +316,14 @@ cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, i
 // Event of (kind, layer, start|stop); recorded only when the pass is timed.
 cudaError_t tmark(dllm_handle* h, bool timed, int kind, int layer, int which) {
   if (!timed) return cudaSuccess;
-  // External: under stream capture the record becomes an event node of the graph
-  // (a plain record would only express a dependency)
-  return cudaEventRecordWithFlags(h->tev[((size_t)kind * h->c.n_layers + layer) * 2 + which], h->st,
-                                  cudaEventRecordExternal);
+  cudaEvent_t ev = h->tev[((size_t)kind * h->c.n_layers + layer) * 2 + which];
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t r = cudaStreamIsCapturing(h->st, &cs);
+  if (r != cudaSuccess) return r;
+  // under stream capture the record must be "external" to become an event node of the
+  // graph (a plain record would only express a dependency); outside capture it is plain
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, h->st, cudaEventRecordExternal);
+  return cudaEventRecord(ev, h->st);
 }
 
 template <int BN>
@@ -381,7 +385,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
     h->launches++;
     if (!h->dense) {
-      router_kernel<<<ceil_div(T, kRouterTok), 256, kRouterTok * d * sizeof(float), h->st>>>(
+      router_kernel<<<dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp)), 256, kRouterTok * d * sizeof(float),
+                      h->st>>>(
           h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits);
       topk_kernel<<<ceil_div((long)T * 32, 256), 256, 0, h->st>>>(h->rlogits, T, h->E, h->k, h->tk_idx, h->tk_w);
       h->launches += 2;
@@ -537,7 +542,8 @@ void drop_graphs(dllm_handle* h) {
 
 int validate(const dllm_config* c, std::string* why) {
   auto bad = [&](const char* m) { *why = m; return DLLM_E_INVAL; };
-  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256) return bad("d_model must be a multiple of 256");
+  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 256 || c->d_model > 256 * kRouterMaxChunks)
+    return bad("d_model must be a multiple of 256, at most 4096");
   if (c->head_dim != 64 && c->head_dim != 176) return bad("head_dim must be 64 or 176");
   if (c->n_heads < 1 || c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads) return bad("n_heads % n_kv_heads != 0");
   if ((c->n_heads * c->head_dim) % 64) return bad("n_heads * head_dim must be a multiple of 64");

@@ -71,48 +71,82 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
 
 // ---------------------------------------------------------------- a7: router + top-k
 
-// logits[t][e] = sum_k (x[t][k] * rstd[t] * g[k]) * Wr[e][k], all in fp32. Each block
-// holds kRouterTok normalised rows in shared memory; each warp walks experts.
+// logits[t][e] = sum_k (x[t][k] * rstd[t] * g[k]) * Wr[e][k], all in fp32.
+// Block (blockIdx.x, blockIdx.y) = (kRouterTok tokens, kRouterExp experts): the tokens'
+// normalised rows sit in shared memory; each of the 8 warps owns kRouterExp / 8 experts,
+// its lanes split the d-long dot products in 8-element chunks, and the chunk loop is
+// unrolled (d <= kRouterMaxChunks * 256) so that all of a warp's weight loads are in
+// flight together instead of one dependent load per iteration.
 constexpr int kRouterTok = 4;
-__global__ void router_kernel(const float* __restrict__ x, const float* __restrict__ rstd,
-                              const float* __restrict__ g, const bf16_t* __restrict__ wr, int T, int d, int E,
-                              float* __restrict__ logits) {
+constexpr int kRouterExp = 32;
+constexpr int kRouterMaxChunks = 16;   // d <= 4096
+__global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ x, const float* __restrict__ rstd,
+                                                     const float* __restrict__ g, const bf16_t* __restrict__ wr,
+                                                     int T, int d, int E, float* __restrict__ logits) {
   extern __shared__ float xs[];   // [kRouterTok][d]
   const int t0 = blockIdx.x * kRouterTok;
-  for (int i = threadIdx.x; i < kRouterTok * d; i += blockDim.x) {
-    const int tk = i / d, k = i % d;
+  for (int i = threadIdx.x; i < kRouterTok * d / 4; i += blockDim.x) {
+    const int tk = (4 * i) / d, k = (4 * i) % d;
     const int t = t0 + tk;
-    xs[i] = (t < T) ? x[(long)t * d + k] * rstd[t] * g[k] : 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < T) {
+      const float r = rstd[t];
+      const float4 xv = *reinterpret_cast<const float4*>(x + (long)t * d + k);
+      const float4 gv = *reinterpret_cast<const float4*>(g + k);
+      v = make_float4(xv.x * r * gv.x, xv.y * r * gv.y, xv.z * r * gv.z, xv.w * r * gv.w);
+    }
+    reinterpret_cast<float4*>(xs)[i] = v;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nw) {
-    float acc[kRouterTok];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int EPW = kRouterExp / 8;   // experts per warp
+  const int e0 = blockIdx.y * kRouterExp + warp * EPW;
+  const int nchunks = d / 256;
+  float acc[EPW][kRouterTok];
 #pragma unroll
-    for (int i = 0; i < kRouterTok; ++i) acc[i] = 0.f;
-    const bf16_t* w = wr + (long)e * d;
-    for (int k = lane * 8; k < d; k += 256) {
-      const uint4 v = *reinterpret_cast<const uint4*>(w + k);
-      const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
-      float wf[8];
+  for (int j = 0; j < EPW; ++j)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        wf[2 * i] = __uint_as_float(ww[i] << 16);
-        wf[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
+    for (int tk = 0; tk < kRouterTok; ++tk) acc[j][tk] = 0.f;
+#pragma unroll
+  for (int c = 0; c < kRouterMaxChunks; ++c) {
+    if (c < nchunks) {
+      const int k = c * 256 + lane * 8;
+      uint4 wv[EPW];
+#pragma unroll
+      for (int j = 0; j < EPW; ++j) {
+        const int e = e0 + j;
+        wv[j] = e < E ? *reinterpret_cast<const uint4*>(wr + (long)e * d + k) : make_uint4(0, 0, 0, 0);
       }
+      float xf[kRouterTok][8];
 #pragma unroll
       for (int tk = 0; tk < kRouterTok; ++tk) {
-        const float* xr = xs + tk * d + k;
+        const float4 a = *reinterpret_cast<const float4*>(xs + tk * d + k);
+        const float4 b = *reinterpret_cast<const float4*>(xs + tk * d + k + 4);
+        xf[tk][0] = a.x; xf[tk][1] = a.y; xf[tk][2] = a.z; xf[tk][3] = a.w;
+        xf[tk][4] = b.x; xf[tk][5] = b.y; xf[tk][6] = b.z; xf[tk][7] = b.w;
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[tk] = fmaf(wf[i], xr[i], acc[tk]);
+      for (int j = 0; j < EPW; ++j) {
+        const uint32_t ww[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float w0 = __uint_as_float(ww[i] << 16), w1 = __uint_as_float(ww[i] & 0xFFFF0000u);
+#pragma unroll
+          for (int tk = 0; tk < kRouterTok; ++tk) {
+            acc[j][tk] = fmaf(w0, xf[tk][2 * i], acc[j][tk]);
+            acc[j][tk] = fmaf(w1, xf[tk][2 * i + 1], acc[j][tk]);
+          }
+        }
       }
     }
+  }
+#pragma unroll
+  for (int j = 0; j < EPW; ++j)
 #pragma unroll
     for (int tk = 0; tk < kRouterTok; ++tk) {
-      const float s = warp_sum(acc[tk]);
-      if (lane == 0 && t0 + tk < T) logits[(long)(t0 + tk) * E + e] = s;
+      const float s = warp_sum(acc[j][tk]);
+      if (lane == 0 && t0 + tk < T && e0 + j < E) logits[(long)(t0 + tk) * E + e0 + j] = s;
     }
-  }
 }
 
 // Top-k experts per token by logit (ties to the lower expert) and gates = softmax of
