@@ -197,6 +197,23 @@ int dllm_op_gemm_bf16(const uint16_t* A, const uint16_t* B, float* D, int M, int
 int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, int V, int mask_id, float* conf,
                          int32_t* argmax, void* stream);
 
+/* dllm_op_lm_head_conf without any device allocation. The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory while they
+ * run, e.g. a host process that reserves the whole device for its own allocator under
+ * a fixed budget and forbids other cudaMalloc calls, or a path where an allocation's
+ * implicit synchronisation or failure is not acceptable.
+ * Arguments and results are those of dllm_op_lm_head_conf (caller-owned device buffers).
+ * Scratch: one fixed device array inside the library (3 MiB), present on every GPU that
+ * loads the library until the process exits. Limits: T <= 1024 rows, V <= 65536;
+ * larger sizes return DLLM_E_INVAL and print the limit to stderr.
+ * The first call on a device looks up that array's device address (once per device,
+ * with the device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and it keeps the last call's contents:
+ * calls that may overlap on the GPU (other streams, other host threads) race on it, so
+ * order them on one stream. Calls no cudaMalloc, cudaFree or allocating library
+ * routine. */
+int dllm_op_lm_head_conf_noalloc(const uint16_t* y, const uint16_t* head, int T, int d, int V, int mask_id,
+                                 float* conf, int32_t* argmax, void* stream);
 
 #ifdef __cplusplus
 }

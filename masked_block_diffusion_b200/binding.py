@@ -35,7 +35,8 @@ EXPORTS = [
     "dllm_create", "dllm_prefill", "dllm_denoise_step", "dllm_generate_block", "dllm_append_kv",
     "dllm_generate", "dllm_reset", "dllm_prefix_len", "dllm_check", "dllm_launch_count",
     "dllm_set_debug", "dllm_debug_read", "dllm_debug_force_routing", "dllm_last_error", "dllm_destroy",
-    "dllm_op_gemm_bf16", "dllm_op_lm_head_conf", "dllm_set_timing", "dllm_timing_read",
+    "dllm_op_gemm_bf16", "dllm_op_lm_head_conf", "dllm_op_lm_head_conf_noalloc", "dllm_set_timing",
+    "dllm_timing_read",
 ]
 DLLM_TIMING_GATE_UP = 0
 DLLM_TIMING_DOWN = 1
@@ -95,6 +96,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dllm_destroy": (None, [_vp]),
         "dllm_op_gemm_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
         "dllm_op_lm_head_conf": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+        "dllm_op_lm_head_conf_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
         "dllm_set_timing": (_i, [_vp, _i]),
         "dllm_timing_read": (_i, [_vp, _vp, _vp, _i]),
     }
@@ -226,3 +228,8 @@ def dllm_timing_read(h, reset: bool = False):
     _check(load().dllm_timing_read(h, ms, n, 1 if reset else 0), "dllm_timing_read", h)
     return list(ms), list(n)
 
+
+def dllm_op_lm_head_conf_noalloc(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, argmax_ptr, stream_ptr):
+    """The fused LM head on a fixed in-library scratch array (no device allocation)."""
+    _check(load().dllm_op_lm_head_conf_noalloc(_vp(y_ptr), _vp(head_ptr), T, d, V, mask_id, _vp(conf_ptr),
+                                               _vp(argmax_ptr), _vp(stream_ptr)), "dllm_op_lm_head_conf_noalloc")

@@ -17,6 +17,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -1126,3 +1127,86 @@ int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free LM head
+//
+// The same fused LM head as dllm_op_lm_head_conf, for callers that cannot allocate
+// device memory at call time: processes whose device memory is reserved up front under
+// a fixed budget (a serving host that hands the whole device to its own allocator and
+// refuses foreign cudaMalloc calls), or code paths where an allocation's implicit
+// synchronisation or possible failure is not acceptable. Its scratch (the per-row,
+// per-vocabulary-tile partials and the error word) lives in one fixed device array in
+// this file instead: every GPU that loads the library holds it, 3 MiB plus a few bytes,
+// until the process exits.
+
+namespace {
+
+constexpr int kNoAllocMaxRows = 1024;    // rows T per call
+constexpr int kNoAllocMaxTiles = 256;    // vocabulary tiles of 256: V <= 65536
+constexpr size_t kNoAllocPartials = (size_t)kNoAllocMaxRows * kNoAllocMaxTiles;
+// layout: m[partials] fp32 | s[partials] fp32 | idx[partials] int32 | error word (+ pad)
+constexpr size_t kNoAllocBytes = kNoAllocPartials * 12 + 256;
+
+// Host code sees only a stand-in for this name; the device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device.
+cudaError_t noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = reinterpret_cast<unsigned char*>(g_noalloc_addr[dev]);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int dllm_op_lm_head_conf_noalloc(const uint16_t* y, const uint16_t* head, int T, int d, int V,
+                                            int mask_id, float* conf, int32_t* argmax, void* stream) {
+  if (!y || !head || !conf || !argmax || T < 1 || d < 64 || d % 64 || V < 256 || V % 256) return DLLM_E_INVAL;
+  if (T > kNoAllocMaxRows || V / 256 > kNoAllocMaxTiles) {
+    fprintf(stderr,
+            "dllm_op_lm_head_conf_noalloc: T=%d, V=%d exceed the fixed scratch (at most %d rows and a "
+            "vocabulary of %d)\n",
+            T, V, kNoAllocMaxRows, kNoAllocMaxTiles * 256);
+    return DLLM_E_INVAL;
+  }
+  dllm_handle tmp;
+  tmp.st = reinterpret_cast<cudaStream_t>(stream);
+  dllm_handle* h = &tmp;
+  unsigned char* base = nullptr;
+  CK(noalloc_scratch(&base));
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, y, T, d, 128) || !make_tmap(&tb, head, V, d, 256)) return DLLM_E_INVAL;
+  const int nvt = V / 256;
+  float* pm = reinterpret_cast<float*>(base);
+  float* ps = pm + kNoAllocPartials;
+  int32_t* pi = reinterpret_cast<int32_t*>(ps + kNoAllocPartials);
+  int* err = reinterpret_cast<int*>(pi + kNoAllocPartials);
+  // the partials are fully rewritten for rows < T; only the error word must start at zero
+  CK(cudaMemsetAsync(err, 0, sizeof(int), tmp.st));
+  tmp.d_err = err;
+  const int mt = ceil_div(T, 128);
+  DenseSched s{T, mt, 256};
+  EpiLMHead<256> e{pm, ps, pi, nvt, mask_id};
+  cudaError_t r = launch_gemm<256, 4, 1, kSplitNone>(h, dim3(mt * nvt), ta, tb, d / 64, 0, s, e);
+  if (r == cudaSuccess) {
+    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax);
+    r = cudaGetLastError();
+  }
+  tmp.d_err = nullptr;
+  return r == cudaSuccess ? DLLM_OK : DLLM_E_CUDA;
+}
