@@ -257,13 +257,8 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
-    if world == 1:
-        return v
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([float(v)], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from masked_block_diffusion_b200.replicas import max_over_ranks as _max
+    return float(v) if world == 1 else _max(v, "cuda")
 
 
 def prefill_flops(cfg, n):
@@ -345,29 +340,31 @@ def run_ours(args):
     launches = binding.dllm_launch_count(h) - launches0
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), world)
     gen_ms = sum(a.elapsed_time(b) for a, b in gen_events)
-    kms, kn = binding.dllm_timing_read(h, reset=True)
+    kms, kn, kbytes = binding.dllm_timing_read(h, reset=True)
     barrier(world)
 
-    tokens = world * args.steps * w.n_canvases * C
-    value = tokens / (elapsed_ms / 1e3)
+    from masked_block_diffusion_b200.replicas import aggregate_rate
+    value = aggregate_rate(args.steps * w.n_canvases * C, world, elapsed_ms / 1e3)
     passes_per_canvas = passes / (args.steps * w.n_canvases)
     peaks, peak_src = load_peaks()
 
     # dominant kernel: the grouped gate/up GEMM (expert weights streamed from HBM)
-    gu_ms = kms[binding.DLLM_TIMING_GATE_UP] / max(1, kn[binding.DLLM_TIMING_GATE_UP])
-    if kn[binding.DLLM_TIMING_GATE_UP] == 0 or gu_ms <= 0:
+    GU, DN = binding.DLLM_TIMING_GATE_UP, binding.DLLM_TIMING_DOWN
+    if kn[GU] == 0 or kms[GU] <= 0:
         raise RuntimeError("no gate/up GEMM launch was timed")
-    gu_bytes = gate_up_bytes(cfg, C)
-    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    gu_ms = kms[GU] / kn[GU]
+    gu_bytes = kbytes[GU] / kn[GU]          # mean algorithmic bytes per launch (routed experts)
+    achieved = kbytes[GU] / (kms[GU] / 1e3) / 1e9
     peak_hbm = float(peaks["hbm_gbs"])
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_hbm, "unit": "GB/s",
                 "frac": round(achieved / peak_hbm, 4), "traffic": recorded_traffic(),
                 "kernel": "grouped expert gate/up GEMM + SwiGLU (tcgen05, one launch per layer)",
-                "bytes_per_launch": gu_bytes, "avg_launch_ms": round(gu_ms, 5),
-                "launches_timed": kn[binding.DLLM_TIMING_GATE_UP],
+                "bytes_per_launch": round(gu_bytes), "bytes_per_launch_all_experts": gate_up_bytes(cfg, C),
+                "avg_launch_ms": round(gu_ms, 5), "launches_timed": kn[GU],
+                "bytes_note": "weights of the experts each launch routed to + token pair rows + SwiGLU output",
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
-    dn_ms = max(1e-9, kms[binding.DLLM_TIMING_DOWN] / max(1, kn[binding.DLLM_TIMING_DOWN]))
-    dn_bytes = max(1, cfg.n_experts) * cfg.d_model * cfg.ffn_dim * 2 + C * cfg.top_k * (cfg.ffn_dim * 4 + cfg.d_model * 4)
+    dn_ms = max(1e-9, kms[DN] / max(1, kn[DN]))
+    dn_gbs = kbytes[DN] / max(1e-9, kms[DN] / 1e3) / 1e9
 
     step_flops = prefill_flops(cfg, w.prefix) + w.n_canvases * (
         passes_per_canvas * pass_flops(cfg, C, w.prefix, C) + pass_flops(cfg, C, w.prefix, 0))
@@ -387,7 +384,10 @@ def run_ours(args):
         "step_tc_note": (f"algorithmic flops per step / step time / sustained bf16 peak {tc_peak} TFLOP/s "
                          f"({peak_src}); batch 1 is HBM-bound on expert weights"),
         "roofline": roofline,
-        "down_gemm": {"avg_launch_ms": round(dn_ms, 5), "achieved_gbs": round(dn_bytes / (dn_ms / 1e3) / 1e9, 1)},
+        "down_gemm": {"avg_launch_ms": round(dn_ms, 5), "achieved_gbs": round(dn_gbs, 1),
+                      "bytes_per_launch": round(kbytes[DN] / max(1, kn[DN]))},
+        "experts_routed_per_layer": round((kbytes[GU] / kn[GU] - C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 4)
+                                          / (2 * cfg.ffn_dim * cfg.d_model * 2), 2),
         "gpu_launches": int(launches),
         "clocks": clk,
     }
