@@ -169,14 +169,16 @@ int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T);
 /* Kernel timing: with timing on, every later canvas pass brackets each layer's grouped
  * gate/up GEMM and grouped down GEMM with CUDA events (recorded inside the pass's CUDA
  * graph) and the elapsed times are summed per kind after each pass of
- * dllm_generate_block. dllm_timing_read fills total_ms[kind] and launches[kind]
- * (arrays of DLLM_TIMING_KINDS) and, if reset, zeroes the sums. Toggling timing drops
- * captured graphs. */
+ * dllm_generate_block. dllm_timing_read fills total_ms[kind], launches[kind] and
+ * bytes[kind] (arrays of DLLM_TIMING_KINDS): bytes are the launches' algorithmic HBM
+ * bytes, i.e. the weights of the experts each layer routed to plus the token operand
+ * rows read and the outputs written. If reset, the sums are zeroed. Toggling timing
+ * drops captured graphs. */
 #define DLLM_TIMING_GATE_UP 0
 #define DLLM_TIMING_DOWN 1
 #define DLLM_TIMING_KINDS 2
 int dllm_set_timing(dllm_handle* h, int on);
-int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, int reset);
+int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, double* bytes, int reset);
 
 const char* dllm_last_error(const dllm_handle* h);
 void dllm_destroy(dllm_handle* h);

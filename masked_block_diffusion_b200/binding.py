@@ -98,7 +98,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dllm_op_lm_head_conf": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
         "dllm_op_lm_head_conf_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
         "dllm_set_timing": (_i, [_vp, _i]),
-        "dllm_timing_read": (_i, [_vp, _vp, _vp, _i]),
+        "dllm_timing_read": (_i, [_vp, _vp, _vp, _vp, _i]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -225,8 +225,9 @@ def dllm_set_timing(h, on: bool):
 def dllm_timing_read(h, reset: bool = False):
     ms = (ctypes.c_double * DLLM_TIMING_KINDS)()
     n = (ctypes.c_longlong * DLLM_TIMING_KINDS)()
-    _check(load().dllm_timing_read(h, ms, n, 1 if reset else 0), "dllm_timing_read", h)
-    return list(ms), list(n)
+    b = (ctypes.c_double * DLLM_TIMING_KINDS)()
+    _check(load().dllm_timing_read(h, ms, n, b, 1 if reset else 0), "dllm_timing_read", h)
+    return list(ms), list(n), list(b)
 
 
 def dllm_op_lm_head_conf_noalloc(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, argmax_ptr, stream_ptr):

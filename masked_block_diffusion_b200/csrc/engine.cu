@@ -89,6 +89,7 @@ struct dllm_handle {
   int E = 1, k = 1;          // experts and top-k as run (dense: 1, 1)
   bool dense = true;
   int qkv_heads = 0;
+  int num_sms = 148;
   long long launches = 0;
   std::vector<void*> allocs;
 
@@ -164,6 +165,12 @@ struct dllm_handle {
   std::vector<cudaEvent_t> tev;  // [kind][layer][start, stop]
   double t_ms[DLLM_TIMING_KINDS] = {0, 0};
   long long t_n[DLLM_TIMING_KINDS] = {0, 0};
+  double t_bytes[DLLM_TIMING_KINDS] = {0, 0};   // algorithmic bytes of the timed launches
+  int32_t* routed = nullptr;        // [E] experts with tokens in the current layer
+  int32_t* n_routed = nullptr;      // [1]
+  int32_t* chunk_prefix = nullptr;  // [E+1] chunk-count prefix over the routed experts
+  int32_t* routed_stat = nullptr;   // [L] n_routed per layer of the last timed pass
+  int last_T = 0;                   // tokens of the last timed pass
 };
 
 namespace {
@@ -215,11 +222,11 @@ int dalloc(dllm_handle* h, T** p, size_t count) {
 int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
 
 int moe_bn_index(int N, int E) {
-  // token chunk width: the smallest width holding 1.5x the mean tokens per expert
+  // token chunk width of the grouped GEMMs: 64, or 128 once the mean tokens per expert
+  // pass 64 (prefill, large batches). Routing is often far from uniform, and every chunk
+  // is its own work item, so a skewed expert costs more items rather than a long pole.
   const double mean = (double)N / (double)E;
-  for (int i = 0; i < 3; ++i)
-    if (mean * 1.5 <= kMoeBN[i]) return i;
-  return 3;
+  return mean <= 64.0 ? 1 : 2;
 }
 
 int attn_splits(const dllm_handle* h, int B) {
@@ -334,18 +341,18 @@ cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, bool ti
   constexpr int STAGES = BN <= 64 ? 6 : BN <= 128 ? 4 : 2;
   cudaError_t r;
   {
-    GroupedSched s{h->offsets, 2 * F, BN};
+    PersistentGroupedSched s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
     EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
     if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-    r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(2 * F / 128, h->E), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e,
+    r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e,
                                             nullptr, &h->tm_xg_lo[bi]);
     if (r != cudaSuccess) return r;
     if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   }
-  GroupedSched s{h->offsets, d, BN};
+  PersistentGroupedSched s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
   EpiDown<BN> e{h->obuf, d};
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(d / 128, h->E), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
+  r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
                                           &h->tm_h_lo[bi]);
   if (r != cudaSuccess) return r;
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
@@ -354,10 +361,8 @@ cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, bool ti
 cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, bool timed) {
   const int bi = moe_bn_index(N, h->E);
   switch (bi) {
-    case 0: return moe_gemms_bn<32>(h, L, bi, l, timed);
     case 1: return moe_gemms_bn<64>(h, L, bi, l, timed);
-    case 2: return moe_gemms_bn<128>(h, L, bi, l, timed);
-    default: return moe_gemms_bn<256>(h, L, bi, l, timed);
+    default: return moe_gemms_bn<128>(h, L, bi, l, timed);
   }
 }
 
@@ -407,7 +412,9 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       h->launches++;
     }
     permute_kernel<<<1, 1024, 34 * h->E * sizeof(int), h->st>>>(h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
-                                                               h->row_token);
+                                                               h->row_token, h->routed, h->n_routed,
+                                                               h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
+                                                               timed ? h->routed_stat + l : nullptr);
     gather_rows_kernel<<<N, 128, 0, h->st>>>(h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo);
     h->launches += 2;
     CK(moe_gemms(h, L, N, l, timed));
@@ -521,14 +528,26 @@ int check_device_error(dllm_handle* h) {
   return DLLM_OK;
 }
 
-void accumulate_timing(dllm_handle* h) {
+// After a timed pass over T tokens: adds each grouped GEMM launch's event time and its
+// algorithmic bytes (weights of the experts the layer routed to, the token operand
+// pair read, the output written).
+void accumulate_timing(dllm_handle* h, int T) {
+  const int L = h->c.n_layers;
+  std::vector<int32_t> nr(L);
+  if (cudaMemcpy(nr.data(), h->routed_stat, sizeof(int32_t) * L, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  const double d = h->c.d_model, F = h->c.ffn_dim, N = (double)T * h->k;
   for (int kind = 0; kind < DLLM_TIMING_KINDS; ++kind)
-    for (int l = 0; l < h->c.n_layers; ++l) {
+    for (int l = 0; l < L; ++l) {
       float ms = 0.f;
-      const size_t i = ((size_t)kind * h->c.n_layers + l) * 2;
+      const size_t i = ((size_t)kind * L + l) * 2;
       if (cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]) == cudaSuccess) {
         h->t_ms[kind] += ms;
         h->t_n[kind] += 1;
+        h->t_bytes[kind] += kind == DLLM_TIMING_GATE_UP ? nr[l] * 2 * F * d * 2 + N * d * 4 + N * F * 4
+                                                        : nr[l] * d * F * 2 + N * F * 4 + N * d * 4;
       } else {
         cudaGetLastError();
       }
@@ -716,6 +735,15 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->tk_idx, (size_t)N);
   DA(h->tk_w, (size_t)N);
   DA(h->offsets, h->E + 1);
+  DA(h->routed, h->E);
+  DA(h->n_routed, 1);
+  DA(h->chunk_prefix, h->E + 1);
+  DA(h->routed_stat, c.n_layers);
+  {
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    CK(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+  }
   DA(h->slot_of, (size_t)N);
   DA(h->row_token, (size_t)N);
   DA(h->xg, (size_t)N * d);
@@ -898,7 +926,7 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
     if ((r = replay_pass(h, B, 0))) return r;
     CK(cudaMemcpyAsync(h->h_remaining, h->d_remaining, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, h->st));
     CK(cudaStreamSynchronize(h->st));
-    if (h->timing) accumulate_timing(h);
+    if (h->timing) accumulate_timing(h, B * C);
     all_done = true;
     for (int b = 0; b < B; ++b) {
       if (h->h_remaining[b] == 0 && done_at[b] < 0) done_at[b] = s + 1;
@@ -1047,14 +1075,16 @@ int dllm_set_timing(dllm_handle* h, int on) {
   return DLLM_OK;
 }
 
-int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, int reset) {
-  if (!h || !total_ms || !launches) return DLLM_E_INVAL;
+int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, double* bytes, int reset) {
+  if (!h || !total_ms || !launches || !bytes) return DLLM_E_INVAL;
   for (int k = 0; k < DLLM_TIMING_KINDS; ++k) {
     total_ms[k] = h->t_ms[k];
     launches[k] = h->t_n[k];
+    bytes[k] = h->t_bytes[k];
     if (reset) {
       h->t_ms[k] = 0;
       h->t_n[k] = 0;
+      h->t_bytes[k] = 0;
     }
   }
   return DLLM_OK;

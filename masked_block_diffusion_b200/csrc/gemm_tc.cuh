@@ -68,6 +68,51 @@ struct GroupedSched {
   }
 };
 
+// Persistent grouped schedule over the routed experts only. One work item is one output
+// tile: (routed expert r, m tile, token chunk of BN). Items of expert r are numbered
+// m_tile * chunks_r + chunk from m_tiles * chunk_prefix[r] on, so the chunks of one
+// weight tile are neighbours: CTAs running them together read that tile from HBM once
+// and from L2 after. CTA c takes items c, c + gridDim.x, ...: every CTA gets the same
+// number of equal-sized tiles whatever the routing skew, and streams them back to back
+// (the next tile's loads overlap this tile's epilogue through the double-buffered
+// accumulator).
+struct PersistentGroupedSched {
+  const int* offsets;        // [E+1] token ranges per expert
+  const int* routed;         // [E] experts with at least one token, ascending
+  const int* n_routed;       // [1]
+  const int* chunk_prefix;   // [n_routed + 1] prefix sums of ceil(count / BN) over routed
+  int rows_per_expert;
+  int m_tiles;
+  int BN;
+  DLLM_DEV int n_items() const { return chunk_prefix[*n_routed] * m_tiles; }
+  DLLM_DEV int count() const {
+    const int n = n_items();
+    return (int)blockIdx.x < n ? (n - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  }
+  DLLM_DEV Tile tile(int j) const {
+    const int i = blockIdx.x + j * gridDim.x;
+    int lo = 0, hi = *n_routed;   // chunk_prefix[lo] * m_tiles <= i < chunk_prefix[hi] * m_tiles
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_prefix[mid] * m_tiles <= i) lo = mid; else hi = mid;
+    }
+    const int e = routed[lo];
+    const int ch = chunk_prefix[lo + 1] - chunk_prefix[lo];
+    const int local = i - chunk_prefix[lo] * m_tiles;
+    const int chunk = local % ch;
+    const int off = offsets[e];
+    const int cnt = offsets[e + 1] - off;
+    Tile t;
+    t.mt = local / ch;
+    t.nt = e;
+    t.a_row = e * rows_per_expert + t.mt * 128;
+    t.b_row = off + chunk * BN;
+    t.m_valid = 128;
+    t.n_valid = min(BN, cnt - chunk * BN);
+    return t;
+  }
+};
+
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
 }

@@ -223,9 +223,14 @@ __global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
 // offsets[E+1]: expert ranges in the sorted order; slot_of[i]: sorted position of
 // assignment i = t*k + j; row_token[slot]: its token. Within an expert, assignments
 // keep their (t, j) order, so the permutation is deterministic.
+// Also lists the experts with at least one assignment (routed[0..n_routed), ascending)
+// with the prefix sums of their chunk counts ceil(count / bn) for the persistent grouped
+// GEMMs, and stores n_routed in *routed_stat when given.
 __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int N, int k, int E,
                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
-                                                       int32_t* __restrict__ row_token) {
+                                                       int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
+                                                       int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
+                                                       int bn, int32_t* __restrict__ routed_stat) {
   extern __shared__ int sh[];
   int* cnt = sh;                 // [E]
   int* base = sh + E;            // [E] running start of each expert
@@ -236,13 +241,21 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
   for (int i = tid; i < N; i += blockDim.x) atomicAdd(&cnt[idx[i]], 1);
   __syncthreads();
   if (tid == 0) {
-    int run = 0;
+    int run = 0, nr = 0, chunks = 0;
     for (int e = 0; e < E; ++e) {
       base[e] = run;
       offsets[e] = run;
       run += cnt[e];
+      if (cnt[e] > 0) {
+        chunk_prefix[nr] = chunks;
+        routed[nr++] = e;
+        chunks += (cnt[e] + bn - 1) / bn;
+      }
     }
     offsets[E] = run;
+    chunk_prefix[nr] = chunks;
+    *n_routed = nr;
+    if (routed_stat) *routed_stat = nr;
   }
   __syncthreads();
   for (int c0 = 0; c0 < N; c0 += blockDim.x) {
