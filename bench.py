@@ -53,6 +53,7 @@ def parse_args():
     # profiling runs only (smaller captures); the reported workload never uses them
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling)")
     ap.add_argument("--max-steps", type=int, default=0, help="override the step budget (profiling)")
+    ap.add_argument("--timing-all", action="store_true", help="time every kernel group (diagnostic)")
     return ap.parse_args()
 
 
@@ -296,7 +297,9 @@ def run_ours(args):
     d_canvas = torch.empty((1, C), dtype=torch.int32, device="cuda")
     torch.cuda.synchronize()
     pol = make_policy(w.policy, w.k, w.tau, w.floor)
-    binding.dllm_set_timing(h, True)
+    # the two grouped expert GEMMs are timed inside the graph (--timing-all: every kernel group)
+    binding.dllm_set_timing(h, (1 << binding.DLLM_TIMING_KINDS) - 1 if args.timing_all
+                            else (1 << binding.DLLM_TIMING_GATE_UP) | (1 << binding.DLLM_TIMING_DOWN))
 
     def step(gen_events=None):
         binding.dllm_reset(h, 0)
@@ -389,6 +392,8 @@ def run_ours(args):
         "experts_routed_per_layer": round((kbytes[GU] / kn[GU] - C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 4)
                                           / (2 * cfg.ffn_dim * cfg.d_model * 2), 2),
         "gpu_launches": int(launches),
+        "kernel_ms_per_pass": {binding.TIMING_NAMES[k]: round(kms[k] / max(1, passes), 4)
+                               for k in range(binding.DLLM_TIMING_KINDS) if kn[k]},
         "clocks": clk,
     }
 
@@ -396,7 +401,7 @@ def run_ours(args):
         prompts = np.ascontiguousarray(prompt_np[None, :])
         toks = np.zeros((1, w.n_canvases * C), dtype=np.int32)
         stp = np.zeros((w.n_canvases,), dtype=np.int32)
-        binding.dllm_set_timing(h, False)
+        binding.dllm_set_timing(h, 0)
         for _ in range(max(1, args.warmup)):
             binding.dllm_generate(h, 1, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
                                   toks.ctypes.data, stp.ctypes.data)

@@ -166,18 +166,28 @@ int dllm_debug_read(dllm_handle* h, int what, int layer, void* dst, size_t bytes
  * DLLM_E_INVAL (dense model, T or an index out of range). */
 int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T);
 
-/* Kernel timing: with timing on, every later canvas pass brackets each layer's grouped
- * gate/up GEMM and grouped down GEMM with CUDA events (recorded inside the pass's CUDA
- * graph) and the elapsed times are summed per kind after each pass of
- * dllm_generate_block. dllm_timing_read fills total_ms[kind], launches[kind] and
- * bytes[kind] (arrays of DLLM_TIMING_KINDS): bytes are the launches' algorithmic HBM
- * bytes, i.e. the weights of the experts each layer routed to plus the token operand
- * rows read and the outputs written. If reset, the sums are zeroed. Toggling timing
- * drops captured graphs. */
+/* Kernel timing: dllm_set_timing(h, kinds) with kinds a bit mask of (1 << DLLM_TIMING_*)
+ * (0 = off). Every later canvas pass then brackets the chosen kernel groups of each
+ * layer with CUDA events (recorded inside the pass's CUDA graph); the elapsed times
+ * are summed per kind after each pass of dllm_generate_block. dllm_timing_read fills
+ * total_ms[kind], launches[kind] and bytes[kind] (arrays of DLLM_TIMING_KINDS); bytes
+ * are filled for the two grouped GEMMs: the launches' algorithmic HBM bytes, i.e. the
+ * weights of the experts each layer routed to plus the token operand rows read and the
+ * outputs written. If reset, the sums are zeroed. Changing the mask drops captured
+ * graphs. Kinds: grouped gate/up GEMM; grouped down GEMM; attention (+ split merge);
+ * QKV GEMM; O GEMM; routing (pre-FFN RMSNorm, router, top-k, permute, gather);
+ * combine of the expert outputs (with the next RMSNorm fused into it);
+ * LM head (final RMSNorm, LM-head GEMM, merge, commit; one per pass). */
 #define DLLM_TIMING_GATE_UP 0
 #define DLLM_TIMING_DOWN 1
-#define DLLM_TIMING_KINDS 2
-int dllm_set_timing(dllm_handle* h, int on);
+#define DLLM_TIMING_ATTN 2
+#define DLLM_TIMING_QKV 3
+#define DLLM_TIMING_OPROJ 4
+#define DLLM_TIMING_ROUTE 5
+#define DLLM_TIMING_NORM 6
+#define DLLM_TIMING_HEAD 7
+#define DLLM_TIMING_KINDS 8
+int dllm_set_timing(dllm_handle* h, int kinds);
 int dllm_timing_read(dllm_handle* h, double* total_ms, long long* launches, double* bytes, int reset);
 
 const char* dllm_last_error(const dllm_handle* h);

@@ -40,7 +40,15 @@ EXPORTS = [
 ]
 DLLM_TIMING_GATE_UP = 0
 DLLM_TIMING_DOWN = 1
-DLLM_TIMING_KINDS = 2
+DLLM_TIMING_ATTN = 2
+DLLM_TIMING_QKV = 3
+DLLM_TIMING_OPROJ = 4
+DLLM_TIMING_ROUTE = 5
+DLLM_TIMING_NORM = 6
+DLLM_TIMING_HEAD = 7
+DLLM_TIMING_KINDS = 8
+TIMING_NAMES = ["gate_up_gemm", "down_gemm", "attention", "qkv_gemm", "o_gemm", "routing", "norm_combine",
+                "lm_head_commit"]
 
 
 class dllm_config(ctypes.Structure):
@@ -218,8 +226,9 @@ def dllm_op_lm_head_conf(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, argmax_ptr
                                        _vp(argmax_ptr), _vp(stream_ptr)), "dllm_op_lm_head_conf")
 
 
-def dllm_set_timing(h, on: bool):
-    _check(load().dllm_set_timing(h, 1 if on else 0), "dllm_set_timing", h)
+def dllm_set_timing(h, kinds: int):
+    """kinds: bit mask of (1 << DLLM_TIMING_*); 0 switches timing off."""
+    _check(load().dllm_set_timing(h, int(kinds)), "dllm_set_timing", h)
 
 
 def dllm_timing_read(h, reset: bool = False):

@@ -44,8 +44,10 @@ struct AttnSmem {
   static constexpr int kTotal = kQ + 4 * kKV;
 };
 
+// 3 CTAs (12 warps) per SM: Q stays in shared memory and is re-read by ldmatrix per key
+// block, which keeps the O accumulators, S tile and temporaries within 170 registers.
 template <int HD, int BK>
-__global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
+__global__ void __launch_bounds__(128, 3) attn_kernel(AttnParams p) {
   static_assert(HD % 16 == 0 && BK % 16 == 0, "shape");
   using S = AttnSmem<HD, BK>;
   constexpr int NT = BK / 8;      // S n-tiles per warp
@@ -103,7 +105,6 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
   const int qpos_a = P0 + q_start + row0 + g;   // absolute positions of this thread's rows
   const int qpos_b = qpos_a + 8;
 
-  uint32_t qf[KS][4];
   float o[ON][4];
 #pragma unroll
   for (int i = 0; i < ON; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
@@ -119,14 +120,6 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    if (blk == 0) {
-#pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        const int r = row0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int c = kk * 16 + 8 * (lane >> 4);
-        ldmatrix_x4(qf[kk], smem_u32(sQ + r * S::kStride + c));
-      }
-    }
     const bf16_t* kb = sK + buf * BK * S::kStride;
     const bf16_t* vb = sV + buf * BK * S::kStride;
 
@@ -135,14 +128,20 @@ __global__ void __launch_bounds__(128) attn_kernel(AttnParams p) {
     for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
+      uint32_t qf[4];
+      {
+        const int r = row0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int c = kk * 16 + 8 * (lane >> 4);
+        ldmatrix_x4(qf, smem_u32(sQ + r * S::kStride + c));
+      }
 #pragma unroll
       for (int np = 0; np < NT / 2; ++np) {
         uint32_t kr[4];
         const int key = np * 16 + (lane & 7) + 8 * (lane >> 4);
         const int c = kk * 16 + 8 * ((lane >> 3) & 1);
         ldmatrix_x4(kr, smem_u32(kb + key * S::kStride + c));
-        mma_bf16_16816(s[2 * np], qf[kk], kr[0], kr[1]);
-        mma_bf16_16816(s[2 * np + 1], qf[kk], kr[2], kr[3]);
+        mma_bf16_16816(s[2 * np], qf, kr[0], kr[1]);
+        mma_bf16_16816(s[2 * np + 1], qf, kr[2], kr[3]);
       }
     }
     // scale, mask, block row maxima

@@ -22,6 +22,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
@@ -48,6 +49,21 @@ EncodeTiledFn encode_fn() {
 
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix, box = 64 columns x box_rows,
 // 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
+// 3-D bf16 tensor map over [d2][d1][d0] (d0 contiguous), box = 64 x b1 x b2, 128-byte swizzle.
+bool make_tmap3(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (d0 * 2) % 16 || b1 == 0 || b1 > 256 || b2 == 0 || b2 > 256)
+    return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -72,6 +88,7 @@ struct LayerW {
   bf16_t* wgu = nullptr;    // [E][2F][d]: per 128-row block, 64 gate rows then the 64 matching up rows
   bf16_t* wd = nullptr;     // [E][d][F]
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd;
+  CUtensorMap tm_k, tm_v;   // this layer's K / V cache as [slot][Hkv][max_ctx] rows of hd
 };
 
 struct Graph {
@@ -134,6 +151,8 @@ struct dllm_handle {
   bf16_t* hbuf_lo = nullptr;
   CUtensorMap tm_y, tm_ao, tm_xg[4], tm_h[4];
   CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
+  CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
+  bool attn_tc = false;     // canvas passes use the tensor-core attention
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
   int32_t* d_P = nullptr;    // [max_batch]
@@ -163,9 +182,10 @@ struct dllm_handle {
 
   bool timing = false;
   std::vector<cudaEvent_t> tev;  // [kind][layer][start, stop]
-  double t_ms[DLLM_TIMING_KINDS] = {0, 0};
-  long long t_n[DLLM_TIMING_KINDS] = {0, 0};
-  double t_bytes[DLLM_TIMING_KINDS] = {0, 0};   // algorithmic bytes of the timed launches
+  uint32_t tmask = 0;            // kinds timed (bit k = DLLM_TIMING kind k)
+  double t_ms[DLLM_TIMING_KINDS] = {};
+  long long t_n[DLLM_TIMING_KINDS] = {};
+  double t_bytes[DLLM_TIMING_KINDS] = {};   // algorithmic bytes of the timed launches
   int32_t* routed = nullptr;        // [E] experts with tokens in the current layer
   int32_t* n_routed = nullptr;      // [1]
   int32_t* chunk_prefix = nullptr;  // [E+1] chunk-count prefix over the routed experts
@@ -230,6 +250,13 @@ int moe_bn_index(int N, int E) {
 }
 
 int attn_splits(const dllm_handle* h, int B) {
+  if (h->attn_tc) {
+    // tensor-core kernel: one CTA per SM, aim at a single full wave
+    const int group = h->c.n_heads / h->c.n_kv_heads;
+    const int ctas = ceil_div((long)h->c.canvas * group, 128) * h->c.n_kv_heads * B;
+    int s = h->num_sms / ctas;
+    return s < 1 ? 1 : (s > 16 ? 16 : s);
+  }
   const int qblocks = ceil_div(h->c.canvas, 64);
   const int ctas = qblocks * h->c.n_heads * B;
   int s = ceil_div(2 * 148, ctas);
@@ -314,16 +341,65 @@ cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq
   return cudaGetLastError();
 }
 
+template <int HD>
+cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, int splits, int split_keys) {
+  const auto& c = h->c;
+  AttnTcParams p;
+  p.out = h->ao;
+  p.out_lo = h->ao_lo;
+  p.part_o = h->apart;
+  p.part_lse = h->alse;
+  p.pos0 = h->d_P;
+  p.slot = h->d_slot;
+  p.tok_per_req = c.canvas;
+  p.T = T;
+  p.H = c.n_heads;
+  p.Hkv = c.n_kv_heads;
+  p.group = c.n_heads / c.n_kv_heads;
+  p.max_ctx = c.max_ctx;
+  p.n_splits = splits;
+  p.split_keys = split_keys;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  p.err = h->d_err;
+  constexpr int smem = AttnTcCfg<HD>::kTotal;
+  cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (r != cudaSuccess) return r;
+  dim3 grid(ceil_div((long)c.canvas * p.group, 128), c.n_kv_heads, nreq * splits);
+  attn_tc_kernel<HD><<<grid, 192, smem, h->st>>>(h->tm_q3, L.tm_k, L.tm_v, p);
+  h->launches++;
+  if (splits > 1) {
+    AttnParams m;
+    m.out = h->ao;
+    m.out_lo = h->ao_lo;
+    m.part_o = h->apart;
+    m.part_lse = h->alse;
+    m.pos0 = h->d_P;
+    m.tok_per_req = c.canvas;
+    m.T = T;
+    m.H = c.n_heads;
+    m.n_splits = splits;
+    m.split_keys = split_keys;
+    attn_merge_kernel<HD><<<ceil_div((long)T * c.n_heads * 32, 256), 256, 0, h->st>>>(m);
+    h->launches++;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
-                      const int* slot, int causal, int splits, int split_keys) {
+                      const int* slot, int causal, int splits, int split_keys, const LayerW* L = nullptr) {
+  if (!causal && h->attn_tc && L) {   // the bidirectional canvas pass on the tensor cores
+    if (h->c.head_dim == 176) return attention_tc_hd<176>(h, *L, T, nreq, splits, split_keys);
+    return attention_tc_hd<64>(h, *L, T, nreq, splits, split_keys);
+  }
   if (h->c.head_dim == 176)
     return attention_hd<176, 32>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
   return attention_hd<64, 64>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
 }
 
 // Event of (kind, layer, start|stop); recorded only when the pass is timed.
-cudaError_t tmark(dllm_handle* h, bool timed, int kind, int layer, int which) {
-  if (!timed) return cudaSuccess;
+cudaError_t tmark(dllm_handle* h, uint32_t tmask, int kind, int layer, int which) {
+  if (!(tmask & (1u << kind))) return cudaSuccess;
   cudaEvent_t ev = h->tev[((size_t)kind * h->c.n_layers + layer) * 2 + which];
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   cudaError_t r = cudaStreamIsCapturing(h->st, &cs);
@@ -335,7 +411,7 @@ cudaError_t tmark(dllm_handle* h, bool timed, int kind, int layer, int which) {
 }
 
 template <int BN>
-cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, bool timed) {
+cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, uint32_t timed) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
   constexpr int STAGES = BN <= 64 ? 6 : BN <= 128 ? 4 : 2;
@@ -358,7 +434,7 @@ cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, bool ti
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
 
-cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, bool timed) {
+cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t timed) {
   const int bi = moe_bn_index(N, h->E);
   switch (bi) {
     case 1: return moe_gemms_bn<64>(h, L, bi, l, timed);
@@ -369,7 +445,7 @@ cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, bool timed)
 // ------------------------------------------------------------------ the pass
 
 int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0, const int* slot, int causal,
-               int splits, int split_keys, bool record, bool timed) {
+               int splits, int split_keys, bool record, uint32_t timed, const float* final_gain) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int N = T * h->k;
@@ -377,10 +453,17 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     const LayerW& L = h->L[l];
     bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
     bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
-    rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
-    h->launches++;
+    if (l == 0) {   // later layers get this norm from the previous layer's combine
+      rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
+      h->launches++;
+    }
+    CK(tmark(h, timed, DLLM_TIMING_QKV, l, 0));
     CK(qkv_gemm(h, L, kc, vc, T, pos0, slot, tok_per_req));
-    CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys));
+    CK(tmark(h, timed, DLLM_TIMING_QKV, l, 1));
+    CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 0));
+    CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys, &L));
+    CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 1));
+    CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 0));
     {
       EpiResidual<64> e{h->x, d};
       const int mt = ceil_div(T, 128);
@@ -388,6 +471,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       CK((launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, c.n_heads * c.head_dim / 64, 0,
                                          s, e, &h->tm_ao_lo)));
     }
+    CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 1));
+    CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 0));
     rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
     h->launches++;
     if (!h->dense) {
@@ -417,9 +502,17 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                                                                timed ? h->routed_stat + l : nullptr);
     gather_rows_kernel<<<N, 128, 0, h->st>>>(h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo);
     h->launches += 2;
+    CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
     CK(moe_gemms(h, L, N, l, timed));
-    combine_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d);
+    CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
+    const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
+    if (next_gain)
+      combine_norm_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d, next_gain, c.rms_eps,
+                                                h->y, h->y_lo);
+    else
+      combine_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d);
     h->launches++;
+    CK(tmark(h, timed, DLLM_TIMING_NORM, l, 1));
     if (record)
       CK(cudaMemcpyAsync(h->dbg_xl + (size_t)l * h->T_canvas_max * d, h->x, sizeof(float) * T * d,
                          cudaMemcpyDeviceToDevice, h->st));
@@ -435,13 +528,13 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
   const int splits = attn_splits(h, B);
   embed_kernel<<<T, 128, 0, h->st>>>(h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x);
   h->launches++;
+  const uint32_t tm = (h->timing && mode == 0) ? h->tmask : 0u;
   int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0,
-                     h->timing && mode == 0);
+                     tm, mode == 0 ? h->final_norm : nullptr);
   if (r) return r;
   if (mode == 1) return DLLM_OK;
   if (h->debug) CK(cudaMemcpyAsync(h->dbg_x, h->x, sizeof(float) * T * d, cudaMemcpyDeviceToDevice, h->st));
-  rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, h->final_norm, d, c.rms_eps, h->y, h->y_lo, nullptr);
-  h->launches++;
+  CK(tmark(h, tm, DLLM_TIMING_HEAD, 0, 0));   // the final RMSNorm ran in the last layer's combine
   const int nvt = c.vocab / 256;
   {
     EpiLMHead<256> e{h->lm_m, h->lm_s, h->lm_i, nvt, c.mask_id};
@@ -456,6 +549,7 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
                                                                  h->d_policy, h->d_step, h->d_remaining, nullptr,
                                                                  nullptr);
   h->launches += 2;
+  CK(tmark(h, tm, DLLM_TIMING_HEAD, 0, 1));
   CK(cudaGetLastError());
   return DLLM_OK;
 }
@@ -539,19 +633,22 @@ void accumulate_timing(dllm_handle* h, int T) {
     return;
   }
   const double d = h->c.d_model, F = h->c.ffn_dim, N = (double)T * h->k;
-  for (int kind = 0; kind < DLLM_TIMING_KINDS; ++kind)
-    for (int l = 0; l < L; ++l) {
+  for (int kind = 0; kind < DLLM_TIMING_KINDS; ++kind) {
+    if (!(h->tmask & (1u << kind))) continue;
+    const int layers = kind == DLLM_TIMING_HEAD ? 1 : L;
+    for (int l = 0; l < layers; ++l) {
       float ms = 0.f;
       const size_t i = ((size_t)kind * L + l) * 2;
-      if (cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]) == cudaSuccess) {
-        h->t_ms[kind] += ms;
-        h->t_n[kind] += 1;
-        h->t_bytes[kind] += kind == DLLM_TIMING_GATE_UP ? nr[l] * 2 * F * d * 2 + N * d * 4 + N * F * 4
-                                                        : nr[l] * d * F * 2 + N * F * 4 + N * d * 4;
-      } else {
+      if (cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]) != cudaSuccess) {
         cudaGetLastError();
+        continue;
       }
+      h->t_ms[kind] += ms;
+      h->t_n[kind] += 1;
+      if (kind == DLLM_TIMING_GATE_UP) h->t_bytes[kind] += nr[l] * 2 * F * d * 2 + N * d * 4 + N * F * 4;
+      if (kind == DLLM_TIMING_DOWN) h->t_bytes[kind] += nr[l] * d * F * 2 + N * F * 4 + N * d * 4;
     }
+  }
 }
 
 void drop_graphs(dllm_handle* h) {
@@ -638,6 +735,14 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   h->E = h->dense ? 1 : c.n_experts;
   h->k = h->dense ? 1 : c.top_k;
   h->qkv_heads = H + 2 * Hkv;
+  {
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    CK(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+  }
+  // tensor-core attention for canvas passes when a query tile of 128 rows holds whole
+  // GQA groups (DLLM_ATTN_LEGACY=1 keeps the warp-MMA kernel, for comparisons)
+  h->attn_tc = (128 % (H / Hkv) == 0) && !getenv("DLLM_ATTN_LEGACY");
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
   // ---- weights
@@ -739,11 +844,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->n_routed, 1);
   DA(h->chunk_prefix, h->E + 1);
   DA(h->routed_stat, c.n_layers);
-  {
-    int dev = 0;
-    CK(cudaGetDevice(&dev));
-    CK(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
-  }
+
   DA(h->slot_of, (size_t)N);
   DA(h->row_token, (size_t)N);
   DA(h->xg, (size_t)N * d);
@@ -757,6 +858,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->lm_i, (size_t)h->T_canvas_max * nvt);
   DA(h->conf, h->T_canvas_max);
   DA(h->argmax, h->T_canvas_max);
+  CK(cudaMemsetAsync(h->q, 0, (size_t)T * qd * 2, h->st));   // padding rows of a query tile read zeros
   CK(cudaMemsetAsync(h->xg, 0, (size_t)N * d * 2, h->st));
   CK(cudaMemsetAsync(h->xg_lo, 0, (size_t)N * d * 2, h->st));
   CK(cudaMemsetAsync(h->hbuf, 0, (size_t)N * F * 2, h->st));
@@ -792,6 +894,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   ok &= make_tmap(&h->tm_ao, h->ao, T, qd, 128);
   ok &= make_tmap(&h->tm_ao_lo, h->ao_lo, T, qd, 128);
   ok &= make_tmap(&h->tm_head, h->head, V, d, 256);
+  if (h->attn_tc) ok &= make_tmap3(&h->tm_q3, h->q, hd, H, T, H / Hkv, 128 / (H / Hkv));
   for (int i = 0; i < 4; ++i) {
     ok &= make_tmap(&h->tm_xg[i], h->xg, N, d, kMoeBN[i]);
     ok &= make_tmap(&h->tm_xg_lo[i], h->xg_lo, N, d, kMoeBN[i]);
@@ -803,6 +906,12 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     ok &= make_tmap(&L.tm_wo, L.wo, d, qd, 64);
     ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
     ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);
+    if (h->attn_tc) {
+      const size_t l = &L - h->L.data();
+      const uint64_t kv_rows = (uint64_t)c.max_batch * Hkv * c.max_ctx;
+      ok &= make_tmap(&L.tm_k, h->kcache + l * h->kv_layer, kv_rows, hd, 64);
+      ok &= make_tmap(&L.tm_v, h->vcache + l * h->kv_layer, kv_rows, hd, 64);
+    }
   }
   if (!ok) return fail(h, DLLM_E_CUDA, "cuTensorMapEncodeTiled failed");
   CK(cudaFuncSetAttribute(reinterpret_cast<const void*>(router_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -834,7 +943,7 @@ int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool pro
   CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
   embed_kernel<<<n, 128, 0, h->st>>>(h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x);
   h->launches++;
-  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false, false);
+  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false, 0u, nullptr);
   if (r) return r;
   h->P[req] = n;
   return upload_P(h);
@@ -1064,13 +1173,14 @@ int dllm_debug_read(dllm_handle* h, int what, int layer, void* dst, size_t bytes
   return DLLM_OK;
 }
 
-int dllm_set_timing(dllm_handle* h, int on) {
+int dllm_set_timing(dllm_handle* h, int kinds) {
   if (!h) return DLLM_E_INVAL;
-  if (on && h->tev.empty()) {
+  if (kinds && h->tev.empty()) {
     h->tev.resize((size_t)DLLM_TIMING_KINDS * h->c.n_layers * 2);
     for (auto& e : h->tev) CK(cudaEventCreate(&e));
   }
-  h->timing = on != 0;
+  h->tmask = (uint32_t)kinds & ((1u << DLLM_TIMING_KINDS) - 1);
+  h->timing = h->tmask != 0;
   drop_graphs(h);
   return DLLM_OK;
 }

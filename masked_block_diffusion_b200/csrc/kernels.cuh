@@ -332,6 +332,60 @@ __global__ void combine_kernel(float* __restrict__ x, const float* __restrict__ 
   }
 }
 
+// combine_kernel followed by the RMSNorm that comes next (the next layer's attention
+// norm, or the final norm before the LM head): x is updated in place, then
+// v = x * rsqrt(mean(x^2) + eps) * g is written as the (hi, lo) bf16 pair. One block per
+// token; the same per-row arithmetic as combine_kernel and rmsnorm_kernel.
+__global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x, const float* __restrict__ o,
+                                                           const int32_t* __restrict__ slot_of,
+                                                           const float* __restrict__ gate, int k, int d,
+                                                           const float* __restrict__ g, float eps,
+                                                           bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo) {
+  const int t = blockIdx.x;
+  float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float w = gate[(long)t * k + j];
+      const float4 v = reinterpret_cast<const float4*>(o + (long)slot_of[(long)t * k + j] * d)[c];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    float4 xv = xr[c];
+    xv.x += acc.x;
+    xv.y += acc.y;
+    xv.z += acc.z;
+    xv.w += acc.w;
+    xr[c] = xv;
+    ss += xv.x * xv.x + xv.y * xv.y + xv.z * xv.z + xv.w * xv.w;
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = rsqrtf(red[0] / (float)d + eps);
+  const float4* gr = reinterpret_cast<const float4*>(g);
+  uint2* yr = reinterpret_cast<uint2*>(y + (long)t * d);
+  uint2* yl = reinterpret_cast<uint2*>(y_lo + (long)t * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    const float4 v = xr[c], gg = gr[c];   // this thread's own writes above
+    uint32_t h0, l0, h1, l1;
+    split_bf16x2(v.x * r * gg.x, v.y * r * gg.y, h0, l0);
+    split_bf16x2(v.z * r * gg.z, v.w * r * gg.w, h1, l1);
+    yr[c] = make_uint2(h0, h1);
+    yl[c] = make_uint2(l0, l1);
+  }
+}
+
 // ---------------------------------------------------------------- a13: LM-head merge
 
 DLLM_DEV void lse_combine(float& m, float& s, int& i, float m2, float s2, int i2) {
