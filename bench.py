@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3-moe26b-canvas")
+    ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     # profiling runs only (smaller captures); the reported workload never uses them
@@ -77,7 +78,7 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_config(w, n_gpus):
+def workload_config(w, n_gpus, batch=None):
     return {
         "workload": f"{w.name}: prompt {w.prefix}, {w.n_canvases} canvas(es) of {w.model.canvas}, "
                     f"{w.model.name} ({w.model.n_layers} layers, d {w.model.d_model}, "
@@ -85,7 +86,7 @@ def workload_config(w, n_gpus):
         "prefix": w.prefix,
         "canvas": w.model.canvas,
         "n_canvases": w.n_canvases,
-        "batch_per_gpu": w.batch,
+        "batch_per_gpu": batch or w.batch,
         "policy": (f"top-{w.k}" if w.policy == "topk" else f"threshold {w.tau} + step-budget floor"),
         "max_steps": w.max_steps,
         "parallelism": "replicas" if n_gpus == 1 else f"replicas x{n_gpus} (independent requests)",
@@ -285,16 +286,18 @@ def run_ours(args):
     w = resolve_workload(args)
     cfg = w.model
     C = cfg.canvas
+    Bq = args.batch or w.batch   # independent requests on this GPU
     max_ctx = w.prefix + w.n_canvases * C
     blob = device_blob(cfg)
-    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=1)
+    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=Bq)
     del blob
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     h, st = den.h, den.stream
-    prompt_np = prompt_tokens(cfg.vocab, w.prompt_seed + rank, w.prefix)   # one request per rank
+    # requests of this rank: seeds prompt_seed + global request id
+    prompt_np = np.stack([prompt_tokens(cfg.vocab, w.prompt_seed + rank * Bq + r, w.prefix) for r in range(Bq)])
     d_prompt = torch.from_numpy(prompt_np).cuda()
-    d_canvas = torch.empty((1, C), dtype=torch.int32, device="cuda")
+    d_canvas = torch.empty((Bq, C), dtype=torch.int32, device="cuda")
     torch.cuda.synchronize()
     pol = make_policy(w.policy, w.k, w.tau, w.floor)
     # the two grouped expert GEMMs are timed inside the graph (--timing-all: every kernel group)
@@ -302,22 +305,23 @@ def run_ours(args):
                             else (1 << binding.DLLM_TIMING_GATE_UP) | (1 << binding.DLLM_TIMING_DOWN))
 
     def step(gen_events=None):
-        binding.dllm_reset(h, 0)
-        binding.dllm_prefill(h, 0, d_prompt.data_ptr(), w.prefix)
+        for r in range(Bq):
+            binding.dllm_reset(h, r)
+            binding.dllm_prefill(h, r, d_prompt[r].data_ptr(), w.prefix)
         passes = 0
         for _ in range(w.n_canvases):
             if gen_events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(st)
-            code, steps = binding.dllm_generate_block(h, 1, w.max_steps, pol, d_canvas.data_ptr())
+            code, steps = binding.dllm_generate_block(h, Bq, w.max_steps, pol, d_canvas.data_ptr())
             if code != 0:
                 raise DllmError(code, "dllm_generate_block", binding.dllm_last_error(h))
             if gen_events is not None:
                 e1 = torch.cuda.Event(enable_timing=True)
                 e1.record(st)
                 gen_events.append((e0, e1))
-            passes += steps[0]
-            binding.dllm_append_kv(h, 1, 0)
+            passes += max(steps)
+            binding.dllm_append_kv(h, Bq, 0)
         return passes
 
     for _ in range(args.warmup):
@@ -347,7 +351,7 @@ def run_ours(args):
     barrier(world)
 
     from masked_block_diffusion_b200.replicas import aggregate_rate
-    value = aggregate_rate(args.steps * w.n_canvases * C, world, elapsed_ms / 1e3)
+    value = aggregate_rate(args.steps * w.n_canvases * C * Bq, world, elapsed_ms / 1e3)
     passes_per_canvas = passes / (args.steps * w.n_canvases)
     peaks, peak_src = load_peaks()
 
@@ -362,15 +366,15 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_hbm, "unit": "GB/s",
                 "frac": round(achieved / peak_hbm, 4), "traffic": recorded_traffic(),
                 "kernel": "grouped expert gate/up GEMM + SwiGLU (tcgen05, one launch per layer)",
-                "bytes_per_launch": round(gu_bytes), "bytes_per_launch_all_experts": gate_up_bytes(cfg, C),
+                "bytes_per_launch": round(gu_bytes), "bytes_per_launch_all_experts": gate_up_bytes(cfg, C * Bq),
                 "avg_launch_ms": round(gu_ms, 5), "launches_timed": kn[GU],
                 "bytes_note": "weights of the experts each launch routed to + token pair rows + SwiGLU output",
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
     dn_ms = max(1e-9, kms[DN] / max(1, kn[DN]))
     dn_gbs = kbytes[DN] / max(1e-9, kms[DN] / 1e3) / 1e9
 
-    step_flops = prefill_flops(cfg, w.prefix) + w.n_canvases * (
-        passes_per_canvas * pass_flops(cfg, C, w.prefix, C) + pass_flops(cfg, C, w.prefix, 0))
+    step_flops = Bq * prefill_flops(cfg, w.prefix) + w.n_canvases * (
+        passes_per_canvas * pass_flops(cfg, C * Bq, w.prefix, C * Bq) + pass_flops(cfg, C * Bq, w.prefix, 0))
     tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     step_tc = step_flops / (elapsed_ms / args.steps / 1e3) / (tc_peak * 1e12)
 
@@ -379,7 +383,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded random-init weights N(0,0.02), uniform prompt tokens)",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, Bq),
         "passes_per_s": round(world * passes / (gen_ms / 1e3), 2) if gen_ms > 0 else None,
         "passes_per_canvas": passes_per_canvas,
         "denoise_ms_per_pass": round(gen_ms / max(1, passes), 4),
@@ -389,7 +393,7 @@ def run_ours(args):
         "roofline": roofline,
         "down_gemm": {"avg_launch_ms": round(dn_ms, 5), "achieved_gbs": round(dn_gbs, 1),
                       "bytes_per_launch": round(kbytes[DN] / max(1, kn[DN]))},
-        "experts_routed_per_layer": round((kbytes[GU] / kn[GU] - C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 4)
+        "experts_routed_per_layer": round((kbytes[GU] / kn[GU] - Bq * C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 4)
                                           / (2 * cfg.ffn_dim * cfg.d_model * 2), 2),
         "gpu_launches": int(launches),
         "kernel_ms_per_pass": {binding.TIMING_NAMES[k]: round(kms[k] / max(1, passes), 4)
@@ -398,25 +402,25 @@ def run_ours(args):
     }
 
     if not args.no_e2e:
-        prompts = np.ascontiguousarray(prompt_np[None, :])
-        toks = np.zeros((1, w.n_canvases * C), dtype=np.int32)
-        stp = np.zeros((w.n_canvases,), dtype=np.int32)
+        prompts = np.ascontiguousarray(prompt_np)
+        toks = np.zeros((Bq, w.n_canvases * C), dtype=np.int32)
+        stp = np.zeros((Bq * w.n_canvases,), dtype=np.int32)
         binding.dllm_set_timing(h, 0)
         for _ in range(max(1, args.warmup)):
-            binding.dllm_generate(h, 1, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
+            binding.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
                                   toks.ctypes.data, stp.ctypes.data)
         barrier(world)
         t0 = time.perf_counter()
         e_passes = 0
         for _ in range(args.steps):
-            binding.dllm_generate(h, 1, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
+            binding.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
                                   toks.ctypes.data, stp.ctypes.data)
-            e_passes += int(stp.sum())
+            e_passes += int(stp.reshape(Bq, w.n_canvases).max(axis=0).sum())
         t1 = time.perf_counter()
         e_s = max_over_ranks(t1 - t0, world)
-        out["e2e"] = {"value": round(world * args.steps * w.n_canvases * C / e_s, 2), "unit": UNIT,
+        out["e2e"] = {"value": round(world * args.steps * w.n_canvases * C * Bq / e_s, 2), "unit": UNIT,
                       "h2d_bytes_per_step": int(prompts.nbytes),
-                      "d2h_bytes_per_step": int(toks.nbytes + 4 * e_passes // args.steps),
+                      "d2h_bytes_per_step": int(toks.nbytes + 4 * Bq * e_passes // args.steps),
                       "api": "dllm_generate (host prompt in, host tokens out)"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

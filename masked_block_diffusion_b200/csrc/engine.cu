@@ -496,7 +496,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       dense_route_kernel<<<ceil_div(T, 256), 256, 0, h->st>>>(T, h->tk_idx, h->tk_w);
       h->launches++;
     }
-    permute_kernel<<<1, 1024, 34 * h->E * sizeof(int), h->st>>>(h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
+    permute_kernel<<<1, 1024, 0, h->st>>>(h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
                                                                h->row_token, h->routed, h->n_routed,
                                                                h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
                                                                timed ? h->routed_stat + l : nullptr);

@@ -219,72 +219,79 @@ __global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
 
 // ---------------------------------------------------------------- a8: permute
 
-// Stable counting sort of the N = T*k assignments by expert (one CTA of 1024 threads).
+// Counting sort of the N = T*k assignments by expert (one CTA of 1024 threads).
 // offsets[E+1]: expert ranges in the sorted order; slot_of[i]: sorted position of
-// assignment i = t*k + j; row_token[slot]: its token. Within an expert, assignments
-// keep their (t, j) order, so the permutation is deterministic.
+// assignment i = t*k + j; row_token[slot]: its token. Within an expert, slots are handed
+// out by an atomic cursor; no value depends on that order (each token's column of an
+// expert GEMM is computed on its own and the combine sums in the fixed j order).
 // Also lists the experts with at least one assignment (routed[0..n_routed), ascending)
 // with the prefix sums of their chunk counts ceil(count / bn) for the persistent grouped
-// GEMMs, and stores n_routed in *routed_stat when given.
+// GEMMs, and stores n_routed in *routed_stat when given. E <= 256.
 __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int N, int k, int E,
                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
                                                        int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
                                                        int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
                                                        int bn, int32_t* __restrict__ routed_stat) {
-  extern __shared__ int sh[];
-  int* cnt = sh;                 // [E]
-  int* base = sh + E;            // [E] running start of each expert
-  int* wcnt = sh + 2 * E;        // [32][E] per-warp counts -> per-warp prefix
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int cnt[256];
+  __shared__ int cur[256];
+  const int tid = threadIdx.x, lane = tid & 31;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int i = tid; i < N; i += blockDim.x) atomicAdd(&cnt[idx[i]], 1);
   __syncthreads();
-  if (tid == 0) {
-    int run = 0, nr = 0, chunks = 0;
-    for (int e = 0; e < E; ++e) {
-      base[e] = run;
-      offsets[e] = run;
-      run += cnt[e];
-      if (cnt[e] > 0) {
-        chunk_prefix[nr] = chunks;
-        routed[nr++] = e;
-        chunks += (cnt[e] + bn - 1) / bn;
+  if (tid < 32) {
+    // lane owns experts [lane * per, lane * per + per); exclusive scans of the counts,
+    // of the routed flags and of the chunk counts
+    const int per = (E + 31) / 32;
+    int c_sum = 0, r_sum = 0, ch_sum = 0;
+    for (int q = 0; q < per; ++q) {
+      const int e = lane * per + q;
+      const int c = e < E ? cnt[e] : 0;
+      c_sum += c;
+      r_sum += c > 0;
+      ch_sum += (c + bn - 1) / bn;
+    }
+    int c_pre = c_sum, r_pre = r_sum, ch_pre = ch_sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, c_pre, o);
+      const int b = __shfl_up_sync(0xffffffffu, r_pre, o);
+      const int d = __shfl_up_sync(0xffffffffu, ch_pre, o);
+      if (lane >= o) {
+        c_pre += a;
+        r_pre += b;
+        ch_pre += d;
       }
     }
-    offsets[E] = run;
-    chunk_prefix[nr] = chunks;
-    *n_routed = nr;
-    if (routed_stat) *routed_stat = nr;
+    c_pre -= c_sum;
+    r_pre -= r_sum;
+    ch_pre -= ch_sum;
+    for (int q = 0; q < per; ++q) {
+      const int e = lane * per + q;
+      if (e >= E) break;
+      const int c = cnt[e];
+      offsets[e] = c_pre;
+      cur[e] = c_pre;
+      if (c > 0) {
+        routed[r_pre] = e;
+        chunk_prefix[r_pre] = ch_pre;
+        ++r_pre;
+        ch_pre += (c + bn - 1) / bn;
+      }
+      c_pre += c;
+    }
+    if (lane == 31) {
+      offsets[E] = c_pre;
+      chunk_prefix[r_pre] = ch_pre;
+      *n_routed = r_pre;
+      if (routed_stat) *routed_stat = r_pre;
+    }
   }
   __syncthreads();
-  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
-    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-    const int i = c0 + tid;
-    const int e = (i < N) ? idx[i] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank_w = __popc(peers & ((1u << lane) - 1u));
-    if (e >= 0 && rank_w == 0) wcnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int run = 0;
-      for (int w = 0; w < 32; ++w) {
-        const int v = wcnt[w * E + ee];
-        wcnt[w * E + ee] = run;
-        run += v;
-      }
-      cnt[ee] = run;   // this chunk's count of expert ee
-    }
-    __syncthreads();
-    if (e >= 0) {
-      const int s = base[e] + wcnt[warp * E + e] + rank_w;
-      slot_of[i] = s;
-      row_token[s] = i / k;
-    }
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) base[ee] += cnt[ee];
-    __syncthreads();
+  for (int i = tid; i < N; i += blockDim.x) {
+    const int s = atomicAdd(&cur[idx[i]], 1);
+    slot_of[i] = s;
+    row_token[s] = i / k;
   }
 }
 
