@@ -48,6 +48,7 @@ struct AttnSmem {
 // block, which keeps the O accumulators, S tile and temporaries within 170 registers.
 template <int HD, int BK>
 __global__ void __launch_bounds__(128, 3) attn_kernel(AttnParams p) {
+  pdl_begin();
   static_assert(HD % 16 == 0 && BK % 16 == 0, "shape");
   using S = AttnSmem<HD, BK>;
   constexpr int NT = BK / 8;      // S n-tiles per warp
@@ -258,6 +259,7 @@ __global__ void __launch_bounds__(128, 3) attn_kernel(AttnParams p) {
 // One warp per (query row, head).
 template <int HD>
 __global__ void attn_merge_kernel(AttnParams p) {
+  pdl_begin();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= p.T * p.H) return;

@@ -87,7 +87,7 @@ struct LayerW {
   bf16_t* wr = nullptr;     // [E][d]
   bf16_t* wgu = nullptr;    // [E][2F][d]: per 128-row block, 64 gate rows then the 64 matching up rows
   bf16_t* wd = nullptr;     // [E][d][F]
-  CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd;
+  CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wr;
   CUtensorMap tm_k, tm_v;   // this layer's K / V cache as [slot][Hkv][max_ctx] rows of hd
 };
 
@@ -153,6 +153,11 @@ struct dllm_handle {
   CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // canvas passes use the tensor-core attention
+  int oproj_mode = 0;       // O projection on few tiles: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs
+  bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
+  bool attn_tp = true;      // tensor-core attention keeps P in TMEM (three-stage K / V rings)
+  bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
+  bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
   int32_t* d_P = nullptr;    // [max_batch]
@@ -269,20 +274,64 @@ int attn_split_keys(const dllm_handle* h, int splits) {
   return ceil_div(ceil_div(h->c.max_ctx, splits), 64) * 64;
 }
 
-// ------------------------------------------------------------------ GEMM launch helpers
+// ------------------------------------------------------------------ launch helpers
+
+// Launches kern on the handle's stream; with h->pdl the launch carries programmatic
+// stream serialisation, so the kernel may start while its predecessor drains (every
+// kernel of the pass waits for its predecessor with griddepcontrol.wait before its first
+// global-memory access).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(dllm_handle* h, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = h->st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = h->pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 
 template <int BN, int STAGES, int ACC, int SPLIT, class Sched, class Epi>
 cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const CUtensorMap& tb, int kblocks,
                         int a_first, const Sched& s, const Epi& e, const CUtensorMap* ta2 = nullptr,
                         const CUtensorMap* tb2 = nullptr) {
   auto kern = gemm_tc_kernel<BN, STAGES, ACC, SPLIT, Sched, Epi>;
-  constexpr int smem = GemmSmem<BN, STAGES, SPLIT, Epi>::kTotal;
+  constexpr int smem = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>::kTotal;
   static_assert(smem <= 232448, "shared memory per CTA");
   cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (r != cudaSuccess) return r;
-  kern<<<grid, 192, smem, h->st>>>(ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e, h->d_err);
+  if constexpr (Sched::kKSplit > 1) {
+    // split-K: clusters of kKSplit consecutive CTAs share one output tile
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = h->st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = Sched::kKSplit;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = h->pdl ? 2 : 1;
+    if (grid.x % Sched::kKSplit || kblocks < Sched::kKSplit) return cudaErrorInvalidValue;
+    r = cudaLaunchKernelEx(&cfg, kern, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e, h->d_err);
+    h->launches++;
+    if (r != cudaSuccess) return r;
+    return cudaGetLastError();
+  }
+  r = launch_k(h, kern, grid, dim3(192), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e,
+               h->d_err);
   h->launches++;
+  if (r != cudaSuccess) return r;
   return cudaGetLastError();
 }
 
@@ -292,10 +341,16 @@ cudaError_t qkv_gemm_hd(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc,
   const auto& c = h->c;
   EpiQKV<HD> e{h->q, kc, vc, h->rope_cos, h->rope_sin, pos0, slot, tok_per_req, c.n_heads, c.n_kv_heads, c.max_ctx};
   const int mt = ceil_div(T, 128);
-  DenseSched s{T, mt, HD};
-  dim3 grid(mt * h->qkv_heads);
   constexpr int STAGES = HD > 128 ? 4 : 5;
-  return launch_gemm<HD, STAGES, 1, kSplitA>(h, grid, h->tm_y, L.tm_wqkv, c.d_model / 64, 0, s, e, &h->tm_y_lo);
+  if (h->qkv_splitk && mt * h->qkv_heads * 2 <= 2 * h->num_sms) {
+    // few tiles (one canvas): split K over CTA pairs so that about twice as many SMs stream
+    DenseSplitKSched<2> s{T, mt, HD};
+    return launch_gemm<HD, STAGES, 1, kSplitA>(h, dim3(mt * h->qkv_heads * 2), h->tm_y, L.tm_wqkv, c.d_model / 64, 0,
+                                               s, e, &h->tm_y_lo);
+  }
+  DenseSched s{T, mt, HD};
+  return launch_gemm<HD, STAGES, 1, kSplitA>(h, dim3(mt * h->qkv_heads), h->tm_y, L.tm_wqkv, c.d_model / 64, 0, s, e,
+                                             &h->tm_y_lo);
 }
 
 cudaError_t qkv_gemm(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, int T, const int* pos0,
@@ -332,11 +387,13 @@ cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (r != cudaSuccess) return r;
   dim3 grid(ceil_div(tok_per_req, 64), c.n_heads, nreq * splits);
-  attn_kernel<HD, BK><<<grid, 128, smem, h->st>>>(p);
+  r = launch_k(h, attn_kernel<HD, BK>, grid, dim3(128), smem, p);
   h->launches++;
+  if (r != cudaSuccess) return r;
   if (splits > 1) {
-    attn_merge_kernel<HD><<<ceil_div((long)T * c.n_heads * 32, 256), 256, 0, h->st>>>(p);
+    r = launch_k(h, attn_merge_kernel<HD>, dim3(ceil_div((long)T * c.n_heads * 32, 256)), dim3(256), 0, p);
     h->launches++;
+    if (r != cudaSuccess) return r;
   }
   return cudaGetLastError();
 }
@@ -361,13 +418,23 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   p.split_keys = split_keys;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.err = h->d_err;
-  constexpr int smem = AttnTcCfg<HD>::kTotal;
-  cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (r != cudaSuccess) return r;
   dim3 grid(ceil_div((long)c.canvas * p.group, 128), c.n_kv_heads, nreq * splits);
-  attn_tc_kernel<HD><<<grid, 192, smem, h->st>>>(h->tm_q3, L.tm_k, L.tm_v, p);
+  cudaError_t r;
+  if (h->attn_tp) {
+    constexpr int smem = AttnTpCfg<HD>::kTotal;
+    r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tp_kernel<HD>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (r != cudaSuccess) return r;
+    r = launch_k(h, attn_tp_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
+  } else {
+    constexpr int smem = AttnTcCfg<HD>::kTotal;
+    r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (r != cudaSuccess) return r;
+    r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
+  }
   h->launches++;
+  if (r != cudaSuccess) return r;
   if (splits > 1) {
     AttnParams m;
     m.out = h->ao;
@@ -380,8 +447,9 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
     m.H = c.n_heads;
     m.n_splits = splits;
     m.split_keys = split_keys;
-    attn_merge_kernel<HD><<<ceil_div((long)T * c.n_heads * 32, 256), 256, 0, h->st>>>(m);
+    r = launch_k(h, attn_merge_kernel<HD>, dim3(ceil_div((long)T * c.n_heads * 32, 256)), dim3(256), 0, m);
     h->launches++;
+    if (r != cudaSuccess) return r;
   }
   return cudaGetLastError();
 }
@@ -408,6 +476,55 @@ cudaError_t tmark(dllm_handle* h, uint32_t tmask, int kind, int layer, int which
   // graph (a plain record would only express a dependency); outside capture it is plain
   if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, h->st, cudaEventRecordExternal);
   return cudaEventRecord(ev, h->st);
+}
+
+// Router logits on the tensor cores: logits[T][E] = y W_r^T with the normalised
+// activations as their (hi, lo) bf16 pair, so each product keeps about 16 mantissa bits
+// of y and the sum is fp32. Experts form 32-column tiles; with few tiles (one canvas:
+// 2 x 4) the K loop is split over clusters of up to 8 CTAs.
+template <int KS>
+cudaError_t router_gemm_ks(dllm_handle* h, const LayerW& L, int T, int mt, int tiles) {
+  EpiStoreF32<32> e{h->rlogits, h->E, h->E};
+  const int kb = h->c.d_model / 64;
+  if constexpr (KS == 1) {
+    DenseSched s{T, mt, 32};
+    return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
+  } else {
+    DenseSplitKSched<KS> s{T, mt, 32};
+    return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles * KS), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
+  }
+}
+
+cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T) {
+  const int mt = ceil_div(T, 128);
+  const int tiles = mt * (h->E / 32);
+  const int kb = h->c.d_model / 64;
+  if (tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
+  if (tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
+  if (tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
+  return router_gemm_ks<1>(h, L, T, mt, tiles);
+}
+
+// Attention output projection with the residual add, x += ao * Wo^T. With few tiles
+// (one canvas: 2 x 44 at d_model 2816) K is split over CTA pairs; two stages per CTA let
+// two CTAs share an SM so that every pair is resident at once.
+cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
+  const auto& c = h->c;
+  const int d = c.d_model;
+  const int kb = c.n_heads * c.head_dim / 64;
+  EpiResidual<64> e{h->x, d};
+  const int mt = ceil_div(T, 128);
+  const int tiles = mt * (d / 64);
+  if (h->oproj_mode == 1 && tiles * 2 <= 2 * h->num_sms && kb >= 2) {
+    DenseSplitKSched<2> s{T, mt, 64};
+    return launch_gemm<64, 2, 1, kSplitA>(h, dim3(tiles * 2), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
+  }
+  if (h->oproj_mode == 2 && tiles * 3 <= 2 * h->num_sms && kb >= 3) {
+    DenseSplitKSched<3> s{T, mt, 64};
+    return launch_gemm<64, 2, 1, kSplitA>(h, dim3(tiles * 3), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
+  }
+  DenseSched s{T, mt, 64};
+  return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
 template <int BN>
@@ -454,7 +571,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
     bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
     if (l == 0) {   // later layers get this norm from the previous layer's combine
-      rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
+      CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(256), 0, h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd));
       h->launches++;
     }
     CK(tmark(h, timed, DLLM_TIMING_QKV, l, 0));
@@ -464,23 +581,21 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys, &L));
     CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 0));
-    {
-      EpiResidual<64> e{h->x, d};
-      const int mt = ceil_div(T, 128);
-      DenseSched s{T, mt, 64};
-      CK((launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, c.n_heads * c.head_dim / 64, 0,
-                                         s, e, &h->tm_ao_lo)));
-    }
+    CK(o_proj(h, L, T));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 0));
-    rmsnorm_kernel<<<T, 256, 0, h->st>>>(h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd);
+    CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(256), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd));
     h->launches++;
     if (!h->dense) {
-      router_kernel<<<dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp)), 256, kRouterTok * d * sizeof(float),
-                      h->st>>>(
-          h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits);
-      topk_kernel<<<ceil_div((long)T * 32, 256), 256, 0, h->st>>>(h->rlogits, T, h->E, h->k, h->tk_idx, h->tk_w);
-      h->launches += 2;
+      if (h->router_tc) {
+        CK(router_gemm(h, L, T));
+      } else {
+        CK(launch_k(h, router_kernel, dim3(dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp))), dim3(256), kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E,
+                                                                 h->rlogits));
+        h->launches++;
+      }
+      CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k, h->tk_idx, h->tk_w));
+      h->launches++;
       if (record) {
         CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
                            sizeof(float) * T * h->E, cudaMemcpyDeviceToDevice, h->st));
@@ -488,29 +603,29 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                            cudaMemcpyDeviceToDevice, h->st));
       }
       if (h->force_routing && T == h->force_T) {
-        force_route_kernel<<<ceil_div(T, 128), 128, 0, h->st>>>(
-            h->rlogits, h->dbg_force + (size_t)l * h->force_T * h->k, T, h->E, h->k, h->tk_idx, h->tk_w);
+        CK(launch_k(h, force_route_kernel, dim3(ceil_div(T, 128)), dim3(128), 0, 
+            h->rlogits, h->dbg_force + (size_t)l * h->force_T * h->k, T, h->E, h->k, h->tk_idx, h->tk_w));
         h->launches++;
       }
     } else {
-      dense_route_kernel<<<ceil_div(T, 256), 256, 0, h->st>>>(T, h->tk_idx, h->tk_w);
+      CK(launch_k(h, dense_route_kernel, dim3(ceil_div(T, 256)), dim3(256), 0, T, h->tk_idx, h->tk_w));
       h->launches++;
     }
-    permute_kernel<<<1, 1024, 0, h->st>>>(h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
+    CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
                                                                h->row_token, h->routed, h->n_routed,
                                                                h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
-                                                               timed ? h->routed_stat + l : nullptr);
-    gather_rows_kernel<<<N, 128, 0, h->st>>>(h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo);
+                                                               timed ? h->routed_stat + l : nullptr));
+    CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(128), 0, h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
     CK(moe_gemms(h, L, N, l, timed));
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
     const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
     if (next_gain)
-      combine_norm_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d, next_gain, c.rms_eps,
-                                                h->y, h->y_lo);
+      CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d, next_gain, c.rms_eps,
+                                                h->y, h->y_lo));
     else
-      combine_kernel<<<T, 256, 0, h->st>>>(h->x, h->obuf, h->slot_of, h->tk_w, h->k, d);
+      CK(launch_k(h, combine_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d));
     h->launches++;
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 1));
     if (record)
@@ -526,7 +641,7 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
   const auto& c = h->c;
   const int C = c.canvas, T = B * C, d = c.d_model;
   const int splits = attn_splits(h, B);
-  embed_kernel<<<T, 128, 0, h->st>>>(h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x);
+  CK(launch_k(h, embed_kernel, dim3(T), dim3(128), 0, h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x));
   h->launches++;
   const uint32_t tm = (h->timing && mode == 0) ? h->tmask : 0u;
   int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0,
@@ -542,12 +657,12 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
     DenseSched s{T, mt, 256};
     CK((launch_gemm<256, 3, 1, kSplitA>(h, dim3(mt * nvt), h->tm_y, h->tm_head, d / 64, 0, s, e, &h->tm_y_lo)));
   }
-  lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, h->st>>>(h->lm_m, h->lm_s, h->lm_i, T, nvt, h->conf,
-                                                                  h->argmax);
+  CK(launch_k(h, lm_merge_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->lm_m, h->lm_s, h->lm_i, T, nvt, h->conf,
+                                                                  h->argmax));
   const int threads = ceil_div(C, 32) * 32;
-  commit_kernel<<<B, threads, C * (sizeof(float) + 1), h->st>>>(h->canvas, h->mask, h->conf, h->argmax, C,
+  CK(launch_k(h, commit_kernel, dim3(B), dim3(threads), C * (sizeof(float) + 1), h->canvas, h->mask, h->conf, h->argmax, C,
                                                                  h->d_policy, h->d_step, h->d_remaining, nullptr,
-                                                                 nullptr);
+                                                                 nullptr));
   h->launches += 2;
   CK(tmark(h, tm, DLLM_TIMING_HEAD, 0, 1));
   CK(cudaGetLastError());
@@ -743,6 +858,12 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   // tensor-core attention for canvas passes when a query tile of 128 rows holds whole
   // GQA groups (DLLM_ATTN_LEGACY=1 keeps the warp-MMA kernel, for comparisons)
   h->attn_tc = (128 % (H / Hkv) == 0) && !getenv("DLLM_ATTN_LEGACY");
+  if (const char* m = getenv("DLLM_OPROJ_MODE")) h->oproj_mode = atoi(m);
+  if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
+  if (const char* m = getenv("DLLM_ATTN_TP")) h->attn_tp = atoi(m) != 0;
+  h->router_tc = !h->dense && h->E % 32 == 0;
+  if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
+  if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
   // ---- weights
@@ -904,6 +1025,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   for (auto& L : h->L) {
     ok &= make_tmap(&L.tm_wqkv, L.wqkv, qd + 2 * kvd, d, hd);
     ok &= make_tmap(&L.tm_wo, L.wo, d, qd, 64);
+    if (h->router_tc) ok &= make_tmap(&L.tm_wr, L.wr, h->E, d, 32);
     ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
     ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);
     if (h->attn_tc) {
@@ -941,7 +1063,7 @@ int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool pro
                      prompt_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, h->st));
   const int32_t s = req;
   CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
-  embed_kernel<<<n, 128, 0, h->st>>>(h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x);
+  CK(launch_k(h, embed_kernel, dim3(n), dim3(128), 0, h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x));
   h->launches++;
   int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false, 0u, nullptr);
   if (r) return r;
@@ -1025,8 +1147,8 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
   if (r) return r;
   if ((r = upload_policy(h, policy, max_steps))) return r;
   const int C = h->c.canvas, B = req_count;
-  canvas_init_kernel<<<ceil_div((long)B * C, 256), 256, 0, h->st>>>(h->canvas, h->mask, B * C, h->c.mask_id,
-                                                                    h->d_step, B);
+  CK(launch_k(h, canvas_init_kernel, dim3(ceil_div((long)B * C, 256)), dim3(256), 0, h->canvas, h->mask, B * C, h->c.mask_id,
+                                                                    h->d_step, B));
   h->launches++;
   std::vector<int> done_at(B, -1);
   int s = 0;

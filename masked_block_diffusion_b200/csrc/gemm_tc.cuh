@@ -25,7 +25,10 @@ struct Tile {
 // One output tile per CTA over an M x N problem; m tiles vary fastest so that the CTAs
 // sharing a weight tile run close together (the second read hits L2).
 struct DenseSched {
+  static constexpr int kSmemBytes = 0;
+  static constexpr int kKSplit = 1;
   int M, n_mtiles, BN;
+  DLLM_DEV void stage(int*) {}
   DLLM_DEV int count() const { return 1; }
   DLLM_DEV Tile tile(int) const {
     Tile t;
@@ -40,30 +43,26 @@ struct DenseSched {
   }
 };
 
-// Grouped (one GEMM per expert), operands swapped so that the expert's weight rows fill
-// the 128-row M side and its few tokens form N. CTA (blockIdx.x, blockIdx.y) = (m tile,
-// expert); its tiles are the expert's token chunks of BN rows, taken from the
-// expert-sorted token buffer between offsets[e] and offsets[e+1].
-struct GroupedSched {
-  const int* offsets;
-  int rows_per_expert;
-  int BN;
-  DLLM_DEV int count() const {
-    int e = blockIdx.y;
-    int cnt = offsets[e + 1] - offsets[e];
-    return (cnt + BN - 1) / BN;
-  }
-  DLLM_DEV Tile tile(int j) const {
+// Dense tiles with the K loop split over a cluster of KS CTAs (consecutive blockIdx.x):
+// CTA rank r of a cluster accumulates k blocks [r*kb/KS, (r+1)*kb/KS) of the same output
+// tile, and the partial sums meet in rank 0's TMEM over distributed shared memory
+// before the epilogue. For problems with fewer tiles than SMs.
+template <int KS>
+struct DenseSplitKSched {
+  static constexpr int kSmemBytes = 0;
+  static constexpr int kKSplit = KS;
+  int M, n_mtiles, BN;
+  DLLM_DEV void stage(int*) {}
+  DLLM_DEV int count() const { return 1; }
+  DLLM_DEV Tile tile(int) const {
     Tile t;
-    int e = blockIdx.y;
-    int off = offsets[e];
-    int cnt = offsets[e + 1] - off;
-    t.mt = blockIdx.x;
-    t.nt = e;
-    t.a_row = e * rows_per_expert + blockIdx.x * 128;
-    t.b_row = off + j * BN;
-    t.m_valid = 128;
-    t.n_valid = min(BN, cnt - j * BN);
+    int id = blockIdx.x / KS;
+    t.mt = id % n_mtiles;
+    t.nt = id / n_mtiles;
+    t.a_row = t.mt * 128;
+    t.b_row = t.nt * BN;
+    t.m_valid = min(128, M - t.a_row);
+    t.n_valid = BN;
     return t;
   }
 };
@@ -76,7 +75,14 @@ struct GroupedSched {
 // number of equal-sized tiles whatever the routing skew, and streams them back to back
 // (the next tile's loads overlap this tile's epilogue through the double-buffered
 // accumulator).
+//
+// The routing tables are copied into shared memory once per CTA (stage(), run by every
+// thread before the roles split), so that finding an item's expert is a short search in
+// shared memory instead of a chain of dependent global loads on the producer's path.
 struct PersistentGroupedSched {
+  static constexpr int kMaxRouted = 256;
+  static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
+  static constexpr int kKSplit = 1;
   const int* offsets;        // [E+1] token ranges per expert
   const int* routed;         // [E] experts with at least one token, ascending
   const int* n_routed;       // [1]
@@ -84,6 +90,33 @@ struct PersistentGroupedSched {
   int rows_per_expert;
   int m_tiles;
   int BN;
+  // shared-memory copies, per routed expert r: token offset and count (set by stage())
+  const int* s_off = nullptr;
+  const int* s_cnt = nullptr;
+  DLLM_DEV void stage(int* s) {
+    const int n = min(*n_routed, kMaxRouted);
+    int* cp = s;
+    int* ex = cp + kMaxRouted + 1;
+    int* of = ex + kMaxRouted;
+    int* ct = of + kMaxRouted;
+    int* nn = ct + kMaxRouted;
+    for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+      cp[i] = chunk_prefix[i];
+      if (i < n) {
+        const int e = routed[i];
+        const int o = offsets[e];
+        ex[i] = e;
+        of[i] = o;
+        ct[i] = offsets[e + 1] - o;
+      }
+    }
+    if (threadIdx.x == 0) *nn = n;
+    chunk_prefix = cp;
+    routed = ex;
+    s_off = of;
+    s_cnt = ct;
+    n_routed = nn;
+  }
   DLLM_DEV int n_items() const { return chunk_prefix[*n_routed] * m_tiles; }
   DLLM_DEV int count() const {
     const int n = n_items();
@@ -100,8 +133,8 @@ struct PersistentGroupedSched {
     const int ch = chunk_prefix[lo + 1] - chunk_prefix[lo];
     const int local = i - chunk_prefix[lo] * m_tiles;
     const int chunk = local % ch;
-    const int off = offsets[e];
-    const int cnt = offsets[e + 1] - off;
+    const int off = s_off[lo];
+    const int cnt = s_cnt[lo];
     Tile t;
     t.mt = local / ch;
     t.nt = e;
@@ -123,7 +156,7 @@ __host__ __device__ constexpr int tmem_cols_for(int bn) {
 // accumulator. kSplitNone: plain; kSplitA: A is a (hi, lo) pair; kSplitB: B is.
 enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
 
-template <int BN, int STAGES, int SPLIT, class Epi>
+template <int BN, int STAGES, int SPLIT, class Epi, class Sched = DenseSched>
 struct GemmSmem {
   static constexpr int kA = 128 * 64 * 2;
   static constexpr int kB = BN * 64 * 2;
@@ -132,10 +165,15 @@ struct GemmSmem {
   static constexpr int kStageBytes = kA + kA2 + kB + kB2;   // TMA bytes per stage
   static constexpr int kOffA2 = STAGES * kA;
   static constexpr int kOffB = kOffA2 + STAGES * kA2;
-  static constexpr int kOffB2 = kOffB + STAGES * kB;
+  // kSplitB keeps each stage's B pair adjacent ([hi rows | lo rows]), so that one MMA
+  // with N = 2 BN reads both: the A tile is then read from shared memory once per k step
+  // instead of once per half.
+  static constexpr int kBStage = kB + kB2;
+  static constexpr int kOffB2 = kOffB + kB;   // the lo half of stage 0 (stage s: + s * kBStage)
   static constexpr int kBarOff = STAGES * kStageBytes;
   static constexpr int kEpiOff = kBarOff + 256;
-  static constexpr int kTotal = kEpiOff + Epi::kSmemBytes + 1024;   // + alignment slack
+  static constexpr int kSchedOff = kEpiOff + Epi::kSmemBytes;
+  static constexpr int kTotal = kSchedOff + Sched::kSmemBytes + 1024;   // + alignment slack
 };
 
 DLLM_DEV void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -154,17 +192,70 @@ DLLM_DEV bool epi_all(bool ok) {
   return r != 0;
 }
 
+// Split-K hand-over of one tile's partial sums inside a cluster (epilogue threads only;
+// thread r owns accumulator row r). Ranks > 0 copy their TMEM partial into their own
+// shared memory ([BN/4][128] float4, over the stage buffers, idle once the tile's last
+// MMA has completed) and signal rank 0, which adds every peer's partial into its TMEM
+// accumulator through distributed shared memory. The cluster barrier at the end of the
+// kernel keeps the peers resident until rank 0 has read them. Returns false (with *err
+// set) when the wait runs out.
+template <int BN, int KS>
+DLLM_DEV bool splitk_reduce(int krank, uint32_t taddr, int r, uint8_t* part_smem, uint64_t* peer_ready,
+                            volatile int* abort_flag, int* err) {
+  float4* part = reinterpret_cast<float4*>(part_smem);
+  if (krank != 0) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        part[((c >> 2) + i) * 128 + r] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+    mbar_arrive_cluster(mapa_shared(smem_u32(peer_ready), 0));
+    return true;
+  }
+  const bool got = mbar_wait_cluster(peer_ready, 0, abort_flag);
+  if (!epi_all(got)) {
+    if (!got) atomicExch(err, kDevTimeoutEpilogue);
+    return false;
+  }
+#pragma unroll 1
+  for (int p = 1; p < KS; ++p) {
+    const uint32_t base = mapa_shared(smem_u32(part), p);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tmem_ld16(taddr + c, v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 w = ld_shared_cluster_v4(base + (uint32_t)((((c >> 2) + i) * 128 + r) * 16));
+        v[4 * i] += w.x;
+        v[4 * i + 1] += w.y;
+        v[4 * i + 2] += w.z;
+        v[4 * i + 3] += w.w;
+      }
+      tmem_st16(taddr + c, v);
+    }
+  }
+  return true;
+}
+
 template <int BN, int STAGES, int ACC_BUFS, int SPLIT, class Sched, class Epi>
 __global__ void __launch_bounds__(192, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a2,
                const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_b2,
-               int k_blocks, int a_stream_first, Sched sched, Epi epi, int* err) {
+               int k_blocks, int a_stream_first, Sched sched_in, Epi epi, int* err) {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
-  using L = GemmSmem<BN, STAGES, SPLIT, Epi>;
-  constexpr int kCols = tmem_cols_for(BN);
+  using L = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>;
+  constexpr int kAccN = SPLIT == kSplitB ? 2 * BN : BN;   // kSplitB: columns [0, BN) hi, [BN, 2 BN) lo
+  static_assert(kAccN <= 256, "UMMA N");
+  constexpr int kCols = tmem_cols_for(kAccN);
   constexpr int kTmemCols = kCols * ACC_BUFS;
   static_assert(kTmemCols <= 512, "TMEM has 512 columns");
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, kAccN);
+  constexpr int KS = Sched::kKSplit;
+  static_assert(KS == 1 || BN * 128 * 4 <= STAGES * L::kStageBytes, "split-K partial fits the stage buffers");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -177,9 +268,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + ACC_BUFS;
   uint64_t* drain = acc_empty + ACC_BUFS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* peer_ready = drain + 1;   // split-K: rank 0 learns that the peers' partials are in place
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* epi_smem = smem + L::kEpiOff;
+  Sched sched = sched_in;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,6 +287,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       mbar_init(&acc_empty[a], 128);
     }
     mbar_init(drain, 1);
+    if (KS > 1) mbar_init(peer_ready, 128 * (KS - 1));
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tma_a);
@@ -208,8 +302,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (KS > 1) cluster_sync();   // the peers' barriers are initialised before anyone arrives on them
+  pdl_trigger();                // after the TMEM allocation
+  pdl_wait();                   // the inputs (and the routing tables) are complete from here on
+  if (Sched::kSmemBytes > 0) {
+    sched.stage(reinterpret_cast<int*>(smem + L::kSchedOff));
+    __syncthreads();
+  }
   const uint32_t tmem_base = *tmem_slot;
   const int ntiles = sched.count();
+  const int krank = KS > 1 ? (int)cluster_ctarank() : 0;
+  const int kb_begin = krank * k_blocks / KS;
+  const int kb_end = (krank + 1) * k_blocks / KS;
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -223,13 +327,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       const Tile t = sched.tile(j);
-      for (int kb = 0; kb < k_blocks; ++kb) {
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
         tma_load_2d(sA + stage * L::kA, &tma_a, &full[stage], kb * 64, t.a_row, pol_a);
         if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
-        tma_load_2d(sB + stage * L::kB, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
-        if (SPLIT == kSplitB) tma_load_2d(sB2 + stage * L::kB2, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
+        tma_load_2d(sB + stage * L::kBStage, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
+        if (SPLIT == kSplitB) tma_load_2d(sB2 + stage * L::kBStage, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -257,21 +361,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * kCols;
-      for (int kb = 0; kb < k_blocks; ++kb) {
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + stage * L::kA);
-        const uint32_t b0 = smem_u32(sB + stage * L::kB);
+        const uint32_t b0 = smem_u32(sB + stage * L::kBStage);
         const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
-        const uint32_t b1 = smem_u32(sB2 + stage * L::kB2);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc,
-                    (kb | kk) != 0);
+                    (kb != kb_begin || kk != 0) ? 1u : 0u);
           if (SPLIT == kSplitA)
             umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc, 1);
-          if (SPLIT == kSplitB)
-            umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b1 + kk * 32), kIdesc, 1);
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -302,7 +403,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       tc_fence_after();
       const Tile t = sched.tile(j);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kCols;
-      epi(t, taddr, r, epi_smem);
+      if constexpr (SPLIT == kSplitB) {
+        // D = D_hi + D_lo, into the first BN columns the epilogue reads
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float hi[16], lo[16];
+          tmem_ld16(taddr + c, hi);
+          tmem_ld16(taddr + BN + c, lo);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hi[i] += lo[i];
+          tmem_st16(taddr + c, hi);
+        }
+      }
+      if constexpr (KS > 1) {
+        if (!splitk_reduce<BN, KS>(krank, taddr, r, smem, peer_ready, abort_flag, err)) {
+          *abort_flag = 1;
+          break;
+        }
+      }
+      if (krank == 0) epi(t, taddr, r, epi_smem);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -311,6 +430,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (KS > 1) cluster_sync();   // no CTA leaves while rank 0 may still read its shared memory
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, kTmemCols);

@@ -12,6 +12,7 @@ namespace dllm {
 // x[t] = Emb[token] as fp32; a masked canvas position reads the [MASK] row.
 __global__ void embed_kernel(const bf16_t* __restrict__ emb, const int32_t* __restrict__ tokens,
                              const uint8_t* __restrict__ mask, int mask_id, int d, float* __restrict__ x) {
+  pdl_begin();
   const int t = blockIdx.x;
   int tok = tokens[t];
   if (mask != nullptr && mask[t]) tok = mask_id;
@@ -37,6 +38,7 @@ __global__ void embed_kernel(const bf16_t* __restrict__ emb, const int32_t* __re
 // y_lo = bf16(v - y) (y_lo may be NULL); rstd[t] kept for the fp32 router.
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
                                bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo, float* __restrict__ rstd) {
+  pdl_begin();
   const int t = blockIdx.x;
   const float4* xr = reinterpret_cast<const float4*>(x + (long)t * d);
   float ss = 0.f;
@@ -83,6 +85,7 @@ constexpr int kRouterMaxChunks = 16;   // d <= 4096
 __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ x, const float* __restrict__ rstd,
                                                      const float* __restrict__ g, const bf16_t* __restrict__ wr,
                                                      int T, int d, int E, float* __restrict__ logits) {
+  pdl_begin();
   extern __shared__ float xs[];   // [kRouterTok][d]
   const int t0 = blockIdx.x * kRouterTok;
   for (int i = threadIdx.x; i < kRouterTok * d / 4; i += blockDim.x) {
@@ -153,6 +156,7 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ x
 // the k selected logits. One warp per token; E <= 256, k <= 32.
 __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
                             float* __restrict__ gate) {
+  pdl_begin();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -198,6 +202,7 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
 // from this pass's own logits at those experts. One thread per token.
 __global__ void force_route_kernel(const float* __restrict__ logits, const int32_t* __restrict__ forced, int T,
                                    int E, int k, int32_t* __restrict__ idx, float* __restrict__ gate) {
+  pdl_begin();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   float mx = -INFINITY;
@@ -213,6 +218,7 @@ __global__ void force_route_kernel(const float* __restrict__ logits, const int32
 
 // Dense FFN as one expert with gate 1.
 __global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
+  pdl_begin();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t < T) { idx[t] = 0; gate[t] = 1.f; }
 }
@@ -232,6 +238,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
                                                        int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
                                                        int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
                                                        int bn, int32_t* __restrict__ routed_stat) {
+  pdl_begin();
   __shared__ int cnt[256];
   __shared__ int cur[256];
   const int tid = threadIdx.x, lane = tid & 31;
@@ -300,6 +307,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
 __global__ void gather_rows_kernel(const bf16_t* __restrict__ y, const bf16_t* __restrict__ y_lo,
                                    const int32_t* __restrict__ row_token, int N, int d, bf16_t* __restrict__ xg,
                                    bf16_t* __restrict__ xg_lo) {
+  pdl_begin();
   const int s = blockIdx.x;
   if (s >= N) return;
   const long src_row = (long)row_token[s] * d;
@@ -316,20 +324,48 @@ __global__ void gather_rows_kernel(const bf16_t* __restrict__ y, const bf16_t* _
 // ---------------------------------------------------------------- a11: combine
 
 // x[t] += sum_j gate[t][j] * o[slot_of[t*k + j]], j in fixed order 0..k-1.
+// Token t's routed rows and gates, held in registers (k <= kMaxK), so that the k row
+// loads of one column chunk are all in flight together.
+constexpr int kMaxK = 8;
+struct CombineRow {
+  const float4* row[kMaxK];
+  float w[kMaxK];
+  int k;
+  DLLM_DEV CombineRow(const float* o, const int32_t* slot_of, const float* gate, int t, int k_, int d) : k(k_) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      const bool on = j < k;
+      row[j] = reinterpret_cast<const float4*>(o + (long)(on ? slot_of[(long)t * k + j] : 0) * d);
+      w[j] = on ? gate[(long)t * k + j] : 0.f;
+    }
+  }
+  // sum_j w_j * o[slot_j][4c .. 4c+3], accumulated in j order
+  DLLM_DEV float4 at(int c) const {
+    float4 v[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) v[j] = j < k ? row[j][c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        acc.x = fmaf(w[j], v[j].x, acc.x);
+        acc.y = fmaf(w[j], v[j].y, acc.y);
+        acc.z = fmaf(w[j], v[j].z, acc.z);
+        acc.w = fmaf(w[j], v[j].w, acc.w);
+      }
+    }
+    return acc;
+  }
+};
+
 __global__ void combine_kernel(float* __restrict__ x, const float* __restrict__ o, const int32_t* __restrict__ slot_of,
                                const float* __restrict__ gate, int k, int d) {
+  pdl_begin();
   const int t = blockIdx.x;
   float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
+  const CombineRow cr(o, slot_of, gate, t, k, d);
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float w = gate[(long)t * k + j];
-      const float4 v = reinterpret_cast<const float4*>(o + (long)slot_of[(long)t * k + j] * d)[c];
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
+    const float4 acc = cr.at(c);
     float4 xv = xr[c];
     xv.x += acc.x;
     xv.y += acc.y;
@@ -348,19 +384,13 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x
                                                            const float* __restrict__ gate, int k, int d,
                                                            const float* __restrict__ g, float eps,
                                                            bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo) {
+  pdl_begin();
   const int t = blockIdx.x;
   float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
   float ss = 0.f;
+  const CombineRow cr(o, slot_of, gate, t, k, d);
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float w = gate[(long)t * k + j];
-      const float4 v = reinterpret_cast<const float4*>(o + (long)slot_of[(long)t * k + j] * d)[c];
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
+    const float4 acc = cr.at(c);
     float4 xv = xr[c];
     xv.x += acc.x;
     xv.y += acc.y;
@@ -414,6 +444,7 @@ DLLM_DEV void lse_combine(float& m, float& s, int& i, float m2, float s2, int i2
 __global__ void lm_merge_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
                                 const int32_t* __restrict__ pi, int rows, int n_tiles, float* __restrict__ conf,
                                 int32_t* __restrict__ argmax) {
+  pdl_begin();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= rows) return;
@@ -455,6 +486,7 @@ __global__ void commit_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict_
                               const int32_t* __restrict__ argmax, int C, const PolicyDev* __restrict__ pol,
                               int32_t* __restrict__ step, int32_t* __restrict__ remaining, float* __restrict__ conf_out,
                               int32_t* __restrict__ argmax_out) {
+  pdl_begin();
   extern __shared__ uint8_t smc[];
   float* sc = reinterpret_cast<float*>(smc);
   uint8_t* sm = smc + C * sizeof(float);
@@ -505,6 +537,7 @@ __global__ void commit_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict_
 
 // Fresh all-[MASK] canvases and zeroed step counters.
 __global__ void canvas_init_kernel(int32_t* canvas, uint8_t* mask, int n, int mask_id, int32_t* step, int B) {
+  pdl_begin();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     canvas[i] = mask_id;
