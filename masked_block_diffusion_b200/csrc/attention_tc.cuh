@@ -37,6 +37,7 @@ struct AttnTcParams {
   int T;                    // total query rows
   int H, Hkv, group, max_ctx;
   int n_splits, split_keys;
+  int causal;               // 1: query i of request b sees keys 0 .. P_b + i (prompt prefill)
   float scale_log2;         // log2(e) / sqrt(HD)
   int* err;
 };
@@ -419,6 +420,10 @@ DLLM_DEV void softmax_rows_tp(const AttnTcParams& p, uint32_t tmem_base, uint64_
   const int q = warp & 3;
   const int r = q * 32 + lane;
   const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+  // keys this row may see end at row_ke: the tile's end, or (causal) the row's own query
+  // position + 1; rows past the last query take the last query's limit (output dropped)
+  int row_ke = ke;
+  if (p.causal) row_ke = min(ke, p.pos0[b] + min(q0 + r / p.group, p.tok_per_req - 1) + 1);
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
   for (int j = 0; j < nblk; ++j) {
@@ -434,7 +439,7 @@ DLLM_DEV void softmax_rows_tp(const AttnTcParams& p, uint32_t tmem_base, uint64_
     float mx = -INFINITY;
 #pragma unroll
     for (int c = 0; c < BK; ++c) {
-      const float v = (key0 + c < ke) ? s[c] * p.scale_log2 : -INFINITY;
+      const float v = (key0 + c < row_ke) ? s[c] * p.scale_log2 : -INFINITY;
       s[c] = v;
       mx = fmaxf(mx, v);
     }
@@ -551,12 +556,13 @@ attn_tp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   pdl_wait();   // pos0 and the K / V written by the QKV projection
-  const int qt = blockIdx.x, g = blockIdx.y;
+  // causal: the last query tiles see the most keys, so they are launched first
+  const int qt = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x, g = blockIdx.y;
   const int b = blockIdx.z / p.n_splits, sp = blockIdx.z % p.n_splits;
   const int C = p.tok_per_req, grp = p.group;
   const int qpt = 128 / grp;
   const int q0 = qt * qpt;
-  const int kend = p.pos0[b] + C;
+  const int kend = p.pos0[b] + (p.causal ? min(C, q0 + qpt) : C);
   const int ks = sp * p.split_keys;
   const int ke = min(kend, ks + p.split_keys);
   if (q0 >= C || ks >= ke) return;   // uniform over the CTA, before any barrier or TMEM use

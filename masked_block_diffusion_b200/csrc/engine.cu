@@ -156,6 +156,8 @@ struct dllm_handle {
   int oproj_mode = 0;       // O projection on few tiles: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
   bool attn_tp = true;      // tensor-core attention keeps P in TMEM (three-stage K / V rings)
+  bool prefill_tc = true;   // causal prefill attention on the tensor cores too
+  bool moe_pair = true;     // grouped GEMMs at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
@@ -399,16 +401,18 @@ cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq
 }
 
 template <int HD>
-cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, int splits, int split_keys) {
+cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, int tok_per_req, const int* pos0,
+                            const int* slot, int causal, int splits, int split_keys) {
   const auto& c = h->c;
   AttnTcParams p;
   p.out = h->ao;
   p.out_lo = h->ao_lo;
   p.part_o = h->apart;
   p.part_lse = h->alse;
-  p.pos0 = h->d_P;
-  p.slot = h->d_slot;
-  p.tok_per_req = c.canvas;
+  p.pos0 = pos0;
+  p.slot = slot;
+  p.tok_per_req = tok_per_req;
+  p.causal = causal;
   p.T = T;
   p.H = c.n_heads;
   p.Hkv = c.n_kv_heads;
@@ -418,9 +422,9 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   p.split_keys = split_keys;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.err = h->d_err;
-  dim3 grid(ceil_div((long)c.canvas * p.group, 128), c.n_kv_heads, nreq * splits);
+  dim3 grid(ceil_div((long)tok_per_req * p.group, 128), c.n_kv_heads, nreq * splits);
   cudaError_t r;
-  if (h->attn_tp) {
+  if (h->attn_tp || causal) {
     constexpr int smem = AttnTpCfg<HD>::kTotal;
     r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tp_kernel<HD>),
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -441,8 +445,8 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
     m.out_lo = h->ao_lo;
     m.part_o = h->apart;
     m.part_lse = h->alse;
-    m.pos0 = h->d_P;
-    m.tok_per_req = c.canvas;
+    m.pos0 = pos0;
+    m.tok_per_req = tok_per_req;
     m.T = T;
     m.H = c.n_heads;
     m.n_splits = splits;
@@ -456,9 +460,12 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
 
 cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
                       const int* slot, int causal, int splits, int split_keys, const LayerW* L = nullptr) {
-  if (!causal && h->attn_tc && L) {   // the bidirectional canvas pass on the tensor cores
-    if (h->c.head_dim == 176) return attention_tc_hd<176>(h, *L, T, nreq, splits, split_keys);
-    return attention_tc_hd<64>(h, *L, T, nreq, splits, split_keys);
+  // tensor cores: the bidirectional canvas pass, and (one key range per query tile) the
+  // causal prompt prefill
+  if (h->attn_tc && L && (!causal || (h->prefill_tc && splits == 1))) {
+    if (h->c.head_dim == 176)
+      return attention_tc_hd<176>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
+    return attention_tc_hd<64>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
   }
   if (h->c.head_dim == 176)
     return attention_hd<176, 32>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
@@ -527,14 +534,17 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
-template <int BN>
+// MPI = 2 (BN = 64): items of two weight tiles sharing the token chunk (48 KB stages);
+// MPI = 1: one weight tile per item (at BN = 128 the two accumulator buffers take all
+// 512 TMEM columns).
+template <int BN, int MPI>
 cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, uint32_t timed) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int STAGES = BN <= 64 ? 6 : BN <= 128 ? 4 : 2;
+  constexpr int STAGES = MPI == 2 || BN >= 128 ? 4 : 6;
   cudaError_t r;
   {
-    PersistentGroupedSched s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
+    PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
     EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
     if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
     r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e,
@@ -542,7 +552,7 @@ cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, uint32_
     if (r != cudaSuccess) return r;
     if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   }
-  PersistentGroupedSched s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
   EpiDown<BN> e{h->obuf, d};
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
   r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
@@ -554,8 +564,8 @@ cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, uint32_
 cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t timed) {
   const int bi = moe_bn_index(N, h->E);
   switch (bi) {
-    case 1: return moe_gemms_bn<64>(h, L, bi, l, timed);
-    default: return moe_gemms_bn<128>(h, L, bi, l, timed);
+    case 1: return h->moe_pair ? moe_gemms_bn<64, 2>(h, L, bi, l, timed) : moe_gemms_bn<64, 1>(h, L, bi, l, timed);
+    default: return moe_gemms_bn<128, 1>(h, L, bi, l, timed);
   }
 }
 
@@ -861,6 +871,8 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   if (const char* m = getenv("DLLM_OPROJ_MODE")) h->oproj_mode = atoi(m);
   if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
   if (const char* m = getenv("DLLM_ATTN_TP")) h->attn_tp = atoi(m) != 0;
+  if (const char* m = getenv("DLLM_PREFILL_TC")) h->prefill_tc = atoi(m) != 0;
+  if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
   h->router_tc = !h->dense && h->E % 32 == 0;
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;

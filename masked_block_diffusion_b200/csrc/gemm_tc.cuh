@@ -20,6 +20,7 @@ struct Tile {
   int m_valid;   // rows of the tile inside the problem
   int n_valid;   // columns of the tile inside the problem
   int mt, nt;    // dense: (m tile, n tile); grouped: (m tile inside the expert, expert)
+  int m_count = 1;   // m tiles of this work item (128 rows apart, sharing the B tile)
 };
 
 // One output tile per CTA over an M x N problem; m tiles vary fastest so that the CTAs
@@ -27,6 +28,7 @@ struct Tile {
 struct DenseSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = 1;
+  static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
   DLLM_DEV int count() const { return 1; }
@@ -51,6 +53,7 @@ template <int KS>
 struct DenseSplitKSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = KS;
+  static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
   DLLM_DEV int count() const { return 1; }
@@ -67,11 +70,12 @@ struct DenseSplitKSched {
   }
 };
 
-// Persistent grouped schedule over the routed experts only. One work item is one output
-// tile: (routed expert r, m tile, token chunk of BN). Items of expert r are numbered
-// m_tile * chunks_r + chunk from m_tiles * chunk_prefix[r] on, so the chunks of one
-// weight tile are neighbours: CTAs running them together read that tile from HBM once
-// and from L2 after. CTA c takes items c, c + gridDim.x, ...: every CTA gets the same
+// Persistent grouped schedule over the routed experts only. One work item is MPI output
+// tiles that share their token chunk: (routed expert r, m tiles MPI*g .. MPI*g+MPI-1,
+// token chunk of BN), so the chunk's B tile is loaded once for MPI weight tiles. Items
+// of expert r are numbered g * chunks_r + chunk from m_groups * chunk_prefix[r] on, so
+// the chunks of one weight tile are neighbours: CTAs running them together read that
+// tile from HBM once and from L2 after. CTA c takes items c, c + gridDim.x, ...: every CTA gets the same
 // number of equal-sized tiles whatever the routing skew, and streams them back to back
 // (the next tile's loads overlap this tile's epilogue through the double-buffered
 // accumulator).
@@ -79,10 +83,12 @@ struct DenseSplitKSched {
 // The routing tables are copied into shared memory once per CTA (stage(), run by every
 // thread before the roles split), so that finding an item's expert is a short search in
 // shared memory instead of a chain of dependent global loads on the producer's path.
+template <int MPI>
 struct PersistentGroupedSched {
   static constexpr int kMaxRouted = 256;
   static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
   static constexpr int kKSplit = 1;
+  static constexpr int kMPerItem = MPI;
   const int* offsets;        // [E+1] token ranges per expert
   const int* routed;         // [E] experts with at least one token, ascending
   const int* n_routed;       // [1]
@@ -117,26 +123,29 @@ struct PersistentGroupedSched {
     s_cnt = ct;
     n_routed = nn;
   }
-  DLLM_DEV int n_items() const { return chunk_prefix[*n_routed] * m_tiles; }
+  DLLM_DEV int m_groups() const { return (m_tiles + MPI - 1) / MPI; }
+  DLLM_DEV int n_items() const { return chunk_prefix[*n_routed] * m_groups(); }
   DLLM_DEV int count() const {
     const int n = n_items();
     return (int)blockIdx.x < n ? (n - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   }
   DLLM_DEV Tile tile(int j) const {
     const int i = blockIdx.x + j * gridDim.x;
-    int lo = 0, hi = *n_routed;   // chunk_prefix[lo] * m_tiles <= i < chunk_prefix[hi] * m_tiles
+    const int mg = m_groups();
+    int lo = 0, hi = *n_routed;   // chunk_prefix[lo] * mg <= i < chunk_prefix[hi] * mg
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (chunk_prefix[mid] * m_tiles <= i) lo = mid; else hi = mid;
+      if (chunk_prefix[mid] * mg <= i) lo = mid; else hi = mid;
     }
     const int e = routed[lo];
     const int ch = chunk_prefix[lo + 1] - chunk_prefix[lo];
-    const int local = i - chunk_prefix[lo] * m_tiles;
+    const int local = i - chunk_prefix[lo] * mg;
     const int chunk = local % ch;
     const int off = s_off[lo];
     const int cnt = s_cnt[lo];
     Tile t;
-    t.mt = local / ch;
+    t.mt = (local / ch) * MPI;
+    t.m_count = min(MPI, m_tiles - t.mt);
     t.nt = e;
     t.a_row = e * rows_per_expert + t.mt * 128;
     t.b_row = off + chunk * BN;
@@ -158,7 +167,8 @@ enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
 
 template <int BN, int STAGES, int SPLIT, class Epi, class Sched = DenseSched>
 struct GemmSmem {
-  static constexpr int kA = 128 * 64 * 2;
+  static constexpr int kAtile = 128 * 64 * 2;              // one 128-row A tile of a k block
+  static constexpr int kA = Sched::kMPerItem * kAtile;     // the item's A tiles
   static constexpr int kB = BN * 64 * 2;
   static constexpr int kA2 = SPLIT == kSplitA ? kA : 0;
   static constexpr int kB2 = SPLIT == kSplitB ? kB : 0;
@@ -223,19 +233,28 @@ DLLM_DEV bool splitk_reduce(int krank, uint32_t taddr, int r, uint8_t* part_smem
 #pragma unroll 1
   for (int p = 1; p < KS; ++p) {
     const uint32_t base = mapa_shared(smem_u32(part), p);
+    // up to 64 columns at a time: the remote loads are issued together, then added
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      tmem_ld16(taddr + c, v);
+    for (int c0 = 0; c0 < BN; c0 += 64) {
+      float4 w[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 w = ld_shared_cluster_v4(base + (uint32_t)((((c >> 2) + i) * 128 + r) * 16));
-        v[4 * i] += w.x;
-        v[4 * i + 1] += w.y;
-        v[4 * i + 2] += w.z;
-        v[4 * i + 3] += w.w;
+      for (int i = 0; i < 16; ++i)
+        if (c0 + 4 * i < BN) w[i] = ld_shared_cluster_v4(base + (uint32_t)((((c0 >> 2) + i) * 128 + r) * 16));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = c0 + 16 * q;
+        if (c >= BN) break;   // uniform
+        float v[16];
+        tmem_ld16(taddr + c, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[4 * i] += w[4 * q + i].x;
+          v[4 * i + 1] += w[4 * q + i].y;
+          v[4 * i + 2] += w[4 * q + i].z;
+          v[4 * i + 3] += w[4 * q + i].w;
+        }
+        tmem_st16(taddr + c, v);
       }
-      tmem_st16(taddr + c, v);
     }
   }
   return true;
@@ -250,8 +269,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   using L = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>;
   constexpr int kAccN = SPLIT == kSplitB ? 2 * BN : BN;   // kSplitB: columns [0, BN) hi, [BN, 2 BN) lo
   static_assert(kAccN <= 256, "UMMA N");
+  constexpr int MPI = Sched::kMPerItem;                   // accumulators per work item
+  static_assert(MPI == 1 || SPLIT != kSplitA, "several m tiles per item share B only");
   constexpr int kCols = tmem_cols_for(kAccN);
-  constexpr int kTmemCols = kCols * ACC_BUFS;
+  constexpr int kTmemCols = kCols * ACC_BUFS * MPI;
   static_assert(kTmemCols <= 512, "TMEM has 512 columns");
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, kAccN);
   constexpr int KS = Sched::kKSplit;
@@ -329,8 +350,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       const Tile t = sched.tile(j);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
-        tma_load_2d(sA + stage * L::kA, &tma_a, &full[stage], kb * 64, t.a_row, pol_a);
+        mbar_arrive_expect_tx(&full[stage], L::kStageBytes - (MPI - t.m_count) * L::kAtile);
+        for (int u = 0; u < t.m_count; ++u)
+          tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
         if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
         tma_load_2d(sB + stage * L::kBStage, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
         if (SPLIT == kSplitB) tma_load_2d(sB2 + stage * L::kBStage, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
@@ -360,7 +382,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       const uint32_t acc_phase = (j / ACC_BUFS) & 1;
       if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * kCols;
+      const int mc = MPI > 1 ? sched.tile(j).m_count : 1;
+      const uint32_t d_tmem = tmem_base + acc * MPI * kCols;
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -373,6 +396,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
                     (kb != kb_begin || kk != 0) ? 1u : 0u);
           if (SPLIT == kSplitA)
             umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc, 1);
+#pragma unroll
+          for (int u = 1; u < MPI; ++u)
+            if (u < mc)
+              umma_bf16(d_tmem + u * kCols, sdesc_k_sw128(a0 + u * L::kAtile + kk * 32), sdesc_k_sw128(b0 + kk * 32),
+                        kIdesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -401,27 +429,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         break;
       }
       tc_fence_after();
-      const Tile t = sched.tile(j);
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * kCols;
-      if constexpr (SPLIT == kSplitB) {
-        // D = D_hi + D_lo, into the first BN columns the epilogue reads
+      const Tile t0 = sched.tile(j);
+      bool aborted = false;
+      for (int u = 0; u < t0.m_count; ++u) {   // the item's m tiles, 128 rows apart
+        Tile t = t0;
+        t.mt += u;
+        t.a_row += u * 128;
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (acc * MPI + u) * kCols;
+        if constexpr (SPLIT == kSplitB) {
+          // D = D_hi + D_lo, into the first BN columns the epilogue reads
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          float hi[16], lo[16];
-          tmem_ld16(taddr + c, hi);
-          tmem_ld16(taddr + BN + c, lo);
+          for (int c = 0; c < BN; c += 16) {
+            float hi[16], lo[16];
+            tmem_ld16(taddr + c, hi);
+            tmem_ld16(taddr + BN + c, lo);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) hi[i] += lo[i];
-          tmem_st16(taddr + c, hi);
+            for (int i = 0; i < 16; ++i) hi[i] += lo[i];
+            tmem_st16(taddr + c, hi);
+          }
         }
-      }
-      if constexpr (KS > 1) {
-        if (!splitk_reduce<BN, KS>(krank, taddr, r, smem, peer_ready, abort_flag, err)) {
-          *abort_flag = 1;
-          break;
+        if constexpr (KS > 1) {
+          if (!splitk_reduce<BN, KS>(krank, taddr, r, smem, peer_ready, abort_flag, err)) {
+            *abort_flag = 1;
+            aborted = true;
+            break;
+          }
         }
+        if (krank == 0) epi(t, taddr, r, epi_smem);
       }
-      if (krank == 0) epi(t, taddr, r, epi_smem);
+      if (aborted) break;
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -492,23 +528,47 @@ struct EpiQKV {
     else if (hh < H + Hkv) dst = kc + (((long)slot[b] * Hkv + (hh - H)) * max_ctx + pos) * HD;
     else dst = vc + (((long)slot[b] * Hkv + (hh - H - Hkv)) * max_ctx + pos) * HD;
     if (hh < H + Hkv) {
+      static_assert(HALF % 8 == 0, "RoPE in 8-pair chunks");
+      // four 8-pair chunks at a time: their cos / sin loads are issued together, ahead of
+      // the TMEM reads, instead of one dependent global load per chunk
 #pragma unroll 1
-      for (int c = 0; c < HALF; c += 8) {
-        float a[8], bb[8];
-        tmem_ld8(taddr + c, a);
-        tmem_ld8(taddr + c + HALF, bb);
-        if (valid) {
-          const float* cs = rope_cos + (long)pos * HALF + c;
-          const float* sn = rope_sin + (long)pos * HALF + c;
-          uint32_t lo[4], hi[4];
+      for (int c0 = 0; c0 < HALF; c0 += 32) {
+        float4 cs[4][2], sn[4][2];
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
-            float c0 = cs[i], c1 = cs[i + 1], s0 = sn[i], s1 = sn[i + 1];
-            lo[i / 2] = pack_bf16x2(a[i] * c0 - bb[i] * s0, a[i + 1] * c1 - bb[i + 1] * s1);
-            hi[i / 2] = pack_bf16x2(bb[i] * c0 + a[i] * s0, bb[i + 1] * c1 + a[i + 1] * s1);
+        for (int q = 0; q < 4; ++q) {
+          const int c = c0 + 8 * q;
+          if (c < HALF && valid) {
+            const float4* pc = reinterpret_cast<const float4*>(rope_cos + (long)pos * HALF + c);
+            const float4* ps = reinterpret_cast<const float4*>(rope_sin + (long)pos * HALF + c);
+            cs[q][0] = pc[0];
+            cs[q][1] = pc[1];
+            sn[q][0] = ps[0];
+            sn[q][1] = ps[1];
+          } else {
+            cs[q][0] = cs[q][1] = sn[q][0] = sn[q][1] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          *reinterpret_cast<uint4*>(dst + c + HALF) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = c0 + 8 * q;
+          if (c >= HALF) break;   // warp-uniform
+          float a[8], bb[8];
+          tmem_ld8(taddr + c, a);
+          tmem_ld8(taddr + c + HALF, bb);
+          if (valid) {
+            const float cv[8] = {cs[q][0].x, cs[q][0].y, cs[q][0].z, cs[q][0].w,
+                                 cs[q][1].x, cs[q][1].y, cs[q][1].z, cs[q][1].w};
+            const float sv[8] = {sn[q][0].x, sn[q][0].y, sn[q][0].z, sn[q][0].w,
+                                 sn[q][1].x, sn[q][1].y, sn[q][1].z, sn[q][1].w};
+            uint32_t lo[4], hi[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              lo[i / 2] = pack_bf16x2(a[i] * cv[i] - bb[i] * sv[i], a[i + 1] * cv[i + 1] - bb[i + 1] * sv[i + 1]);
+              hi[i / 2] = pack_bf16x2(bb[i] * cv[i] + a[i] * sv[i], bb[i + 1] * cv[i + 1] + a[i + 1] * sv[i + 1]);
+            }
+            *reinterpret_cast<uint4*>(dst + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4*>(dst + c + HALF) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          }
         }
       }
     } else {
@@ -532,22 +592,31 @@ struct EpiResidual {
   float* x;
   int ldx;
   DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    static_assert(BN % 64 == 0, "64-column groups");
     float* row = x + (long)(t.a_row + r) * ldx + t.b_row;
+    const bool valid = r < t.m_valid;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      tmem_ld16(taddr + c, v);
-      if (r < t.m_valid) {
-        float4* p = reinterpret_cast<float4*>(row + c);
+    for (int c0 = 0; c0 < BN; c0 += 64) {
+      // the row's 64 residual values are loaded together, then the accumulator
+      float4 o[16];
+      float4* p = reinterpret_cast<float4*>(row + c0);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[i] = valid ? p[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[16];
+        tmem_ld16(taddr + c0 + 16 * q, v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float4 o = p[i];
-          o.x += v[4 * i + 0];
-          o.y += v[4 * i + 1];
-          o.z += v[4 * i + 2];
-          o.w += v[4 * i + 3];
-          p[i] = o;
+          o[4 * q + i].x += v[4 * i + 0];
+          o[4 * q + i].y += v[4 * i + 1];
+          o[4 * q + i].z += v[4 * i + 2];
+          o[4 * q + i].w += v[4 * i + 3];
         }
+      }
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = o[i];
       }
     }
   }
