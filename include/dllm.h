@@ -93,7 +93,8 @@ typedef struct {
  *   (dense: Wg, Wu, Wd); final_norm[d]; head[V][d].
  * weights_on_device: 1 if `weights` is device memory, 0 for host memory. The blob is
  * copied and repacked; the caller may free it after the call returns.
- * cuda_stream: a cudaStream_t (NULL = the legacy default stream).
+ * cuda_stream: a cudaStream_t, used as given; NULL: the handle creates its own non-blocking
+ *   stream (destroyed with the handle).
  * Errors: DLLM_E_INVAL (shape), DLLM_E_OOM, DLLM_E_CUDA. On error *out is NULL. */
 int dllm_create(const dllm_config* cfg, const void* weights, size_t weight_bytes, int weights_on_device,
                 void* cuda_stream, dllm_handle** out);

@@ -1,23 +1,27 @@
-// Tensor-core (tcgen05 / TMEM) attention for the bidirectional canvas pass.
+// Tensor-core (tcgen05 / TMEM) attention for the canvas passes and the prompt prefill.
 //
 // Every canvas query of request b sees keys 0 .. P_b + C - 1: the cached prefix and the
 // canvas, whose K/V the QKV epilogue has written at P_b .. P_b + C - 1 ("Diffusion LLMs:
-// what changes ...", section 2 property 1 and section 4.2 "Block decoding").
+// what changes ...", section 2 property 1 and section 4.2 "Block decoding"). A prompt
+// token (causal prefill) sees the keys up to its own position.
 //
 // One CTA = one 128-row query tile of one KV head over one split of the key range. The
 // tile holds the GQA group's heads for 128 / group queries (row r = query r / group,
 // head r % group), so each K/V block is loaded once for all heads that read it.
 // Roles (192 threads):
-//   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys (2-stage ring);
+//   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys into two
+//                  three-stage rings (a K stage is refilled once the S = Q K^T that read
+//                  it completes, a V stage once its P V does);
 //   warp 1         TMEM allocation; lane 0 issues S = Q K^T into one of two TMEM S
 //                  buffers, then O += P_hi V + P_lo V for the previous block, so the next
 //                  block's S overlaps this block's softmax;
 //   warps 2..5     one query row per thread: read S from TMEM, scale and mask, running
-//                  maximum, P = exp2(s - m_ref) written to shared memory as a bf16 (hi, lo)
-//                  pair in the 128-byte-swizzled K-major layout the MMA reads, running sum;
-//                  O in TMEM is rescaled only when the maximum grows by more than 2^8
-//                  (P stays below 256, exact enough, and rescales are rare). At the end
-//                  they read O, divide by the sum and write the output (or a split partial).
+//                  maximum, P = exp2(s - m_ref) as a bf16 (hi, lo) pair written back into
+//                  TMEM with tcgen05.st (the P V MMA reads its A operand from TMEM, so P
+//                  needs no shared memory), running sum; O in TMEM is rescaled only when
+//                  the maximum grows by more than 2^8 (P stays below 256, exact enough,
+//                  and rescales are rare). At the end they read O, divide by the sum and
+//                  write the output (or a split partial).
 // Every wait is bounded, as in gemm_tc.cuh.
 #pragma once
 
@@ -42,27 +46,6 @@ struct AttnTcParams {
   int* err;
 };
 
-template <int HD>
-struct AttnTcCfg {
-  static constexpr int BK = 64;                          // keys per block
-  static constexpr int ATOMS = (HD + 63) / 64;           // 64-element (128-byte) chunks of a row
-  static constexpr int STAGES = 2;                       // K/V ring
-  static constexpr int kQ = ATOMS * 128 * 128;           // Q tile bytes
-  static constexpr int kKatom = BK * 128;                // one 64-dim chunk of a K (or V) block
-  static constexpr int kKV = ATOMS * kKatom;             // K block bytes (V block the same)
-  static constexpr int kP = 128 * 128;                   // P tile (128 rows x 64 keys bf16)
-  static constexpr int kOffK = kQ;
-  static constexpr int kOffV = kOffK + STAGES * kKV;
-  static constexpr int kOffP = kOffV + STAGES * kKV;     // [buf 2][hi, lo]
-  static constexpr int kOffBar = kOffP + 4 * kP;
-  static constexpr int kTotal = kOffBar + 256 + 1024;
-  static constexpr int kSCols = BK;                      // TMEM columns of one S buffer
-  static constexpr int kOCol = 2 * BK;                   // O accumulator column
-  static constexpr int kTmemCols = 512;
-  static_assert(kOCol + HD <= kTmemCols, "TMEM");
-  static_assert(kTotal <= 232448, "shared memory");
-};
-
 // Shared-memory descriptor of an MN-major operand stored with the 128-byte swizzle:
 // 64 contiguous elements (128 B) along N per row, rows along K 128 B apart, 8-row groups
 // 1024 B apart (SBO), 64-element N chunks `lbo` bytes apart (LBO).
@@ -83,8 +66,6 @@ DLLM_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
       "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-
-DLLM_DEV void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 2^x with the hardware approximation (PTX ex2.approx; relative error about 2^-22,
 // far below the 2^-16 kept by the (hi, lo) bf16 pair P is stored as). ex2(-inf) = 0.
@@ -108,290 +89,10 @@ DLLM_DEV bool sm_all(bool ok) {
   return r != 0;
 }
 
-// Warps 2..5 of attn_tc_kernel: thread r owns query row r of the tile (TMEM lane r).
-template <int HD>
-DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint8_t* sP, uint64_t* s_full, uint64_t* s_empty,
-                           uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final,
-                           volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
-                           int nblk) {
-  using G = AttnTcCfg<HD>;
-  constexpr int BK = G::BK;
-  const int q = warp & 3;
-  const int r = q * 32 + lane;
-  const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-  float m_ref = -INFINITY, l = 0.f;
-  bool ok = true;
-  for (int j = 0; j < nblk; ++j) {
-    const int sb = j & 1;
-    if (!sm_all(mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
-    tc_fence_after();
-    static_assert(BK == 64, "one 64-column TMEM load per block");
-    float s[BK];
-    tmem_ld64(lane_base + sb * G::kSCols, s);
-    tc_fence_before();
-    mbar_arrive(&s_empty[sb]);
-    const int key0 = ks + j * BK;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < BK; ++c) {
-      const float v = (key0 + c < ke) ? s[c] * p.scale_log2 : -INFINITY;
-      s[c] = v;
-      mx = fmaxf(mx, v);
-    }
-    if (j == 0) {
-      m_ref = mx;   // block 0 always holds a visible key
-    } else {
-      const bool need = mx > m_ref + 8.0f;
-      if (__any_sync(0xffffffffu, need)) {
-        // the O rows of this warp are rescaled in TMEM once the previous block's P V
-        // has landed (its completion is phase j-1 of o_done)
-        const bool got = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
-        if (got) {
-          tc_fence_after();
-          const float f = need ? exp2f(m_ref - mx) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < HD; c += 16) {
-            float v[16];
-            tmem_ld16(lane_base + G::kOCol + c, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= f;
-            tmem_st16(lane_base + G::kOCol + c, v);
-          }
-          tc_fence_before();
-          if (need) {
-            l *= f;
-            m_ref = mx;
-          }
-        } else {
-          ok = false;   // all four warps leave together at the next agreement below
-        }
-      }
-    }
-    uint32_t hi[BK / 2], lo[BK / 2];
-    float psum = 0.f;
-#pragma unroll
-    for (int c = 0; c < BK; c += 2) {
-      const float p0 = ex2_approx(s[c] - m_ref), p1 = ex2_approx(s[c + 1] - m_ref);
-      psum += p0 + p1;
-      split_bf16x2(p0, p1, hi[c / 2], lo[c / 2]);
-    }
-    l += psum;
-    const int pb = j & 1;
-    if (!sm_all(ok && mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, abort_flag))) { ok = false; break; }
-    uint8_t* ph = sP + (pb * 2 + 0) * G::kP + r * 128;
-    uint8_t* pl = sP + (pb * 2 + 1) * G::kP + r * 128;
-#pragma unroll
-    for (int cc = 0; cc < BK / 8; ++cc) {   // 16-byte chunk cc of the row, 128-byte swizzle
-      const int sw = (cc ^ (r & 7)) * 16;
-      *reinterpret_cast<uint4*>(ph + sw) = make_uint4(hi[4 * cc], hi[4 * cc + 1], hi[4 * cc + 2], hi[4 * cc + 3]);
-      *reinterpret_cast<uint4*>(pl + sw) = make_uint4(lo[4 * cc], lo[4 * cc + 1], lo[4 * cc + 2], lo[4 * cc + 3]);
-    }
-    fence_async_smem();
-    mbar_arrive(&p_full[pb]);
-  }
-  if (ok) ok = sm_all(mbar_wait(o_final, 0, abort_flag));
-  if (!ok) {
-    atomicExch(p.err, kDevTimeoutEpilogue);
-    *abort_flag = 1;
-    return;
-  }
-  tc_fence_after();
-  // output row r: query q0 + r / group of head g * group + r % group
-  const int i = r / p.group;
-  const int h = blockIdx.y * p.group + r % p.group;
-  const bool valid = q0 + i < p.tok_per_req;
-  const long t = (long)b * p.tok_per_req + q0 + i;
-  const float inv = 1.0f / l;
-#pragma unroll 1
-  for (int c = 0; c < HD; c += 16) {
-    float v[16];
-    tmem_ld16(lane_base + G::kOCol + c, v);
-    if (!valid) continue;
-    if (p.n_splits == 1) {
-      uint32_t hw[8], lw[8];
-#pragma unroll
-      for (int e = 0; e < 16; e += 2) split_bf16x2(v[e] * inv, v[e + 1] * inv, hw[e / 2], lw[e / 2]);
-      bf16_t* oh = p.out + (t * p.H + h) * HD + c;
-      bf16_t* ol = p.out_lo + (t * p.H + h) * HD + c;
-      reinterpret_cast<uint4*>(oh)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      reinterpret_cast<uint4*>(oh)[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-      reinterpret_cast<uint4*>(ol)[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      reinterpret_cast<uint4*>(ol)[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-    } else {
-      float4* po = reinterpret_cast<float4*>(p.part_o + (((long)sp * p.T + t) * p.H + h) * HD + c);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        po[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv, v[4 * e + 3] * inv);
-    }
-  }
-  if (valid && p.n_splits > 1) p.part_lse[((long)sp * p.T + t) * p.H + h] = m_ref + __log2f(l);
-}
-
-template <int HD>
-__global__ void __launch_bounds__(192, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, AttnTcParams p) {
-  using G = AttnTcCfg<HD>;
-  constexpr int BK = G::BK, AT = G::ATOMS, ST = G::STAGES;
-  constexpr uint32_t kIdQK = idesc_bf16_f32(128, BK);
-  constexpr uint32_t kIdPV = idesc_bf16_f32_bmn(128, HD);
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + G::kOffK;
-  uint8_t* sV = smem + G::kOffV;
-  uint8_t* sP = smem + G::kOffP;
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + G::kOffBar);
-  uint64_t* kv_full = q_full + 1;
-  uint64_t* kv_empty = kv_full + ST;
-  uint64_t* s_full = kv_empty + ST;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_done = p_empty + 2;
-  uint64_t* o_final = o_done + 1;
-  uint64_t* drain = o_final + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  pdl_wait();   // pos0 and the K / V written by the QKV projection
-  const int qt = blockIdx.x, g = blockIdx.y;
-  const int b = blockIdx.z / p.n_splits, sp = blockIdx.z % p.n_splits;
-  const int C = p.tok_per_req, grp = p.group;
-  const int qpt = 128 / grp;
-  const int q0 = qt * qpt;
-  const int kend = p.pos0[b] + C;
-  const int ks = sp * p.split_keys;
-  const int ke = min(kend, ks + p.split_keys);
-  if (q0 >= C || ks >= ke) return;   // uniform over the CTA, before any barrier or TMEM use
-  const int nblk = (ke - ks + BK - 1) / BK;
-  const int kv_row0 = (p.slot[b] * p.Hkv + g) * p.max_ctx;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&p_empty[i], 1);
-    }
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, G::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  pdl_trigger();   // after the TMEM allocation
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    const uint64_t pol = policy_evict_last();   // each K/V block is read by every query tile of its head
-    bool ok = true;
-    mbar_arrive_expect_tx(q_full, G::kQ);
-    for (int a = 0; a < AT; ++a) tma_load_3d(sQ + a * 128 * 128, &tm_q, q_full, a * 64, g * grp, b * C + q0);
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % ST;
-      if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      mbar_arrive_expect_tx(&kv_full[st], 2 * G::kKV);
-      const int row = kv_row0 + ks + j * BK;
-      for (int a = 0; a < AT; ++a) {
-        tma_load_2d(sK + st * G::kKV + a * G::kKatom, &tm_k, &kv_full[st], a * 64, row, pol);
-        tma_load_2d(sV + st * G::kKV + a * G::kKatom, &tm_v, &kv_full[st], a * 64, row, pol);
-      }
-    }
-    if (!ok) {
-      atomicExch(p.err, kDevTimeoutProducer);
-      *abort_flag = 1;
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    bool ok = mbar_wait(q_full, 0, abort_flag);
-    const uint32_t d_o = tmem_base + G::kOCol;
-    auto issue_pv = [&](int jj) -> bool {
-      const int pb = jj & 1, st = jj % ST;
-      if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t ph = smem_u32(sP + (pb * 2 + 0) * G::kP);
-      const uint32_t pl = smem_u32(sP + (pb * 2 + 1) * G::kP);
-      const uint32_t v0 = smem_u32(sV + st * G::kKV);
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t bdesc = sdesc_mn_sw128(v0 + kk * 16 * 128, G::kKatom);
-        umma_bf16(d_o, sdesc_k_sw128(ph + kk * 32), bdesc, kIdPV, (jj | kk) != 0);
-        umma_bf16(d_o, sdesc_k_sw128(pl + kk * 32), bdesc, kIdPV, 1);
-      }
-      umma_commit(&p_empty[pb]);
-      umma_commit(&kv_empty[st]);
-      umma_commit(o_done);
-      return true;
-    };
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % ST, sb = j & 1;
-      if (!mbar_wait(&kv_full[st], (j / ST) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_s = tmem_base + sb * G::kSCols;
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK + st * G::kKV);
-#pragma unroll
-      for (int a = 0; a < AT; ++a)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(d_s, sdesc_k_sw128(q_base + a * 128 * 128 + kk * 32),
-                    sdesc_k_sw128(k_base + a * G::kKatom + kk * 32), kIdQK, (a | kk) != 0);
-      umma_commit(&s_full[sb]);
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
-    }
-    if (ok && !issue_pv(nblk - 1)) ok = false;
-    if (ok) umma_commit(o_final);
-    if (!ok) {
-      atomicExch(p.err, kDevTimeoutMma);
-      *abort_flag = 1;
-    }
-    umma_commit(drain);
-    unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
-  } else if (warp >= 2) {
-    softmax_rows<HD>(p, tmem_base, sP, s_full, s_empty, p_full, p_empty, o_done, o_final, abort_flag, warp, lane,
-                     q0, b, sp, ks, ke, nblk);
-  }
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem_base, G::kTmemCols);
-  }
-}
-
-// ------------------------------------------------------------------------------------
-// Variant with P kept in tensor memory. The softmax threads write P (hi, lo) into TMEM
-// with tcgen05.st and the P V product reads it as the A operand straight from TMEM, so
-// P needs no shared memory, no swizzled stores and no proxy fence; the shared memory it
-// frees holds a third K and V stage, and K and V have rings of their own: a K stage is
-// refilled once the S = Q K^T that read it completes, a V stage once its P V does.
-//
 // TMEM columns: S buffers 0..63 and 64..127; P buffer pb at 128 + 64 pb (hi in the first
 // 32 columns, lo in the next 32, two bf16 per column); O from column 256.
 template <int HD>
-struct AttnTpCfg {
+struct AttnTcCfg {
   static constexpr int BK = 64;
   static constexpr int ATOMS = (HD + 63) / 64;
   static constexpr int STAGES = 3;
@@ -411,11 +112,11 @@ struct AttnTpCfg {
 };
 
 template <int HD>
-DLLM_DEV void softmax_rows_tp(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
+DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
                               uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final,
                               volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
                               int nblk) {
-  using G = AttnTpCfg<HD>;
+  using G = AttnTcCfg<HD>;
   constexpr int BK = G::BK;
   const int q = warp & 3;
   const int r = q * 32 + lane;
@@ -528,9 +229,9 @@ DLLM_DEV void softmax_rows_tp(const AttnTcParams& p, uint32_t tmem_base, uint64_
 
 template <int HD>
 __global__ void __launch_bounds__(192, 1)
-attn_tp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, AttnTcParams p) {
-  using G = AttnTpCfg<HD>;
+  using G = AttnTcCfg<HD>;
   constexpr int BK = G::BK, AT = G::ATOMS, ST = G::STAGES;
   constexpr uint32_t kIdQK = idesc_bf16_f32(128, BK);
   constexpr uint32_t kIdPV = idesc_bf16_f32_bmn(128, HD);
@@ -674,7 +375,7 @@ attn_tp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     unsigned long long t0 = global_ns();
     while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
   } else if (warp >= 2) {
-    softmax_rows_tp<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final, abort_flag, warp, lane, q0,
+    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final, abort_flag, warp, lane, q0,
                         b, sp, ks, ke, nblk);
   }
   __syncwarp();

@@ -155,7 +155,6 @@ struct dllm_handle {
   bool attn_tc = false;     // canvas passes use the tensor-core attention
   int oproj_mode = 0;       // O projection on few tiles: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
-  bool attn_tp = true;      // tensor-core attention keeps P in TMEM (three-stage K / V rings)
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
   bool moe_pair = true;     // grouped GEMMs at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
@@ -197,6 +196,7 @@ struct dllm_handle {
   int32_t* n_routed = nullptr;      // [1]
   int32_t* chunk_prefix = nullptr;  // [E+1] chunk-count prefix over the routed experts
   int32_t* routed_stat = nullptr;   // [L] n_routed per layer of the last timed pass
+  int32_t* bn_sel = nullptr;        // [1] chunk width the permute kernel chose for this layer
   int last_T = 0;                   // tokens of the last timed pass
 };
 
@@ -423,20 +423,11 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.err = h->d_err;
   dim3 grid(ceil_div((long)tok_per_req * p.group, 128), c.n_kv_heads, nreq * splits);
-  cudaError_t r;
-  if (h->attn_tp || causal) {
-    constexpr int smem = AttnTpCfg<HD>::kTotal;
-    r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tp_kernel<HD>),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (r != cudaSuccess) return r;
-    r = launch_k(h, attn_tp_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
-  } else {
-    constexpr int smem = AttnTcCfg<HD>::kTotal;
-    r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (r != cudaSuccess) return r;
-    r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
-  }
+  constexpr int smem = AttnTcCfg<HD>::kTotal;
+  cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (r != cudaSuccess) return r;
+  r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
   h->launches++;
   if (r != cudaSuccess) return r;
   if (splits > 1) {
@@ -534,39 +525,62 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
-// MPI = 2 (BN = 64): items of two weight tiles sharing the token chunk (48 KB stages);
-// MPI = 1: one weight tile per item (at BN = 128 the two accumulator buffers take all
-// 512 TMEM columns).
-template <int BN, int MPI>
-cudaError_t moe_gemms_bn(dllm_handle* h, const LayerW& L, int bi, int l, uint32_t timed) {
+// One grouped gate/up + down pair at chunk width BN with MPI weight tiles per work item
+// and ACC accumulator buffers (MPI * ACC * 2 BN TMEM columns <= 512). gate: the device
+// chunk-width choice this launch serves (nullptr: always works).
+template <int BN, int MPI, int ACC>
+cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L, int bi, const int* gate) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int STAGES = MPI == 2 || BN >= 128 ? 4 : 6;
-  cudaError_t r;
-  {
-    PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
-    EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-    if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-    r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e,
-                                            nullptr, &h->tm_xg_lo[bi]);
-    if (r != cudaSuccess) return r;
-    if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
-  }
-  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
-  EpiDown<BN> e{h->obuf, d};
-  if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  r = launch_gemm<BN, STAGES, 2, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
-                                          &h->tm_h_lo[bi]);
-  if (r != cudaSuccess) return r;
-  return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
+  constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN, gate};
+  EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e, nullptr,
+                                               &h->tm_xg_lo[bi]);
 }
 
+template <int BN, int MPI, int ACC>
+cudaError_t moe_down(dllm_handle* h, const LayerW& L, int bi, const int* gate) {
+  const auto& c = h->c;
+  const int F = c.ffn_dim, d = c.d_model;
+  constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN, gate};
+  EpiDown<BN> e{h->obuf, d};
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
+                                               &h->tm_h_lo[bi]);
+}
+
+// Grouped expert GEMMs of one layer. With many tokens per expert (prefill, large
+// batches) the chunk width is 128, one weight tile per item, two accumulator buffers.
+// Otherwise the permute kernel picks the width from the routing (64 for spread routing,
+// 128 for few heavily loaded experts) and both variants are launched, the unchosen one
+// doing nothing: 64 with two weight tiles per item and two buffers, or 128 with two
+// weight tiles per item and one buffer (about one item per SM then).
 cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t timed) {
   const int bi = moe_bn_index(N, h->E);
-  switch (bi) {
-    case 1: return h->moe_pair ? moe_gemms_bn<64, 2>(h, L, bi, l, timed) : moe_gemms_bn<64, 1>(h, L, bi, l, timed);
-    default: return moe_gemms_bn<128, 1>(h, L, bi, l, timed);
+  cudaError_t r;
+  if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
+  if (bi >= 2) {
+    r = moe_gate_up<128, 1, 2>(h, L, 2, nullptr);
+  } else if (!h->moe_pair) {
+    r = moe_gate_up<64, 1, 2>(h, L, 1, nullptr);
+  } else {
+    r = moe_gate_up<64, 2, 2>(h, L, 1, h->bn_sel);
+    if (r == cudaSuccess) r = moe_gate_up<128, 2, 1>(h, L, 2, h->bn_sel);
   }
+  if (r != cudaSuccess) return r;
+  if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
+  if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
+  if (bi >= 2) {
+    r = moe_down<128, 1, 2>(h, L, 2, nullptr);
+  } else if (!h->moe_pair) {
+    r = moe_down<64, 1, 2>(h, L, 1, nullptr);
+  } else {
+    r = moe_down<64, 2, 2>(h, L, 1, h->bn_sel);
+    if (r == cudaSuccess) r = moe_down<128, 2, 1>(h, L, 2, h->bn_sel);
+  }
+  if (r != cudaSuccess) return r;
+  return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
 
 // ------------------------------------------------------------------ the pass
@@ -600,11 +614,12 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       if (h->router_tc) {
         CK(router_gemm(h, L, T));
       } else {
-        CK(launch_k(h, router_kernel, dim3(dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp))), dim3(256), kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E,
-                                                                 h->rlogits));
+        CK(launch_k(h, router_kernel, dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp)), dim3(256),
+                    kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits));
         h->launches++;
       }
-      CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k, h->tk_idx, h->tk_w));
+      CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
+                  h->tk_idx, h->tk_w));
       h->launches++;
       if (record) {
         CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
@@ -613,8 +628,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                            cudaMemcpyDeviceToDevice, h->st));
       }
       if (h->force_routing && T == h->force_T) {
-        CK(launch_k(h, force_route_kernel, dim3(ceil_div(T, 128)), dim3(128), 0, 
-            h->rlogits, h->dbg_force + (size_t)l * h->force_T * h->k, T, h->E, h->k, h->tk_idx, h->tk_w));
+        CK(launch_k(h, force_route_kernel, dim3(ceil_div(T, 128)), dim3(128), 0, h->rlogits,
+                    h->dbg_force + (size_t)l * h->force_T * h->k, T, h->E, h->k, h->tk_idx, h->tk_w));
         h->launches++;
       }
     } else {
@@ -622,9 +637,9 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       h->launches++;
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
-                                                               h->row_token, h->routed, h->n_routed,
-                                                               h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
-                                                               timed ? h->routed_stat + l : nullptr));
+                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)], 128,
+                (moe_bn_index(N, h->E) < 2 && h->moe_pair) ? h->bn_sel : nullptr,
+                timed ? h->routed_stat + l : nullptr));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(128), 0, h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
@@ -632,8 +647,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
     const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
     if (next_gain)
-      CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d, next_gain, c.rms_eps,
-                                                h->y, h->y_lo));
+      CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d,
+                  next_gain, c.rms_eps, h->y, h->y_lo));
     else
       CK(launch_k(h, combine_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d));
     h->launches++;
@@ -651,7 +666,8 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
   const auto& c = h->c;
   const int C = c.canvas, T = B * C, d = c.d_model;
   const int splits = attn_splits(h, B);
-  CK(launch_k(h, embed_kernel, dim3(T), dim3(128), 0, h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d, h->x));
+  CK(launch_k(h, embed_kernel, dim3(T), dim3(128), 0, h->emb, h->canvas, mode == 0 ? h->mask : nullptr, c.mask_id, d,
+              h->x));
   h->launches++;
   const uint32_t tm = (h->timing && mode == 0) ? h->tmask : 0u;
   int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0,
@@ -667,12 +683,11 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
     DenseSched s{T, mt, 256};
     CK((launch_gemm<256, 3, 1, kSplitA>(h, dim3(mt * nvt), h->tm_y, h->tm_head, d / 64, 0, s, e, &h->tm_y_lo)));
   }
-  CK(launch_k(h, lm_merge_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->lm_m, h->lm_s, h->lm_i, T, nvt, h->conf,
-                                                                  h->argmax));
+  CK(launch_k(h, lm_merge_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->lm_m, h->lm_s, h->lm_i, T, nvt,
+              h->conf, h->argmax));
   const int threads = ceil_div(C, 32) * 32;
-  CK(launch_k(h, commit_kernel, dim3(B), dim3(threads), C * (sizeof(float) + 1), h->canvas, h->mask, h->conf, h->argmax, C,
-                                                                 h->d_policy, h->d_step, h->d_remaining, nullptr,
-                                                                 nullptr));
+  CK(launch_k(h, commit_kernel, dim3(B), dim3(threads), C * (sizeof(float) + 1), h->canvas, h->mask, h->conf,
+              h->argmax, C, h->d_policy, h->d_step, h->d_remaining, nullptr, nullptr));
   h->launches += 2;
   CK(tmark(h, tm, DLLM_TIMING_HEAD, 0, 1));
   CK(cudaGetLastError());
@@ -870,7 +885,6 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   h->attn_tc = (128 % (H / Hkv) == 0) && !getenv("DLLM_ATTN_LEGACY");
   if (const char* m = getenv("DLLM_OPROJ_MODE")) h->oproj_mode = atoi(m);
   if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_ATTN_TP")) h->attn_tp = atoi(m) != 0;
   if (const char* m = getenv("DLLM_PREFILL_TC")) h->prefill_tc = atoi(m) != 0;
   if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
   h->router_tc = !h->dense && h->E % 32 == 0;
@@ -977,6 +991,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->n_routed, 1);
   DA(h->chunk_prefix, h->E + 1);
   DA(h->routed_stat, c.n_layers);
+  DA(h->bn_sel, 1);
 
   DA(h->slot_of, (size_t)N);
   DA(h->row_token, (size_t)N);
@@ -1159,8 +1174,8 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
   if (r) return r;
   if ((r = upload_policy(h, policy, max_steps))) return r;
   const int C = h->c.canvas, B = req_count;
-  CK(launch_k(h, canvas_init_kernel, dim3(ceil_div((long)B * C, 256)), dim3(256), 0, h->canvas, h->mask, B * C, h->c.mask_id,
-                                                                    h->d_step, B));
+  CK(launch_k(h, canvas_init_kernel, dim3(ceil_div((long)B * C, 256)), dim3(256), 0, h->canvas, h->mask, B * C,
+              h->c.mask_id, h->d_step, B));
   h->launches++;
   std::vector<int> done_at(B, -1);
   int s = 0;
