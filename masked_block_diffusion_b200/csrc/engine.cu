@@ -87,7 +87,7 @@ struct LayerW {
   bf16_t* wr = nullptr;     // [E][d]
   bf16_t* wgu = nullptr;    // [E][2F][d]: per 128-row block, 64 gate rows then the 64 matching up rows
   bf16_t* wd = nullptr;     // [E][d][F]
-  CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wr;
+  CUtensorMap tm_wqkv, tm_wo, tm_wo128, tm_wgu, tm_wd, tm_wr;
   CUtensorMap tm_k, tm_v;   // this layer's K / V cache as [slot][Hkv][max_ctx] rows of hd
 };
 
@@ -151,9 +151,11 @@ struct dllm_handle {
   bf16_t* hbuf_lo = nullptr;
   CUtensorMap tm_y, tm_ao, tm_xg[4], tm_h[4];
   CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
+  CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // canvas passes use the tensor-core attention
-  int oproj_mode = 0;       // O projection on few tiles: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs
+  int oproj_mode = 0;       // O projection: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs (few tiles),
+                            // 3 operands swapped (weights as M, stacked token halves as N)
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
   bool moe_pair = true;     // grouped GEMMs at BN = 64: two weight tiles per work item
@@ -520,6 +522,15 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   if (h->oproj_mode == 2 && tiles * 3 <= 2 * h->num_sms && kb >= 3) {
     DenseSplitKSched<3> s{T, mt, 64};
     return launch_gemm<64, 2, 1, kSplitA>(h, dim3(tiles * 3), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
+  }
+  if (h->oproj_mode == 3) {
+    // swap-AB: weight rows (output features) are M, 64-token chunks N with the (hi, lo)
+    // halves stacked into one N = 128 MMA, so each weight tile is read from shared memory
+    // once per k step
+    EpiResidualT<64> et{h->x, d, T};
+    DenseSched s{d, d / 128, 64};
+    return launch_gemm<64, 6, 1, kSplitB>(h, dim3((d / 128) * ceil_div(T, 64)), L.tm_wo128, h->tm_ao64, kb, 1, s, et,
+                                          nullptr, &h->tm_ao64_lo);
   }
   DenseSched s{T, mt, 64};
   return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
@@ -1041,6 +1052,8 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   ok &= make_tmap(&h->tm_y_lo, h->y_lo, T, d, 128);
   ok &= make_tmap(&h->tm_ao, h->ao, T, qd, 128);
   ok &= make_tmap(&h->tm_ao_lo, h->ao_lo, T, qd, 128);
+  ok &= make_tmap(&h->tm_ao64, h->ao, T, qd, 64);
+  ok &= make_tmap(&h->tm_ao64_lo, h->ao_lo, T, qd, 64);
   ok &= make_tmap(&h->tm_head, h->head, V, d, 256);
   if (h->attn_tc) ok &= make_tmap3(&h->tm_q3, h->q, hd, H, T, H / Hkv, 128 / (H / Hkv));
   for (int i = 0; i < 4; ++i) {
@@ -1052,6 +1065,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   for (auto& L : h->L) {
     ok &= make_tmap(&L.tm_wqkv, L.wqkv, qd + 2 * kvd, d, hd);
     ok &= make_tmap(&L.tm_wo, L.wo, d, qd, 64);
+    ok &= make_tmap(&L.tm_wo128, L.wo, d, qd, 128);
     if (h->router_tc) ok &= make_tmap(&L.tm_wr, L.wr, h->E, d, 32);
     ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
     ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);

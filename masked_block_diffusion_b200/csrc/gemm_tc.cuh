@@ -668,6 +668,37 @@ struct EpiSwiGLU {
   }
 };
 
+// x[token][feature] += D with the operands swapped (the attention output projection run
+// as Wo x ao^T): accumulator rows are output features a_row + r, columns the chunk's
+// tokens b_row + c. Lanes hold consecutive features, so each column's read-modify-write
+// of x is one coalesced 128-byte access per warp.
+template <int BN>
+struct EpiResidualT {
+  static constexpr int kSmemBytes = 0;
+  float* x;
+  int ldx;
+  int T;   // token rows
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    const int f = t.a_row + r;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float old[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int tok = t.b_row + c0 + i;
+        old[i] = (tok < T && r < t.m_valid) ? x[(long)tok * ldx + f] : 0.f;
+      }
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int tok = t.b_row + c0 + i;
+        if (tok < T && r < t.m_valid) x[(long)tok * ldx + f] = old[i] + v[i];
+      }
+    }
+  }
+};
+
 // Grouped down epilogue: accumulator rows are output features 128*mt + r, columns the
 // chunk's tokens; o[slot][feature] in fp32 for the combine.
 template <int BN>
