@@ -178,7 +178,11 @@ int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T);
  * graphs. Kinds: grouped gate/up GEMM; grouped down GEMM; attention (+ split merge);
  * QKV GEMM; O GEMM; routing (pre-FFN RMSNorm, router, top-k, permute, gather);
  * combine of the expert outputs (with the next RMSNorm fused into it);
- * LM head (final RMSNorm, LM-head GEMM, merge, commit; one per pass). */
+ * LM head (final RMSNorm, LM-head GEMM, merge, commit; one per pass).
+ * Bits 16..23 of kinds, if nonzero, give a layer stride S: only layers l % S == 0 are
+ * bracketed (fewer event nodes in the graph, so the timed pass runs closer to an
+ * untimed one); launches[] counts the bracketed launches only. */
+#define DLLM_TIMING_STRIDE_SHIFT 16
 #define DLLM_TIMING_GATE_UP 0
 #define DLLM_TIMING_DOWN 1
 #define DLLM_TIMING_ATTN 2

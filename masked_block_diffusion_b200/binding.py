@@ -47,6 +47,7 @@ DLLM_TIMING_ROUTE = 5
 DLLM_TIMING_NORM = 6
 DLLM_TIMING_HEAD = 7
 DLLM_TIMING_KINDS = 8
+DLLM_TIMING_STRIDE_SHIFT = 16   # bits 16..23 of the timing mask: bracket every S-th layer only
 TIMING_NAMES = ["gate_up_gemm", "down_gemm", "attention", "qkv_gemm", "o_gemm", "routing", "norm_combine",
                 "lm_head_commit"]
 
@@ -227,7 +228,8 @@ def dllm_op_lm_head_conf(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, argmax_ptr
 
 
 def dllm_set_timing(h, kinds: int):
-    """kinds: bit mask of (1 << DLLM_TIMING_*); 0 switches timing off."""
+    """kinds: bit mask of (1 << DLLM_TIMING_*), optionally | (S << DLLM_TIMING_STRIDE_SHIFT) to time
+    every S-th layer only; 0 switches timing off."""
     _check(load().dllm_set_timing(h, int(kinds)), "dllm_set_timing", h)
 
 

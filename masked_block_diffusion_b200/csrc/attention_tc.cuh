@@ -136,14 +136,22 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     tmem_ld64(lane_base + sb * G::kSCols, s);
     tc_fence_before();
     mbar_arrive(&s_empty[sb]);
-    const int key0 = ks + j * BK;
-    float mx = -INFINITY;
+    // the maximum is taken on the raw scores (scaling by a positive constant commutes
+    // with it, rounding included); keys past the row's end are masked only in the
+    // blocks that have some
+    const int nvis = row_ke - (ks + j * BK);
+    float mx_raw = -INFINITY;
+    if (nvis >= BK) {
 #pragma unroll
-    for (int c = 0; c < BK; ++c) {
-      const float v = (key0 + c < row_ke) ? s[c] * p.scale_log2 : -INFINITY;
-      s[c] = v;
-      mx = fmaxf(mx, v);
+      for (int c = 0; c < BK; ++c) mx_raw = fmaxf(mx_raw, s[c]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < BK; ++c) {
+        if (c >= nvis) s[c] = -INFINITY;
+        mx_raw = fmaxf(mx_raw, s[c]);
+      }
     }
+    const float mx = mx_raw * p.scale_log2;
     if (j == 0) {
       m_ref = mx;
     } else {
@@ -175,7 +183,8 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     float psum = 0.f;
 #pragma unroll
     for (int c = 0; c < BK; c += 2) {
-      const float p0 = ex2_approx(s[c] - m_ref), p1 = ex2_approx(s[c + 1] - m_ref);
+      const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_ref));
+      const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_ref));
       psum += p0 + p1;
       split_bf16x2(p0, p1, hi[c / 2], lo[c / 2]);
     }

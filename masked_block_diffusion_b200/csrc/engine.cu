@@ -154,11 +154,11 @@ struct dllm_handle {
   CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // canvas passes use the tensor-core attention
-  int oproj_mode = 0;       // O projection: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs (few tiles),
+  int oproj_mode = 3;       // O projection: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs (few tiles),
                             // 3 operands swapped (weights as M, stacked token halves as N)
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
-  bool moe_pair = true;     // grouped GEMMs at BN = 64: two weight tiles per work item
+  bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
@@ -191,6 +191,7 @@ struct dllm_handle {
   bool timing = false;
   std::vector<cudaEvent_t> tev;  // [kind][layer][start, stop]
   uint32_t tmask = 0;            // kinds timed (bit k = DLLM_TIMING kind k)
+  int tstride = 1;          // time layers l % tstride == 0 only
   double t_ms[DLLM_TIMING_KINDS] = {};
   long long t_n[DLLM_TIMING_KINDS] = {};
   double t_bytes[DLLM_TIMING_KINDS] = {};   // algorithmic bytes of the timed launches
@@ -198,7 +199,6 @@ struct dllm_handle {
   int32_t* n_routed = nullptr;      // [1]
   int32_t* chunk_prefix = nullptr;  // [E+1] chunk-count prefix over the routed experts
   int32_t* routed_stat = nullptr;   // [L] n_routed per layer of the last timed pass
-  int32_t* bn_sel = nullptr;        // [1] chunk width the permute kernel chose for this layer
   int last_T = 0;                   // tokens of the last timed pass
 };
 
@@ -468,6 +468,7 @@ cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, i
 // Event of (kind, layer, start|stop); recorded only when the pass is timed.
 cudaError_t tmark(dllm_handle* h, uint32_t tmask, int kind, int layer, int which) {
   if (!(tmask & (1u << kind))) return cudaSuccess;
+  if (layer % h->tstride) return cudaSuccess;
   cudaEvent_t ev = h->tev[((size_t)kind * h->c.n_layers + layer) * 2 + which];
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   cudaError_t r = cudaStreamIsCapturing(h->st, &cs);
@@ -536,60 +537,45 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
-// One grouped gate/up + down pair at chunk width BN with MPI weight tiles per work item
-// and ACC accumulator buffers (MPI * ACC * 2 BN TMEM columns <= 512). gate: the device
-// chunk-width choice this launch serves (nullptr: always works).
+// One grouped gate/up (or down) GEMM at chunk width BN with MPI weight tiles per work
+// item and ACC accumulator buffers (MPI * ACC * 2 BN TMEM columns <= 512).
 template <int BN, int MPI, int ACC>
-cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L, int bi, const int* gate) {
+cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L, int bi) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN, gate};
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
   return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e, nullptr,
                                                &h->tm_xg_lo[bi]);
 }
 
 template <int BN, int MPI, int ACC>
-cudaError_t moe_down(dllm_handle* h, const LayerW& L, int bi, const int* gate) {
+cudaError_t moe_down(dllm_handle* h, const LayerW& L, int bi) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN, gate};
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
   EpiDown<BN> e{h->obuf, d};
   return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
                                                &h->tm_h_lo[bi]);
 }
 
-// Grouped expert GEMMs of one layer. With many tokens per expert (prefill, large
-// batches) the chunk width is 128, one weight tile per item, two accumulator buffers.
-// Otherwise the permute kernel picks the width from the routing (64 for spread routing,
-// 128 for few heavily loaded experts) and both variants are launched, the unchosen one
-// doing nothing: 64 with two weight tiles per item and two buffers, or 128 with two
-// weight tiles per item and one buffer (about one item per SM then).
+// Grouped expert GEMMs of one layer. Chunk width 64 tokens while the mean tokens per
+// expert stay below 64 (canvas passes), else 128 (prefill, large batches). At width 64,
+// down takes two weight tiles per work item (its 22 m tiles leave enough items to spread
+// over the SMs) and gate/up one (with 11 m tiles, pairs would leave too few items per
+// layer to balance).
 cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t timed) {
   const int bi = moe_bn_index(N, h->E);
   cudaError_t r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-  if (bi >= 2) {
-    r = moe_gate_up<128, 1, 2>(h, L, 2, nullptr);
-  } else if (!h->moe_pair) {
-    r = moe_gate_up<64, 1, 2>(h, L, 1, nullptr);
-  } else {
-    r = moe_gate_up<64, 2, 2>(h, L, 1, h->bn_sel);
-    if (r == cudaSuccess) r = moe_gate_up<128, 2, 1>(h, L, 2, h->bn_sel);
-  }
+  r = bi >= 2 ? moe_gate_up<128, 1, 2>(h, L, 2) : moe_gate_up<64, 1, 2>(h, L, 1);
   if (r != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  if (bi >= 2) {
-    r = moe_down<128, 1, 2>(h, L, 2, nullptr);
-  } else if (!h->moe_pair) {
-    r = moe_down<64, 1, 2>(h, L, 1, nullptr);
-  } else {
-    r = moe_down<64, 2, 2>(h, L, 1, h->bn_sel);
-    if (r == cudaSuccess) r = moe_down<128, 2, 1>(h, L, 2, h->bn_sel);
-  }
+  r = bi >= 2 ? moe_down<128, 1, 2>(h, L, 2)
+              : (h->moe_pair ? moe_down<64, 2, 2>(h, L, 1) : moe_down<64, 1, 2>(h, L, 1));
   if (r != cudaSuccess) return r;
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
@@ -648,8 +634,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       h->launches++;
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
-                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)], 128,
-                (moe_bn_index(N, h->E) < 2 && h->moe_pair) ? h->bn_sel : nullptr,
+                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
                 timed ? h->routed_stat + l : nullptr));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(128), 0, h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
@@ -787,7 +772,7 @@ void accumulate_timing(dllm_handle* h, int T) {
   for (int kind = 0; kind < DLLM_TIMING_KINDS; ++kind) {
     if (!(h->tmask & (1u << kind))) continue;
     const int layers = kind == DLLM_TIMING_HEAD ? 1 : L;
-    for (int l = 0; l < layers; ++l) {
+    for (int l = 0; l < layers; l += h->tstride) {
       float ms = 0.f;
       const size_t i = ((size_t)kind * L + l) * 2;
       if (cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]) != cudaSuccess) {
@@ -1002,7 +987,6 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->n_routed, 1);
   DA(h->chunk_prefix, h->E + 1);
   DA(h->routed_stat, c.n_layers);
-  DA(h->bn_sel, 1);
 
   DA(h->slot_of, (size_t)N);
   DA(h->row_token, (size_t)N);
@@ -1343,6 +1327,8 @@ int dllm_set_timing(dllm_handle* h, int kinds) {
     for (auto& e : h->tev) CK(cudaEventCreate(&e));
   }
   h->tmask = (uint32_t)kinds & ((1u << DLLM_TIMING_KINDS) - 1);
+  const int stride = ((uint32_t)kinds >> DLLM_TIMING_STRIDE_SHIFT) & 0xFF;
+  h->tstride = stride > 0 ? stride : 1;
   h->timing = h->tmask != 0;
   drop_graphs(h);
   return DLLM_OK;

@@ -96,9 +96,6 @@ struct PersistentGroupedSched {
   int rows_per_expert;
   int m_tiles;
   int BN;
-  // when set, the launch works only if the routing chose this chunk width (*bn_sel == BN);
-  // the variant of the other width is launched beside it and does nothing
-  const int* bn_sel = nullptr;
   // shared-memory copies, per routed expert r: token offset and count (set by stage())
   const int* s_off = nullptr;
   const int* s_cnt = nullptr;
@@ -129,7 +126,6 @@ struct PersistentGroupedSched {
   DLLM_DEV int m_groups() const { return (m_tiles + MPI - 1) / MPI; }
   DLLM_DEV int n_items() const { return chunk_prefix[*n_routed] * m_groups(); }
   DLLM_DEV int count() const {
-    if (bn_sel && *bn_sel != BN) return 0;
     const int n = n_items();
     return (int)blockIdx.x < n ? (n - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   }

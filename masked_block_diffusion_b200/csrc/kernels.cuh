@@ -237,8 +237,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
                                                        int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
                                                        int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
-                                                       int bn, int bn_big, int32_t* __restrict__ bn_sel,
-                                                       int32_t* __restrict__ routed_stat) {
+                                                       int bn, int32_t* __restrict__ routed_stat) {
   pdl_begin();
   __shared__ int cnt[256];
   __shared__ int cur[256];
@@ -257,19 +256,6 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
       const int c = e < E ? cnt[e] : 0;
       c_sum += c;
       r_sum += c > 0;
-    }
-    if (bn_sel) {
-      // chunk width from the routing: bn_big once the routed experts hold more than
-      // 3/4 bn_big tokens on average (few, heavily loaded experts), else bn
-      int routed_total = r_sum;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) routed_total += __shfl_xor_sync(0xffffffffu, routed_total, o);
-      if ((long)N * 4 > (long)routed_total * 3 * bn_big) bn = bn_big;
-      if (lane == 0) *bn_sel = bn;
-    }
-    for (int q = 0; q < per; ++q) {
-      const int e = lane * per + q;
-      const int c = e < E ? cnt[e] : 0;
       ch_sum += (c + bn - 1) / bn;
     }
     int c_pre = c_sum, r_pre = r_sum, ch_pre = ch_sum;
