@@ -8,14 +8,15 @@
 // One CTA = one 128-row query tile of one KV head over one split of the key range. The
 // tile holds the GQA group's heads for 128 / group queries (row r = query r / group,
 // head r % group), so each K/V block is loaded once for all heads that read it.
-// Roles (192 threads):
+// Roles (320 threads):
 //   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys into two
 //                  three-stage rings (a K stage is refilled once the S = Q K^T that read
 //                  it completes, a V stage once its P V does);
 //   warp 1         TMEM allocation; lane 0 issues S = Q K^T into one of two TMEM S
 //                  buffers, then O += P_hi V + P_lo V for the previous block, so the next
 //                  block's S overlaps this block's softmax;
-//   warps 2..5     one query row per thread: read S from TMEM, scale and mask, running
+//   warps 2..9     two warpgroups, each on one half (32 keys) of a block, one query row
+//                  per thread in each: read S from TMEM, scale and mask, running
 //                  maximum, P = exp2(s - m_ref) as a bf16 (hi, lo) pair written back into
 //                  TMEM with tcgen05.st (the P V MMA reads its A operand from TMEM, so P
 //                  needs no shared memory), running sum; O in TMEM is rescaled only when
@@ -75,13 +76,13 @@ DLLM_DEV float ex2_approx(float x) {
   return y;
 }
 
-// True on all 128 softmax threads iff true on each (named barrier 2).
+// True on all 256 softmax threads iff true on each (named barrier 2).
 DLLM_DEV bool sm_all(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 2, 128, p;\n\t"
+      "bar.red.and.pred q, 2, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
       : "r"((uint32_t)ok)
@@ -102,7 +103,9 @@ struct AttnTcCfg {
   static constexpr int kOffK = kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
   static constexpr int kOffBar = kOffV + STAGES * kKV;
-  static constexpr int kTotal = kOffBar + 256 + 1024;
+  static constexpr int kOffRed = kOffBar + 256;          // softmax halves: maxima [2][2][128], sums [2][128]
+  static constexpr int kTotal = kOffRed + 768 * 4 + 1024;
+  static constexpr int kOSplit = ((HD / 2 + 15) / 16) * 16;   // O columns of the first softmax half
   static constexpr int kSCols = BK;
   static constexpr int kPCol = 2 * BK;
   static constexpr int kOCol = 256;
@@ -111,16 +114,27 @@ struct AttnTcCfg {
   static_assert(kTotal <= 232448, "shared memory");
 };
 
+// Warps 2..9: two warpgroups, the first on keys 0..31 of each block, the second on keys
+// 32..63; thread (warp w, lane) owns query row r = 32 (w % 4) + lane (TMEM lane r) in
+// both, so each row's exponentials are split over two warps of the same SM sub-partition
+// pair. The halves agree on the row maximum through shared memory (red[parity][half][r],
+// one 64-thread named barrier per lane quarter), so they take the same rescaling
+// decisions; each rescales and finally writes its own column range of O, and the row sum
+// is combined once at the end.
 template <int HD>
 DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
-                              uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final,
-                              volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
-                              int nblk) {
+                           uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final, float* red,
+                           volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
+                           int nblk) {
   using G = AttnTcCfg<HD>;
-  constexpr int BK = G::BK;
+  constexpr int BK = G::BK, HB = BK / 2;   // keys per half
+  static_assert(BK == 64, "two 32-key halves per block");
   const int q = warp & 3;
+  const int half = (warp - 2) >> 2;
   const int r = q * 32 + lane;
   const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+  const int o_lo = half == 0 ? 0 : G::kOSplit, o_hi = half == 0 ? G::kOSplit : HD;   // this half's O columns
+  const int pair_bar = 3 + q;   // named barrier of the two warps sharing lane quarter q
   // keys this row may see end at row_ke: the tile's end, or (causal) the row's own query
   // position + 1; rows past the last query take the last query's limit (output dropped)
   int row_ke = ke;
@@ -131,29 +145,32 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     const int sb = j & 1;
     if (!sm_all(mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
     tc_fence_after();
-    static_assert(BK == 64, "one 64-column TMEM load per block");
-    float s[BK];
-    tmem_ld64(lane_base + sb * G::kSCols, s);
+    float s[HB];
+    tmem_ld32(lane_base + sb * G::kSCols + half * HB, s);
     tc_fence_before();
     mbar_arrive(&s_empty[sb]);
     // the maximum is taken on the raw scores (scaling by a positive constant commutes
     // with it, rounding included); keys past the row's end are masked only in the
     // blocks that have some
-    const int nvis = row_ke - (ks + j * BK);
+    const int nvis = row_ke - (ks + j * BK + half * HB);
     float mx_raw = -INFINITY;
-    if (nvis >= BK) {
+    if (nvis >= HB) {
 #pragma unroll
-      for (int c = 0; c < BK; ++c) mx_raw = fmaxf(mx_raw, s[c]);
+      for (int c = 0; c < HB; ++c) mx_raw = fmaxf(mx_raw, s[c]);
     } else {
 #pragma unroll
-      for (int c = 0; c < BK; ++c) {
+      for (int c = 0; c < HB; ++c) {
         if (c >= nvis) s[c] = -INFINITY;
         mx_raw = fmaxf(mx_raw, s[c]);
       }
     }
+    float* slot = red + (j & 1) * 256;
+    slot[half * 128 + r] = mx_raw;
+    named_bar_sync(pair_bar, 64);
+    mx_raw = fmaxf(mx_raw, slot[(half ^ 1) * 128 + r]);
     const float mx = mx_raw * p.scale_log2;
     if (j == 0) {
-      m_ref = mx;
+      m_ref = mx;   // block 0 always holds a visible key of every row
     } else {
       const bool need = mx > m_ref + 8.0f;
       if (__any_sync(0xffffffffu, need)) {
@@ -162,7 +179,7 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
           tc_fence_after();
           const float f = need ? exp2f(m_ref - mx) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < HD; c += 16) {
+          for (int c = o_lo; c < o_hi; c += 16) {
             float v[16];
             tmem_ld16(lane_base + G::kOCol + c, v);
 #pragma unroll
@@ -179,10 +196,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
         }
       }
     }
-    uint32_t hi[BK / 2], lo[BK / 2];
+    uint32_t hi[HB / 2], lo[HB / 2];
     float psum = 0.f;
 #pragma unroll
-    for (int c = 0; c < BK; c += 2) {
+    for (int c = 0; c < HB; c += 2) {
       const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_ref));
       const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_ref));
       psum += p0 + p1;
@@ -192,9 +209,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     const int pb = j & 1;
     if (!sm_all(ok && mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, abort_flag))) { ok = false; break; }
     tc_fence_after();
-    const uint32_t pcol = lane_base + G::kPCol + pb * 2 * (BK / 2);
-    tmem_st32_nowait(pcol, hi);
-    tmem_st32_nowait(pcol + BK / 2, lo);
+    // P buffer pb: hi pairs of keys 0..63 in columns 0..31, lo pairs in 32..63
+    const uint32_t pcol = lane_base + G::kPCol + pb * BK + half * (HB / 2);
+    tmem_st16_nowait(pcol, hi);
+    tmem_st16_nowait(pcol + BK / 2, lo);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&p_full[pb]);
@@ -205,6 +223,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     *abort_flag = 1;
     return;
   }
+  // row sum of both halves
+  red[512 + half * 128 + r] = l;
+  named_bar_sync(pair_bar, 64);
+  l += red[512 + (half ^ 1) * 128 + r];
   tc_fence_after();
   const int i = r / p.group;
   const int h = blockIdx.y * p.group + r % p.group;
@@ -212,7 +234,7 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
   const long t = (long)b * p.tok_per_req + q0 + i;
   const float inv = 1.0f / l;
 #pragma unroll 1
-  for (int c = 0; c < HD; c += 16) {
+  for (int c = o_lo; c < o_hi; c += 16) {
     float v[16];
     tmem_ld16(lane_base + G::kOCol + c, v);
     if (!valid) continue;
@@ -233,11 +255,11 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
         po[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv, v[4 * e + 3] * inv);
     }
   }
-  if (valid && p.n_splits > 1) p.part_lse[((long)sp * p.T + t) * p.H + h] = m_ref + __log2f(l);
+  if (valid && half == 0 && p.n_splits > 1) p.part_lse[((long)sp * p.T + t) * p.H + h] = m_ref + __log2f(l);
 }
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, AttnTcParams p) {
   using G = AttnTcCfg<HD>;
@@ -290,8 +312,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_empty[i], 256);
+      mbar_init(&p_full[i], 256);
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_done, 1);
@@ -384,8 +406,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     unsigned long long t0 = global_ns();
     while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
   } else if (warp >= 2) {
-    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final, abort_flag, warp, lane, q0,
-                        b, sp, ks, ke, nblk);
+    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final,
+                     reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);
   }
   __syncwarp();
   tc_fence_before();

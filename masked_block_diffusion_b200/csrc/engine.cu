@@ -429,7 +429,7 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (r != cudaSuccess) return r;
-  r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(192), smem, h->tm_q3, L.tm_k, L.tm_v, p);
+  r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(320), smem, h->tm_q3, L.tm_k, L.tm_v, p);
   h->launches++;
   if (r != cudaSuccess) return r;
   if (splits > 1) {
