@@ -12,6 +12,7 @@
 
 #include "dllm.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -154,8 +155,7 @@ struct dllm_handle {
   CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // canvas passes use the tensor-core attention
-  int oproj_mode = 3;       // O projection: 0 one CTA per tile, 1 / 2 K split over 2 / 3 CTAs (few tiles),
-                            // 3 operands swapped (weights as M, stacked token halves as N)
+  bool oproj_swap = true;   // O projection with swapped operands (weights as M, stacked token halves as N)
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
@@ -257,6 +257,10 @@ int moe_bn_index(int N, int E) {
   const double mean = (double)N / (double)E;
   return mean <= 64.0 ? 1 : 2;
 }
+
+// Threads of a one-row-per-block kernel over d floats: one float4 column each (up to
+// 1024), so that all of a row's loads are in flight at once.
+int row_threads(int d) { return std::min(1024, (d / 4 + 31) / 32 * 32); }
 
 int attn_splits(const dllm_handle* h, int B) {
   if (h->attn_tc) {
@@ -506,35 +510,25 @@ cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T) {
   return router_gemm_ks<1>(h, L, T, mt, tiles);
 }
 
-// Attention output projection with the residual add, x += ao * Wo^T. With few tiles
-// (one canvas: 2 x 44 at d_model 2816) K is split over CTA pairs; two stages per CTA let
-// two CTAs share an SM so that every pair is resident at once.
+// Attention output projection with the residual add, x += ao * Wo^T. By default the
+// operands are swapped: weight rows (output features) are M and 64-token chunks N, with
+// the token operand's (hi, lo) halves stacked into one N = 128 MMA, so each weight tile
+// is read from shared memory once per k step. Otherwise tokens are M and the (hi, lo)
+// pair is the A operand (two MMAs per k step).
 cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int kb = c.n_heads * c.head_dim / 64;
-  EpiResidual<64> e{h->x, d};
-  const int mt = ceil_div(T, 128);
-  const int tiles = mt * (d / 64);
-  if (h->oproj_mode == 1 && tiles * 2 <= 2 * h->num_sms && kb >= 2) {
-    DenseSplitKSched<2> s{T, mt, 64};
-    return launch_gemm<64, 2, 1, kSplitA>(h, dim3(tiles * 2), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
-  }
-  if (h->oproj_mode == 2 && tiles * 3 <= 2 * h->num_sms && kb >= 3) {
-    DenseSplitKSched<3> s{T, mt, 64};
-    return launch_gemm<64, 2, 1, kSplitA>(h, dim3(tiles * 3), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
-  }
-  if (h->oproj_mode == 3) {
-    // swap-AB: weight rows (output features) are M, 64-token chunks N with the (hi, lo)
-    // halves stacked into one N = 128 MMA, so each weight tile is read from shared memory
-    // once per k step
+  if (h->oproj_swap) {
     EpiResidualT<64> et{h->x, d, T};
     DenseSched s{d, d / 128, 64};
     return launch_gemm<64, 6, 1, kSplitB>(h, dim3((d / 128) * ceil_div(T, 64)), L.tm_wo128, h->tm_ao64, kb, 1, s, et,
                                           nullptr, &h->tm_ao64_lo);
   }
+  EpiResidual<64> e{h->x, d};
+  const int mt = ceil_div(T, 128);
   DenseSched s{T, mt, 64};
-  return launch_gemm<64, 5, 1, kSplitA>(h, dim3(tiles), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
+  return launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
 // One grouped gate/up (or down) GEMM at chunk width BN with MPI weight tiles per work
@@ -592,7 +586,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
     bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
     if (l == 0) {   // later layers get this norm from the previous layer's combine
-      CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(256), 0, h->x, L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd));
+      CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.attn_norm, d, c.rms_eps, h->y,
+                  h->y_lo, h->rstd));
       h->launches++;
     }
     CK(tmark(h, timed, DLLM_TIMING_QKV, l, 0));
@@ -605,7 +600,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(o_proj(h, L, T));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 0));
-    CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(256), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, h->rstd));
+    CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo,
+                h->rstd));
     h->launches++;
     if (!h->dense) {
       if (h->router_tc) {
@@ -636,17 +632,18 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
                 h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
                 timed ? h->routed_stat + l : nullptr));
-    CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(128), 0, h->y, h->y_lo, h->row_token, N, d, h->xg, h->xg_lo));
+    CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(std::min(1024, (d / 8 + 31) / 32 * 32)), 0, h->y, h->y_lo,
+                h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
     CK(moe_gemms(h, L, N, l, timed));
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
     const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
     if (next_gain)
-      CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d,
-                  next_gain, c.rms_eps, h->y, h->y_lo));
+      CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k,
+                  d, next_gain, c.rms_eps, h->y, h->y_lo));
     else
-      CK(launch_k(h, combine_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d));
+      CK(launch_k(h, combine_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d));
     h->launches++;
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 1));
     if (record)
@@ -879,7 +876,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   // tensor-core attention for canvas passes when a query tile of 128 rows holds whole
   // GQA groups (DLLM_ATTN_LEGACY=1 keeps the warp-MMA kernel, for comparisons)
   h->attn_tc = (128 % (H / Hkv) == 0) && !getenv("DLLM_ATTN_LEGACY");
-  if (const char* m = getenv("DLLM_OPROJ_MODE")) h->oproj_mode = atoi(m);
+  if (const char* m = getenv("DLLM_OPROJ_SWAP")) h->oproj_swap = atoi(m) != 0;
   if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
   if (const char* m = getenv("DLLM_PREFILL_TC")) h->prefill_tc = atoi(m) != 0;
   if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
