@@ -379,7 +379,7 @@ __global__ void combine_kernel(float* __restrict__ x, const float* __restrict__ 
 // norm, or the final norm before the LM head): x is updated in place, then
 // v = x * rsqrt(mean(x^2) + eps) * g is written as the (hi, lo) bf16 pair. One block per
 // token; the same per-row arithmetic as combine_kernel and rmsnorm_kernel.
-__global__ void __launch_bounds__(1024) combine_norm_kernel(float* __restrict__ x, const float* __restrict__ o,
+__global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x, const float* __restrict__ o,
                                                            const int32_t* __restrict__ slot_of,
                                                            const float* __restrict__ gate, int k, int d,
                                                            const float* __restrict__ g, float eps,
