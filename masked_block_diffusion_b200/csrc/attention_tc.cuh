@@ -341,22 +341,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     bool ok = true;
     mbar_arrive_expect_tx(q_full, G::kQ);
     for (int a = 0; a < AT; ++a) tma_load_3d(sQ + a * 128 * 128, &tm_q, q_full, a * 64, g * grp, b * C + q0);
-    // K and V blocks are brought into L2 kPrefetch blocks ahead of their loads
-    constexpr int kPrefetch = 8;
-    auto prefetch_block = [&](int jb) {
-      if (jb >= nblk) return;
-      const int prow = kv_row0 + ks + jb * BK;
-      for (int a = 0; a < AT; ++a) {
-        tma_prefetch_l2_2d(&tm_k, a * 64, prow);
-        tma_prefetch_l2_2d(&tm_v, a * 64, prow);
-      }
-    };
-    for (int jb = 0; jb < kPrefetch; ++jb) prefetch_block(jb);
     for (int j = 0; j < nblk && ok; ++j) {
       const int st = j % ST;
       const uint32_t ph = ((j / ST) & 1) ^ 1;
       const int row = kv_row0 + ks + j * BK;
-      prefetch_block(j + kPrefetch);
       if (!mbar_wait(&k_empty[st], ph, abort_flag)) { ok = false; break; }
       mbar_arrive_expect_tx(&k_full[st], G::kKV);
       for (int a = 0; a < AT; ++a) tma_load_2d(sK + st * G::kKV + a * G::kKatom, &tm_k, &k_full[st], a * 64, row, pol);

@@ -176,13 +176,6 @@ DLLM_DEV void tma_prefetch_desc(const CUtensorMap* map) {
 
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 // x is the inner (contiguous) coordinate in elements, y the row.
-// Brings one box of a 2-D tensor map into L2 (no shared memory, no barrier); boxes
-// outside the tensor are ignored.
-DLLM_DEV void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x), "r"(y)
-               : "memory");
-}
-
 DLLM_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                           uint64_t cache_hint) {
   asm volatile(

@@ -161,7 +161,6 @@ struct dllm_handle {
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
-  int l2_prefetch = 16;     // GEMMs prefetch their weight tiles into L2 this many k blocks ahead
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
   int32_t* d_P = nullptr;    // [max_batch]
@@ -332,14 +331,13 @@ cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const 
     cfg.attrs = at;
     cfg.numAttrs = h->pdl ? 2 : 1;
     if (grid.x % Sched::kKSplit || kblocks < Sched::kKSplit) return cudaErrorInvalidValue;
-    r = cudaLaunchKernelEx(&cfg, kern, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, h->l2_prefetch, s,
-                           e, h->d_err);
+    r = cudaLaunchKernelEx(&cfg, kern, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e, h->d_err);
     h->launches++;
     if (r != cudaSuccess) return r;
     return cudaGetLastError();
   }
-  r = launch_k(h, kern, grid, dim3(192), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first,
-               h->l2_prefetch, s, e, h->d_err);
+  r = launch_k(h, kern, grid, dim3(192), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e,
+               h->d_err);
   h->launches++;
   if (r != cudaSuccess) return r;
   return cudaGetLastError();
@@ -884,7 +882,6 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
   h->router_tc = !h->dense && h->E % 32 == 0;
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_L2_PREFETCH")) h->l2_prefetch = atoi(m) < 0 ? 0 : atoi(m);
   if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 

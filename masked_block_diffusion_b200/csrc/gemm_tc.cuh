@@ -264,7 +264,7 @@ template <int BN, int STAGES, int ACC_BUFS, int SPLIT, class Sched, class Epi>
 __global__ void __launch_bounds__(192, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a2,
                const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_b2,
-               int k_blocks, int a_stream_first, int prefetch, Sched sched_in, Epi epi, int* err) {
+               int k_blocks, int a_stream_first, Sched sched_in, Epi epi, int* err) {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   using L = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>;
   constexpr int kAccN = SPLIT == kSplitB ? 2 * BN : BN;   // kSplitB: columns [0, BN) hi, [BN, 2 BN) lo
@@ -346,29 +346,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     uint32_t phase = 0;
     int issued = 0;
     bool ok = true;
-    // L2 prefetch of the streamed operand (the weights), `prefetch` k blocks ahead of the
-    // loads and across work items, so that the TMA loads find their tiles in L2 instead
-    // of waiting for HBM with only the shared-memory stages in flight
-    int pj = 0, pkb = kb_begin;
-    Tile pt = ntiles > 0 ? sched.tile(0) : Tile{};
-    auto prefetch_next = [&]() {
-      if (pj >= ntiles) return;
-      if (a_stream_first) {
-        for (int u = 0; u < pt.m_count; ++u) tma_prefetch_l2_2d(&tma_a, pkb * 64, pt.a_row + u * 128);
-      } else {
-        tma_prefetch_l2_2d(&tma_b, pkb * 64, pt.b_row);
-      }
-      if (++pkb == kb_end) {
-        pkb = kb_begin;
-        if (++pj < ntiles) pt = sched.tile(pj);
-      }
-    };
-    for (int i = 0; i < prefetch; ++i) prefetch_next();
     for (int j = 0; j < ntiles && ok; ++j) {
       const Tile t = sched.tile(j);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-        if (prefetch > 0) prefetch_next();
         mbar_arrive_expect_tx(&full[stage], L::kStageBytes - (MPI - t.m_count) * L::kAtile);
         for (int u = 0; u < t.m_count; ++u)
           tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
