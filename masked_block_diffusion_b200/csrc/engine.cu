@@ -160,6 +160,8 @@ struct dllm_handle {
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
+  int router_ks = 8;        // largest K split of the router GEMM
+  bool fuse_topk = true;    // canvas passes: top-k inside the permute kernel
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
@@ -504,9 +506,10 @@ cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T) {
   const int mt = ceil_div(T, 128);
   const int tiles = mt * (h->E / 32);
   const int kb = h->c.d_model / 64;
-  if (tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
-  if (tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
-  if (tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
+  const int cap = h->router_ks;   // largest split allowed (1, 2, 4 or 8)
+  if (cap >= 8 && tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
+  if (cap >= 4 && tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
+  if (cap >= 2 && tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
   return router_gemm_ks<1>(h, L, T, mt, tiles);
 }
 
@@ -603,6 +606,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo,
                 h->rstd));
     h->launches++;
+    bool fuse_topk = false;
     if (!h->dense) {
       if (h->router_tc) {
         CK(router_gemm(h, L, T));
@@ -611,9 +615,14 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                     kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits));
         h->launches++;
       }
-      CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
-                  h->tk_idx, h->tk_w));
-      h->launches++;
+      // with few tokens the permute kernel takes the top-k itself (one launch less); the
+      // debug paths that read or replace the top-k before the permute keep it separate
+      fuse_topk = !record && !(h->force_routing && T == h->force_T) && T <= 512 && h->fuse_topk;
+      if (!fuse_topk) {
+        CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
+                    h->tk_idx, h->tk_w));
+        h->launches++;
+      }
       if (record) {
         CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
                            sizeof(float) * T * h->E, cudaMemcpyDeviceToDevice, h->st));
@@ -631,7 +640,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
                 h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
-                timed ? h->routed_stat + l : nullptr));
+                timed ? h->routed_stat + l : nullptr, fuse_topk ? h->rlogits : nullptr, h->tk_w));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(std::min(1024, (d / 8 + 31) / 32 * 32)), 0, h->y, h->y_lo,
                 h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
@@ -883,6 +892,8 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   h->router_tc = !h->dense && h->E % 32 == 0;
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
+  if (const char* m = getenv("DLLM_ROUTER_KS")) h->router_ks = atoi(m);
+  if (const char* m = getenv("DLLM_FUSE_TOPK")) h->fuse_topk = atoi(m) != 0;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
   // ---- weights

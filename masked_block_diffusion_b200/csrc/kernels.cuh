@@ -152,14 +152,9 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ x
     }
 }
 
-// Top-k experts per token by logit (ties to the lower expert) and gates = softmax of
-// the k selected logits. One warp per token; E <= 256, k <= 32.
-__global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
-                            float* __restrict__ gate) {
-  pdl_begin();
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+// Top-k of token t's E logits (ties to the lower expert) and the softmax of the k
+// selected logits as gates, by one warp (E <= 256, k <= 32).
+DLLM_DEV void topk_token(const float* logits, int t, int E, int k, int32_t* idx, float* gate, int lane) {
   float v[8];
   bool taken[8];
 #pragma unroll
@@ -198,6 +193,15 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
   }
 }
 
+__global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
+                            float* __restrict__ gate) {
+  pdl_begin();
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  topk_token(logits, t, E, k, idx, gate, lane);
+}
+
 // Debug: replace the top-k experts with given ones (the oracle's), gates recomputed
 // from this pass's own logits at those experts. One thread per token.
 __global__ void force_route_kernel(const float* __restrict__ logits, const int32_t* __restrict__ forced, int T,
@@ -233,15 +237,21 @@ __global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
 // Also lists the experts with at least one assignment (routed[0..n_routed), ascending)
 // with the prefix sums of their chunk counts ceil(count / bn) for the persistent grouped
 // GEMMs, and stores n_routed in *routed_stat when given. E <= 256.
-__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int N, int k, int E,
+__global__ void __launch_bounds__(1024) permute_kernel(int32_t* idx, int N, int k, int E,
                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
                                                        int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
                                                        int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
-                                                       int bn, int32_t* __restrict__ routed_stat) {
+                                                       int bn, int32_t* __restrict__ routed_stat,
+                                                       const float* __restrict__ logits, float* __restrict__ gate) {
   pdl_begin();
   __shared__ int cnt[256];
   __shared__ int cur[256];
   const int tid = threadIdx.x, lane = tid & 31;
+  if (logits) {
+    // top-k of every token first (a warp per token), when the pass has few tokens
+    for (int t = tid >> 5; t < N / k; t += blockDim.x >> 5) topk_token(logits, t, E, k, idx, gate, lane);
+    __syncthreads();
+  }
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int i = tid; i < N; i += blockDim.x) atomicAdd(&cnt[idx[i]], 1);
