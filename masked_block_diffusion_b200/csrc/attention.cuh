@@ -18,6 +18,11 @@
 
 namespace dllm {
 
+// Keys of one split of a request's key range [0, kend): whole 64-key blocks, about
+// kend / n_splits of them, so the splits stay balanced whatever the prefix length (the
+// last split may be shorter, or empty when kend is small).
+DLLM_DEV int split_len(int kend, int n_splits) { return ((kend + n_splits - 1) / n_splits + 63) / 64 * 64; }
+
 struct AttnParams {
   const bf16_t* q;          // [T][H][HD]
   const bf16_t* kc;         // layer cache [slots][Hkv][max_ctx][HD]
@@ -32,7 +37,7 @@ struct AttnParams {
   int T;                    // total query rows
   int H, Hkv, max_ctx;
   int causal;
-  int n_splits, split_keys;
+  int n_splits;
   float scale_log2;         // log2(e) / sqrt(HD)
 };
 
@@ -69,8 +74,9 @@ __global__ void __launch_bounds__(128, 3) attn_kernel(AttnParams p) {
   const int kvh = (h * p.Hkv) / p.H;
   const int P0 = p.pos0[b];
   const int kend = p.causal ? P0 + min(q_start + 64, nq) : P0 + nq;
-  const int ks = sp * p.split_keys;
-  const int ke = min(kend, ks + p.split_keys);
+  const int sk = split_len(kend, p.n_splits);
+  const int ks = sp * sk;
+  const int ke = min(kend, ks + sk);
   if (ks >= ke) return;
   const int nblk = (ke - ks + BK - 1) / BK;
 
@@ -266,7 +272,8 @@ __global__ void attn_merge_kernel(AttnParams p) {
   const int t = w / p.H, h = w % p.H;
   const int b = t / p.tok_per_req;
   const int kend = p.pos0[b] + p.tok_per_req;
-  const int ns = min(p.n_splits, (kend + p.split_keys - 1) / p.split_keys);
+  const int sk = split_len(kend, p.n_splits);
+  const int ns = min(p.n_splits, (kend + sk - 1) / sk);
   float mx = -INFINITY;
   for (int s = 0; s < ns; ++s) mx = fmaxf(mx, p.part_lse[((long)s * p.T + t) * p.H + h]);
   float wsum = 0.f;

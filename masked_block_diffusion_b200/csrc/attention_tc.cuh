@@ -41,7 +41,7 @@ struct AttnTcParams {
   int tok_per_req;          // canvas positions C
   int T;                    // total query rows
   int H, Hkv, group, max_ctx;
-  int n_splits, split_keys;
+  int n_splits;
   int causal;               // 1: query i of request b sees keys 0 .. P_b + i (prompt prefill)
   float scale_log2;         // log2(e) / sqrt(HD)
   int* err;
@@ -295,8 +295,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int qpt = 128 / grp;
   const int q0 = qt * qpt;
   const int kend = p.pos0[b] + (p.causal ? min(C, q0 + qpt) : C);
-  const int ks = sp * p.split_keys;
-  const int ke = min(kend, ks + p.split_keys);
+  const int sk = split_len(kend, p.n_splits);
+  const int ks = sp * sk;
+  const int ke = min(kend, ks + sk);
   if (q0 >= C || ks >= ke) return;   // uniform over the CTA, before any barrier or TMEM use
   const int nblk = (ke - ks + BK - 1) / BK;
   const int kv_row0 = (p.slot[b] * p.Hkv + g) * p.max_ctx;

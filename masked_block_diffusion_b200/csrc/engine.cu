@@ -161,7 +161,6 @@ struct dllm_handle {
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   int router_ks = 8;        // largest K split of the router GEMM
-  bool fuse_topk = true;    // canvas passes: top-k inside the permute kernel
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
@@ -280,10 +279,6 @@ int attn_splits(const dllm_handle* h, int B) {
   return s;
 }
 
-int attn_split_keys(const dllm_handle* h, int splits) {
-  return ceil_div(ceil_div(h->c.max_ctx, splits), 64) * 64;
-}
-
 // ------------------------------------------------------------------ launch helpers
 
 // Launches kern on the handle's stream; with h->pdl the launch carries programmatic
@@ -371,7 +366,7 @@ cudaError_t qkv_gemm(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, in
 
 template <int HD, int BK>
 cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
-                         const int* slot, int causal, int splits, int split_keys) {
+                         const int* slot, int causal, int splits) {
   const auto& c = h->c;
   AttnParams p;
   p.q = h->q;
@@ -390,7 +385,6 @@ cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq
   p.max_ctx = c.max_ctx;
   p.causal = causal;
   p.n_splits = splits;
-  p.split_keys = split_keys;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   constexpr int smem = AttnSmem<HD, BK>::kTotal;
   cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_kernel<HD, BK>),
@@ -410,7 +404,7 @@ cudaError_t attention_hd(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq
 
 template <int HD>
 cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, int tok_per_req, const int* pos0,
-                            const int* slot, int causal, int splits, int split_keys) {
+                            const int* slot, int causal, int splits) {
   const auto& c = h->c;
   AttnTcParams p;
   p.out = h->ao;
@@ -427,7 +421,6 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   p.group = c.n_heads / c.n_kv_heads;
   p.max_ctx = c.max_ctx;
   p.n_splits = splits;
-  p.split_keys = split_keys;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.err = h->d_err;
   dim3 grid(ceil_div((long)tok_per_req * p.group, 128), c.n_kv_heads, nreq * splits);
@@ -449,7 +442,6 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
     m.T = T;
     m.H = c.n_heads;
     m.n_splits = splits;
-    m.split_keys = split_keys;
     r = launch_k(h, attn_merge_kernel<HD>, dim3(ceil_div((long)T * c.n_heads * 32, 256)), dim3(256), 0, m);
     h->launches++;
     if (r != cudaSuccess) return r;
@@ -458,17 +450,17 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
 }
 
 cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, int tok_per_req, const int* pos0,
-                      const int* slot, int causal, int splits, int split_keys, const LayerW* L = nullptr) {
+                      const int* slot, int causal, int splits, const LayerW* L = nullptr) {
   // tensor cores: the bidirectional canvas pass, and (one key range per query tile) the
   // causal prompt prefill
   if (h->attn_tc && L && (!causal || (h->prefill_tc && splits == 1))) {
     if (h->c.head_dim == 176)
-      return attention_tc_hd<176>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
-    return attention_tc_hd<64>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
+      return attention_tc_hd<176>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits);
+    return attention_tc_hd<64>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits);
   }
   if (h->c.head_dim == 176)
-    return attention_hd<176, 32>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
-  return attention_hd<64, 64>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys);
+    return attention_hd<176, 32>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits);
+  return attention_hd<64, 64>(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits);
 }
 
 // Event of (kind, layer, start|stop); recorded only when the pass is timed.
@@ -580,7 +572,7 @@ cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t ti
 // ------------------------------------------------------------------ the pass
 
 int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0, const int* slot, int causal,
-               int splits, int split_keys, bool record, uint32_t timed, const float* final_gain) {
+               int splits, bool record, uint32_t timed, const float* final_gain) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int N = T * h->k;
@@ -597,7 +589,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(qkv_gemm(h, L, kc, vc, T, pos0, slot, tok_per_req));
     CK(tmark(h, timed, DLLM_TIMING_QKV, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 0));
-    CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, split_keys, &L));
+    CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, &L));
     CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 0));
     CK(o_proj(h, L, T));
@@ -606,7 +598,6 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo,
                 h->rstd));
     h->launches++;
-    bool fuse_topk = false;
     if (!h->dense) {
       if (h->router_tc) {
         CK(router_gemm(h, L, T));
@@ -615,14 +606,9 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
                     kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits));
         h->launches++;
       }
-      // with few tokens the permute kernel takes the top-k itself (one launch less); the
-      // debug paths that read or replace the top-k before the permute keep it separate
-      fuse_topk = !record && !(h->force_routing && T == h->force_T) && T <= 512 && h->fuse_topk;
-      if (!fuse_topk) {
-        CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
-                    h->tk_idx, h->tk_w));
-        h->launches++;
-      }
+      CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
+                  h->tk_idx, h->tk_w));
+      h->launches++;
       if (record) {
         CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
                            sizeof(float) * T * h->E, cudaMemcpyDeviceToDevice, h->st));
@@ -640,7 +626,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
                 h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
-                timed ? h->routed_stat + l : nullptr, fuse_topk ? h->rlogits : nullptr, h->tk_w));
+                timed ? h->routed_stat + l : nullptr));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(std::min(1024, (d / 8 + 31) / 32 * 32)), 0, h->y, h->y_lo,
                 h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
@@ -672,7 +658,7 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
               h->x));
   h->launches++;
   const uint32_t tm = (h->timing && mode == 0) ? h->tmask : 0u;
-  int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, attn_split_keys(h, splits), h->debug && mode == 0,
+  int r = run_layers(h, T, B, C, h->d_P, h->d_slot, 0, splits, h->debug && mode == 0,
                      tm, mode == 0 ? h->final_norm : nullptr);
   if (r) return r;
   if (mode == 1) return DLLM_OK;
@@ -893,7 +879,6 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_KS")) h->router_ks = atoi(m);
-  if (const char* m = getenv("DLLM_FUSE_TOPK")) h->fuse_topk = atoi(m) != 0;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
   // ---- weights
@@ -1098,7 +1083,7 @@ int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool pro
   CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
   CK(launch_k(h, embed_kernel, dim3(n), dim3(128), 0, h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x));
   h->launches++;
-  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, c.max_ctx, false, 0u, nullptr);
+  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, false, 0u, nullptr);
   if (r) return r;
   h->P[req] = n;
   return upload_P(h);

@@ -237,21 +237,15 @@ __global__ void dense_route_kernel(int T, int32_t* idx, float* gate) {
 // Also lists the experts with at least one assignment (routed[0..n_routed), ascending)
 // with the prefix sums of their chunk counts ceil(count / bn) for the persistent grouped
 // GEMMs, and stores n_routed in *routed_stat when given. E <= 256.
-__global__ void __launch_bounds__(1024) permute_kernel(int32_t* idx, int N, int k, int E,
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int N, int k, int E,
                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
                                                        int32_t* __restrict__ row_token, int32_t* __restrict__ routed,
                                                        int32_t* __restrict__ n_routed, int32_t* __restrict__ chunk_prefix,
-                                                       int bn, int32_t* __restrict__ routed_stat,
-                                                       const float* __restrict__ logits, float* __restrict__ gate) {
+                                                       int bn, int32_t* __restrict__ routed_stat) {
   pdl_begin();
   __shared__ int cnt[256];
   __shared__ int cur[256];
   const int tid = threadIdx.x, lane = tid & 31;
-  if (logits) {
-    // top-k of every token first (a warp per token), when the pass has few tokens
-    for (int t = tid >> 5; t < N / k; t += blockDim.x >> 5) topk_token(logits, t, E, k, idx, gate, lane);
-    __syncthreads();
-  }
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int i = tid; i < N; i += blockDim.x) atomicAdd(&cnt[idx[i]], 1);

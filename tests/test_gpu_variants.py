@@ -10,8 +10,7 @@ same step-by-step comparison with the oracle runs on a two-layer model:
 - DLLM_QKV_SPLITK=0 with DLLM_PDL=0: QKV without the split-K cluster, launches without
   programmatic dependent launch;
 - DLLM_PREFILL_TC=0: causal prefill on the mma.sync flash kernel;
-- DLLM_FUSE_TOPK=0 with DLLM_ROUTER_KS=2: top-k as its own kernel in the undebugged
-  passes too, router K split over 2 CTAs instead of 8.
+- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8.
 
 A GQA group of 3 (6 query heads over 2 KV heads) does not divide the 128-row query tile
 of the tensor-core attention, so that model runs both its prefill and its canvas passes
@@ -46,7 +45,7 @@ VARIANTS = {
     "simt-router": {"DLLM_ROUTER_TC": "0"},
     "qkv-no-splitk-no-pdl": {"DLLM_QKV_SPLITK": "0", "DLLM_PDL": "0"},
     "prefill-mma-sync": {"DLLM_PREFILL_TC": "0"},
-    "topk-kernel-router-ks2": {"DLLM_FUSE_TOPK": "0", "DLLM_ROUTER_KS": "2"},
+    "router-ks2": {"DLLM_ROUTER_KS": "2"},
 }
 
 
