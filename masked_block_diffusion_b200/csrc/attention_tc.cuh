@@ -43,8 +43,6 @@ struct AttnTcParams {
   int H, Hkv, group, max_ctx;
   int n_splits;
   int causal;               // 1: query i of request b sees keys 0 .. P_b + i (prompt prefill)
-  int cluster_merge;        // 1: the n_splits CTAs of a query tile form a cluster and rank 0
-                            //    merges their partials over distributed shared memory
   float scale_log2;         // log2(e) / sqrt(HD)
   int* err;
 };
@@ -114,7 +112,6 @@ struct AttnTcCfg {
   static constexpr int kTmemCols = 512;
   static_assert(kPCol + 2 * BK <= kOCol && kOCol + HD <= kTmemCols, "TMEM");
   static_assert(kTotal <= 232448, "shared memory");
-  static_assert((HD * 128 + 128) * 4 <= 2 * STAGES * kKV, "merge partial fits the K/V stages");
 };
 
 // Warps 2..9: two warpgroups, the first on keys 0..31 of each block, the second on keys
@@ -128,7 +125,7 @@ template <int HD>
 DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
                            uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final, float* red,
                            volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
-                           int nblk, int crank, float* part, uint64_t* peer_ready) {
+                           int nblk) {
   using G = AttnTcCfg<HD>;
   constexpr int BK = G::BK, HB = BK / 2;   // keys per half
   static_assert(BK == 64, "two 32-key halves per block");
@@ -236,72 +233,6 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
   const bool valid = q0 + i < p.tok_per_req;
   const long t = (long)b * p.tok_per_req + q0 + i;
   const float inv = 1.0f / l;
-  if (p.cluster_merge) {
-    // the splits of this query tile merge in the cluster: ranks > 0 leave their normalised
-    // partial O ([HD][128] fp32) and log-sum-exp in their own shared memory (the idle K/V
-    // stages) and signal rank 0, which weighs every split by 2^(lse_s - max) and writes
-    // the output; an empty split has lse = -inf and weight 0
-    float* lse_s = part + HD * 128;
-    if (crank != 0) {
-      if (nblk > 0) {
-#pragma unroll 1
-        for (int c = o_lo; c < o_hi; c += 16) {
-          float v[16];
-          tmem_ld16(lane_base + G::kOCol + c, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) part[(c + e) * 128 + r] = v[e] * inv;
-        }
-      }
-      if (half == 0) lse_s[r] = nblk > 0 ? m_ref + __log2f(l) : -INFINITY;
-      mbar_arrive_cluster(mapa_shared(smem_u32(peer_ready), 0));
-      return;
-    }
-    const bool got = mbar_wait_cluster(peer_ready, 0, abort_flag);
-    if (!sm_all(got)) {
-      if (!got) atomicExch(p.err, kDevTimeoutEpilogue);
-      *abort_flag = 1;
-      return;
-    }
-    const int S = p.n_splits;
-    float lse[8], wgt[8];
-    lse[0] = m_ref + __log2f(l);
-    float mxl = lse[0];
-    for (int s2 = 1; s2 < S; ++s2) {
-      lse[s2] = ld_shared_cluster_f32(mapa_shared(smem_u32(lse_s + r), s2));
-      mxl = fmaxf(mxl, lse[s2]);
-    }
-    float wsum = 0.f;
-    for (int s2 = 0; s2 < S; ++s2) {
-      wgt[s2] = lse[s2] == -INFINITY ? 0.f : exp2f(lse[s2] - mxl);
-      wsum += wgt[s2];
-    }
-    const float w0 = wgt[0] / wsum * inv;   // own O in TMEM is not yet divided by its sum
-#pragma unroll 1
-    for (int c = o_lo; c < o_hi; c += 16) {
-      float v[16];
-      tmem_ld16(lane_base + G::kOCol + c, v);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] *= w0;
-      for (int s2 = 1; s2 < S; ++s2) {
-        if (wgt[s2] == 0.f) continue;
-        const float ws = wgt[s2] / wsum;
-        const uint32_t base = mapa_shared(smem_u32(part + c * 128 + r), s2);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] += ws * ld_shared_cluster_f32(base + (uint32_t)(e * 128 * 4));
-      }
-      if (!valid) continue;
-      uint32_t hw[8], lw[8];
-#pragma unroll
-      for (int e = 0; e < 16; e += 2) split_bf16x2(v[e], v[e + 1], hw[e / 2], lw[e / 2]);
-      bf16_t* oh = p.out + (t * p.H + h) * HD + c;
-      bf16_t* ol = p.out_lo + (t * p.H + h) * HD + c;
-      reinterpret_cast<uint4*>(oh)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      reinterpret_cast<uint4*>(oh)[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-      reinterpret_cast<uint4*>(ol)[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      reinterpret_cast<uint4*>(ol)[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-    }
-    return;
-  }
 #pragma unroll 1
   for (int c = o_lo; c < o_hi; c += 16) {
     float v[16];
@@ -353,8 +284,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* o_done = p_empty + 2;
   uint64_t* o_final = o_done + 1;
   uint64_t* drain = o_final + 1;
-  uint64_t* peer_ready = drain + 1;   // cluster merge: rank 0 learns that the peers' partials are in place
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   pdl_wait();   // pos0 and the K / V written by the QKV projection
@@ -368,11 +298,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int sk = split_len(kend, p.n_splits);
   const int ks = sp * sk;
   const int ke = min(kend, ks + sk);
-  // uniform over the CTA, before any barrier or TMEM use; in a merging cluster an empty
-  // split still takes part (with no key blocks and weight 0)
-  if (q0 >= C || (!p.cluster_merge && ks >= ke)) return;
-  const int nblk = ke > ks ? (ke - ks + BK - 1) / BK : 0;
-  const int crank = p.cluster_merge ? (int)cluster_ctarank() : 0;
+  if (q0 >= C || ks >= ke) return;   // uniform over the CTA, before any barrier or TMEM use
+  const int nblk = (ke - ks + BK - 1) / BK;
   const int kv_row0 = (p.slot[b] * p.Hkv + g) * p.max_ctx;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -393,7 +320,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
-    if (p.cluster_merge && crank == 0) mbar_init(peer_ready, 256 * (p.n_splits - 1));
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -407,7 +333,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (p.cluster_merge) cluster_sync();   // rank 0's barrier is initialised before any peer arrives
   pdl_trigger();   // after the TMEM allocation
   const uint32_t tmem_base = *tmem_slot;
 
@@ -472,7 +397,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       umma_commit(&k_empty[st]);
       if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
     }
-    if (ok && nblk > 0 && !issue_pv(nblk - 1)) ok = false;
+    if (ok && !issue_pv(nblk - 1)) ok = false;
     if (ok) umma_commit(o_final);
     if (!ok) {
       atomicExch(p.err, kDevTimeoutMma);
@@ -483,14 +408,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
   } else if (warp >= 2) {
     softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final,
-                     reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk,
-                     crank, reinterpret_cast<float*>(smem + G::kOffK), peer_ready);
+                     reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);
   }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (p.cluster_merge) cluster_sync();   // no CTA leaves while rank 0 may still read its partials
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, G::kTmemCols);

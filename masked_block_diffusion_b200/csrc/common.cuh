@@ -159,12 +159,6 @@ DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* ab
   }
 }
 
-DLLM_DEV float ld_shared_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
-
 DLLM_DEV float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"

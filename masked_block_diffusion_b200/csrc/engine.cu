@@ -158,7 +158,6 @@ struct dllm_handle {
   bool oproj_swap = true;   // O projection with swapped operands (weights as M, stacked token halves as N)
   bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
   bool prefill_tc = true;   // causal prefill attention on the tensor cores too
-  bool attn_cluster_merge = true;   // attention splits merge inside a cluster
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   int router_ks = 8;        // largest K split of the router GEMM
@@ -424,34 +423,11 @@ cudaError_t attention_tc_hd(dllm_handle* h, const LayerW& L, int T, int nreq, in
   p.n_splits = splits;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.err = h->d_err;
-  // the splits of one query tile as a cluster that merges in distributed shared memory
-  // (no partials in HBM, no merge kernel), up to the portable cluster size
-  p.cluster_merge = (splits > 1 && splits <= 8 && h->attn_cluster_merge) ? 1 : 0;
   dim3 grid(ceil_div((long)tok_per_req * p.group, 128), c.n_kv_heads, nreq * splits);
   constexpr int smem = AttnTcCfg<HD>::kTotal;
   cudaError_t r = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<HD>),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (r != cudaSuccess) return r;
-  if (p.cluster_merge) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(320);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = h->st;
-    cudaLaunchAttribute at[2];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 1;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = splits;
-    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = h->pdl ? 2 : 1;
-    r = cudaLaunchKernelEx(&cfg, attn_tc_kernel<HD>, h->tm_q3, L.tm_k, L.tm_v, p);
-    h->launches++;
-    if (r != cudaSuccess) return r;
-    return cudaGetLastError();
-  }
   r = launch_k(h, attn_tc_kernel<HD>, grid, dim3(320), smem, h->tm_q3, L.tm_k, L.tm_v, p);
   h->launches++;
   if (r != cudaSuccess) return r;
@@ -898,7 +874,6 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   if (const char* m = getenv("DLLM_OPROJ_SWAP")) h->oproj_swap = atoi(m) != 0;
   if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
   if (const char* m = getenv("DLLM_PREFILL_TC")) h->prefill_tc = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_ATTN_CLUSTER_MERGE")) h->attn_cluster_merge = atoi(m) != 0;
   if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
   h->router_tc = !h->dense && h->E % 32 == 0;
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;

@@ -10,9 +10,7 @@ same step-by-step comparison with the oracle runs on a two-layer model:
 - DLLM_QKV_SPLITK=0 with DLLM_PDL=0: QKV without the split-K cluster, launches without
   programmatic dependent launch;
 - DLLM_PREFILL_TC=0: causal prefill on the mma.sync flash kernel;
-- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8;
-- DLLM_ATTN_CLUSTER_MERGE=0: attention splits write partials to HBM and a merge kernel
-  combines them, instead of merging inside the cluster.
+- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8.
 
 A GQA group of 3 (6 query heads over 2 KV heads) does not divide the 128-row query tile
 of the tensor-core attention, so that model runs both its prefill and its canvas passes
@@ -48,7 +46,6 @@ VARIANTS = {
     "qkv-no-splitk-no-pdl": {"DLLM_QKV_SPLITK": "0", "DLLM_PDL": "0"},
     "prefill-mma-sync": {"DLLM_PREFILL_TC": "0"},
     "router-ks2": {"DLLM_ROUTER_KS": "2"},
-    "attention-merge-kernel": {"DLLM_ATTN_CLUSTER_MERGE": "0"},
 }
 
 
