@@ -12,9 +12,9 @@
 //   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys into two
 //                  three-stage rings (a K stage is refilled once the S = Q K^T that read
 //                  it completes, a V stage once its P V does);
-//   warp 1         TMEM allocation; lane 0 issues S = Q K^T into one of two TMEM S
-//                  buffers, then O += P_hi V + P_lo V for the previous block, so the next
-//                  block's S overlaps this block's softmax;
+//   warp 1         TMEM allocation; lane 0 issues S = Q K^T into one of three TMEM S
+//                  buffers two blocks ahead of O += P_hi V + P_lo V, so the scores of the
+//                  next blocks are ready while the softmax works on the current one;
 //   warps 2..9     two warpgroups, each on one half (32 keys) of a block, one query row
 //                  per thread in each: read S from TMEM, scale and mask, running
 //                  maximum, P = exp2(s - m_ref) as a bf16 (hi, lo) pair written back into
@@ -90,8 +90,8 @@ DLLM_DEV bool sm_all(bool ok) {
   return r != 0;
 }
 
-// TMEM columns: S buffers 0..63 and 64..127; P buffer pb at 128 + 64 pb (hi in the first
-// 32 columns, lo in the next 32, two bf16 per column); O from column 256.
+// TMEM columns: S buffers at 0, 64 and 128; P buffer pb at 192 + 64 pb (hi in the first 32
+// columns, lo in the next 32, two bf16 per column); O from column 320.
 template <int HD>
 struct AttnTcCfg {
   static constexpr int BK = 64;
@@ -106,9 +106,10 @@ struct AttnTcCfg {
   static constexpr int kOffRed = kOffBar + 256;          // softmax halves: maxima [2][2][128], sums [2][128]
   static constexpr int kTotal = kOffRed + 768 * 4 + 1024;
   static constexpr int kOSplit = ((HD / 2 + 15) / 16) * 16;   // O columns of the first softmax half
+  static constexpr int kSBufs = 3;                       // S buffers: S(j+2) is issued before P V(j)
   static constexpr int kSCols = BK;
-  static constexpr int kPCol = 2 * BK;
-  static constexpr int kOCol = 256;
+  static constexpr int kPCol = kSBufs * BK;
+  static constexpr int kOCol = kPCol + 2 * BK;
   static constexpr int kTmemCols = 512;
   static_assert(kPCol + 2 * BK <= kOCol && kOCol + HD <= kTmemCols, "TMEM");
   static_assert(kTotal <= 232448, "shared memory");
@@ -123,7 +124,7 @@ struct AttnTcCfg {
 // is combined once at the end.
 template <int HD>
 DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
-                           uint64_t* p_full, uint64_t* p_empty, uint64_t* o_done, uint64_t* o_final, float* red,
+                           uint64_t* p_full, uint64_t* p_empty, uint64_t* o_final, float* red,
                            volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
                            int nblk) {
   using G = AttnTcCfg<HD>;
@@ -142,8 +143,8 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
   for (int j = 0; j < nblk; ++j) {
-    const int sb = j & 1;
-    if (!sm_all(mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+    const int sb = j % G::kSBufs;
+    if (!sm_all(mbar_wait(&s_full[sb], (j / G::kSBufs) & 1, abort_flag))) { ok = false; break; }
     tc_fence_after();
     float s[HB];
     tmem_ld32(lane_base + sb * G::kSCols + half * HB, s);
@@ -174,7 +175,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     } else {
       const bool need = mx > m_ref + 8.0f;
       if (__any_sync(0xffffffffu, need)) {
-        const bool got = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, abort_flag));
+        // O is rescaled once P V(j-1) has landed: its completion is the commit on P buffer
+        // (j-1)&1 (with S issued ahead of P V, S(j) being ready no longer implies it)
+        const bool got =
+            __all_sync(0xffffffffu, mbar_wait(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag));
         if (got) {
           tc_fence_after();
           const float f = need ? exp2f(m_ref - mx) : 1.0f;
@@ -278,11 +282,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* v_full = k_empty + ST;
   uint64_t* v_empty = v_full + ST;
   uint64_t* s_full = v_empty + ST;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
+  uint64_t* s_empty = s_full + G::kSBufs;
+  uint64_t* p_full = s_empty + G::kSBufs;
   uint64_t* p_empty = p_full + 2;
-  uint64_t* o_done = p_empty + 2;
-  uint64_t* o_final = o_done + 1;
+  uint64_t* o_final = p_empty + 2;
   uint64_t* drain = o_final + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -311,13 +314,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < G::kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 256);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], 256);
       mbar_init(&p_empty[i], 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -377,13 +381,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       umma_commit(&p_empty[pb]);
       umma_commit(&v_empty[st]);
-      umma_commit(o_done);
       return true;
     };
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int st = j % ST, sb = j & 1;
-      if (!mbar_wait(&k_full[st], (j / ST) & 1, abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+    // S = Q K^T for block jj into S buffer jj % kSBufs
+    auto issue_s = [&](int jj) -> bool {
+      const int st = jj % ST, sb = jj % G::kSBufs;
+      if (!mbar_wait(&k_full[st], (jj / ST) & 1, abort_flag)) return false;
+      if (!mbar_wait(&s_empty[sb], ((jj / G::kSBufs) & 1) ^ 1, abort_flag)) return false;
       tc_fence_after();
       const uint32_t d_s = tmem_base + sb * G::kSCols;
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK + st * G::kKV);
@@ -395,9 +399,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     sdesc_k_sw128(k_base + a * G::kKatom + kk * 32), kIdQK, (a | kk) != 0);
       umma_commit(&s_full[sb]);
       umma_commit(&k_empty[st]);
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      return true;
+    };
+    // S runs kSBufs - 1 blocks ahead of P V, so the tensor pipe always has the next
+    // scores queued while the softmax warps work on the current block
+    constexpr int kAhead = G::kSBufs - 1;
+    for (int j = 0; j < kAhead && j < nblk && ok; ++j) ok = issue_s(j);
+    for (int j = 0; j < nblk && ok; ++j) {
+      if (j + kAhead < nblk && !issue_s(j + kAhead)) { ok = false; break; }
+      if (!issue_pv(j)) { ok = false; break; }
     }
-    if (ok && !issue_pv(nblk - 1)) ok = false;
     if (ok) umma_commit(o_final);
     if (!ok) {
       atomicExch(p.err, kDevTimeoutMma);
@@ -407,7 +418,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     unsigned long long t0 = global_ns();
     while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
   } else if (warp >= 2) {
-    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_done, o_final,
+    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_final,
                      reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);
   }
   __syncwarp();
