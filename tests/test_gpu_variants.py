@@ -10,7 +10,9 @@ same step-by-step comparison with the oracle runs on a two-layer model:
 - DLLM_QKV_SPLITK=0 with DLLM_PDL=0: QKV without the split-K cluster, launches without
   programmatic dependent launch;
 - DLLM_PREFILL_TC=0: causal prefill on the mma.sync flash kernel;
-- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8.
+- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8;
+- DLLM_ATTN_LEGACY=1: canvas attention on the mma.sync flash kernel too;
+- DLLM_NO_GRAPH=1: every pass launched eagerly instead of replaying its CUDA graph.
 
 A GQA group of 3 (6 query heads over 2 KV heads) does not divide the 128-row query tile
 of the tensor-core attention, so that model runs both its prefill and its canvas passes
@@ -46,6 +48,8 @@ VARIANTS = {
     "qkv-no-splitk-no-pdl": {"DLLM_QKV_SPLITK": "0", "DLLM_PDL": "0"},
     "prefill-mma-sync": {"DLLM_PREFILL_TC": "0"},
     "router-ks2": {"DLLM_ROUTER_KS": "2"},
+    "attention-mma-sync": {"DLLM_ATTN_LEGACY": "1"},
+    "no-graph": {"DLLM_NO_GRAPH": "1"},
 }
 
 
@@ -69,3 +73,36 @@ def test_gqa_group_of_three_on_mma_sync_attention():
     assert steps <= 8
     assert stats["route_pinned"] > 0.9 * stats["route_total"]
     assert stats["arg_pinned"] > 0.9 * stats["arg_total"]
+
+
+_FAULT_SCRIPT = """
+import sys
+sys.path.insert(0, {root!r})
+from masked_block_diffusion_b200 import binding
+from synth import WORKLOADS, blob_from_weights, gen_weights
+cfg = WORKLOADS["c1-tiny-dense"].model
+blob = blob_from_weights(cfg, gen_weights(cfg))
+c = binding.make_config(cfg, max_ctx=256, max_batch=1)
+try:
+    h = binding.dllm_create(c, blob.ctypes.data, blob.nbytes, False, 0)
+    print("CODE", 0)
+    binding.dllm_destroy(h)
+except binding.DllmError as e:
+    print("CODE", e.code)
+"""
+
+
+def test_allocation_failure_is_reported_cleanly():
+    """The n-th device allocation fails on the host (DLLM_FAULT_ALLOC_AT): dllm_create
+    returns DLLM_E_OOM with no handle, after releasing what it had allocated."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for n in (1, 5, 20):
+        env = dict(os.environ, DLLM_FAULT_ALLOC_AT=str(n))
+        out = subprocess.run([sys.executable, "-c", _FAULT_SCRIPT.format(root=root)], env=env,
+                             capture_output=True, text=True, timeout=300)
+        assert out.returncode == 0, out.stderr[-2000:]
+        line = [x for x in out.stdout.splitlines() if x.startswith("CODE")][-1]
+        assert line == "CODE -2", line
