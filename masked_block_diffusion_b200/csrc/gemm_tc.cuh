@@ -161,8 +161,10 @@ __host__ __device__ constexpr int tmem_cols_for(int bn) {
 
 // Operand splitting. Weights are bf16; an activation operand can be carried as a pair
 // of bf16 tensors (hi = bf16(v), lo = bf16(v - hi)) so that products keep about 16
-// mantissa bits of the activation: every k step then issues two MMAs into the same
-// accumulator. kSplitNone: plain; kSplitA: A is a (hi, lo) pair; kSplitB: B is.
+// mantissa bits of the activation. kSplitNone: plain. kSplitA: A is a (hi, lo) pair and
+// every k step issues two MMAs into the same accumulator. kSplitB: B is the pair; its
+// hi and lo rows sit next to each other in the stage, one MMA of width 2 BN reads both,
+// and the epilogue first adds the accumulator's two column halves.
 enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
 
 template <int BN, int STAGES, int SPLIT, class Epi, class Sched = DenseSched>
