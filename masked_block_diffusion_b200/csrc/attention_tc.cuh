@@ -76,16 +76,18 @@ DLLM_DEV float ex2_approx(float x) {
   return y;
 }
 
-// True on all 256 softmax threads iff true on each (named barrier 2).
-DLLM_DEV bool sm_all(bool ok) {
+// True on both warps of a lane-quarter pair (the two softmax halves of the same rows)
+// iff true on each of their 64 threads (named barrier `id`). The pairs agree on leaving
+// the loop together without holding the other pairs back.
+DLLM_DEV bool pair_all(bool ok, int id) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 2, 256, p;\n\t"
+      "bar.red.and.pred q, %2, 64, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "r"(id)
       : "memory");
   return r != 0;
 }
@@ -144,7 +146,7 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
   bool ok = true;
   for (int j = 0; j < nblk; ++j) {
     const int sb = j % G::kSBufs;
-    if (!sm_all(mbar_wait(&s_full[sb], (j / G::kSBufs) & 1, abort_flag))) { ok = false; break; }
+    if (!pair_all(mbar_wait(&s_full[sb], (j / G::kSBufs) & 1, abort_flag), pair_bar)) { ok = false; break; }
     tc_fence_after();
     float s[HB];
     tmem_ld32(lane_base + sb * G::kSCols + half * HB, s);
@@ -211,7 +213,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     }
     l += psum;
     const int pb = j & 1;
-    if (!sm_all(ok && mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, abort_flag))) { ok = false; break; }
+    if (!pair_all(ok && mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, abort_flag), pair_bar)) {
+      ok = false;
+      break;
+    }
     tc_fence_after();
     // P buffer pb: hi pairs of keys 0..63 in columns 0..31, lo pairs in 32..63
     const uint32_t pcol = lane_base + G::kPCol + pb * BK + half * (HB / 2);
@@ -221,7 +226,7 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     tc_fence_before();
     mbar_arrive(&p_full[pb]);
   }
-  if (ok) ok = sm_all(mbar_wait(o_final, 0, abort_flag));
+  if (ok) ok = pair_all(mbar_wait(o_final, 0, abort_flag), pair_bar);
   if (!ok) {
     atomicExch(p.err, kDevTimeoutEpilogue);
     *abort_flag = 1;
