@@ -27,6 +27,17 @@ def test_header_and_binding_agree():
     assert declared_symbols() == sorted(binding.EXPORTS)
 
 
+def test_binding_constants_match_header_defines():
+    """Every integer #define of the header that the binding also names has the same value."""
+    text = open(os.path.join(ROOT, "include", "dllm.h")).read()
+    defines = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+(DLLM_\w+)\s+\(?(-?\d+)\)?", text)}
+    shared = [n for n in defines if hasattr(binding, n)]
+    assert len(shared) >= 10, shared
+    for n in shared:
+        assert getattr(binding, n) == defines[n], n
+    assert "DLLM_TIMING_STRIDE_SHIFT" in shared and "DLLM_E_OOM" in shared
+
+
 def test_library_exports_every_declared_symbol(lib_path):
     out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True, check=True).stdout
     exported = set(re.findall(r"\b(dllm_\w+)\b", out))
