@@ -43,20 +43,29 @@ Readings where the pages are silent (all listed in the design notes):
    position; threshold: every masked position with conf > tau, and at least
    n_min = max(1, ceil(R / (S_max - s))) of the most confident ones so that the
    canvas completes within the step budget;
-10. precision: the weights are bf16 values and the KV cache holds bf16 values, so
-   Q, K and V after RoPE are rounded to bf16 (Q too: it is formed once and read only
-   by attention); every other quantity (normalised activations, attention output,
-   SwiGLU output, residual stream, router, softmax statistics) is computed in fp64;
-   router and LM-head logits are rounded to fp32 before the top-k / argmax decision,
-   and conf to fp32 before commit ranking.
+10. precision: the task fixes bf16 operands with fp32 accumulation. The oracle
+   applies that rounding to the operands the model hands from one operation to the
+   next as data: the weights (the tiny model's fp32 weights enter every product as
+   their bf16 roundings) and the attention operands Q, K and V, rounded after RoPE (K
+   and V also stay in the KV cache from pass to pass). The operands formed inside an
+   operation from fp32 arithmetic (normalised activations, softmax probabilities,
+   attention output, SwiGLU output) are kept exact here; the kernels carry them as a
+   bf16 (hi, lo) pair, more precisely than bf16 operands. Residual stream, router and
+   softmax statistics are fp64; router and LM-head logits are rounded to fp32 before
+   the top-k / argmax decision, and conf to fp32 before commit ranking.
 
-Parity pins (tests/test_oracle_pins.py): attention against brute force and closed
-forms; RoPE relative-position invariance; KV-cache pass equal to an uncached
-block-causal sequence forward; MoE top-k against brute force over all subsets and
-the k = E / E = 1 reductions; LM-head confidence against a zero-gain closed form and
-log-sum-exp; commit schedule and sampler invariants. Values produced for random
-weights beyond those properties are "parity unpinned": no page prints a worked
-example.
+Parity pins (tests/test_oracle_pins.py), one or more per function: RMSNorm against
+closed forms (constant and +-a rows, a hand-worked row, scale invariance); bf16
+rounding against its ties-to-even cases, subnormals and torch's conversion;
+attention against brute force and closed forms; RoPE against a hand-worked pairing
+case and relative-position invariance; the SwiGLU expert against a closed form at
+sigmoid(ln 3) = 3/4; MoE top-k against brute force over all subsets and the k = E
+reduction; LM-head confidence against a zero-gain closed form and log-sum-exp; commit
+schedule, strict threshold and sampler invariants; the KV-cache pass against an
+uncached block-causal sequence forward. tests/test_oracle_mutations.py plants a
+plausible mistake in each function in turn and checks that a pin fails. Values
+produced for random weights beyond those properties are "parity unpinned": no page
+prints a worked example.
 """
 
 from __future__ import annotations
@@ -266,7 +275,8 @@ class OracleModel:
     def __init__(self, cfg, weights: Dict[str, np.ndarray]):
         self.cfg = cfg
         c = cfg
-        # every matrix is a bf16 operand (reading 10); norm gains stay as given
+        # every matrix enters its products as a bf16 operand (reading 10); norm gains
+        # stay as given
         self.emb = bf16_store(weights["emb"])
         self.layers = []
         for l in range(c.n_layers):
@@ -305,7 +315,7 @@ class OracleModel:
         k = (y @ lw["wk"].T).reshape(T, c.n_kv_heads, c.head_dim)
         v = (y @ lw["wv"].T).reshape(T, c.n_kv_heads, c.head_dim)
         cos, sin = rope_cos_sin(positions, c.head_dim, c.rope_theta)
-        q = bf16(apply_rope(q, cos, sin))
+        q = bf16(apply_rope(q, cos, sin))      # the attention operands are bf16 (reading 10)
         k = bf16(apply_rope(k, cos, sin))
         v = bf16(v)
         if k_prev is not None and k_prev.shape[0] > 0:

@@ -296,46 +296,81 @@ def test_prefix_kv_is_causal():
         assert not np.array_equal(k_a[l][8:], m.requests[1].k[l][8:])
 
 
-# ---------------------------------------------------------------- planted mistakes
 
-def test_planted_mistakes_are_caught(monkeypatch):
-    """Each pin above must fail when a plausible mistake is planted in the oracle."""
-    q, k, v = rnd((5, 4, 8), 1), rnd((7, 2, 8), 2), rnd((7, 2, 8), 3)
-    good = brute_attention(q, k, v)
 
-    # dropped 1/sqrt(hd) scale
-    def attn_noscale(q, k, v, allowed=None):
-        return oracle.model.attention(q * math.sqrt(q.shape[2]), k, v, allowed)
-    assert not np.allclose(attn_noscale(q, k, v), good, atol=1e-6)
+# ---------------------------------------------------------------- RMSNorm
 
-    # wrong GQA mapping (h % Hkv instead of floor(h * Hkv / H))
-    def attn_mod(q, k, v):
-        out = np.zeros_like(q)
-        for h in range(q.shape[1]):
-            s = q[:, h] @ k[:, h % k.shape[1]].T / math.sqrt(q.shape[2])
-            p = scipy.special.softmax(s, axis=1)
-            out[:, h] = p @ v[:, h % k.shape[1]]
-        return out
-    assert not np.allclose(attn_mod(q, k, v), good, atol=1e-6)
+def test_rmsnorm_closed_forms():
+    eps = 1e-6
+    d = 8
+    # a constant row c: mean(x^2) = c^2, so y = c / sqrt(c^2 + eps); at c = 1e-3 the
+    # eps term is as large as c^2, so it must sit inside the square root
+    for c in (1e-3, 0.5, 3.0, -2.0):
+        y = oracle.rmsnorm(np.full((1, d), c), np.ones(d), eps)
+        assert np.allclose(y, c / math.sqrt(c * c + eps), rtol=1e-13, atol=0)
+    # a row of +-a: every entry keeps its sign and has magnitude a / sqrt(a^2 + eps)
+    sgn = np.array([1, -1, 1, 1, -1, -1, 1, -1], np.float64)
+    y = oracle.rmsnorm(0.25 * sgn[None], np.ones(d), eps)
+    assert np.allclose(y[0], sgn * 0.25 / math.sqrt(0.0625 + eps), rtol=1e-13, atol=0)
+    # by hand: x = (1, 2, 3, 4), mean(x^2) = 30 / 4 = 7.5, gains (1, 0.5, 2, -1)
+    y = oracle.rmsnorm(np.array([[1.0, 2.0, 3.0, 4.0]]), np.array([1.0, 0.5, 2.0, -1.0]), eps)
+    assert np.allclose(y[0], np.array([1.0, 1.0, 6.0, -4.0]) / math.sqrt(7.5 + eps), rtol=1e-13, atol=0)
+    # scale invariance: with eps negligible against mean(x^2), y does not depend on |x|
+    x = rnd((3, 16), 18)
+    g = rnd((16,), 19)
+    assert np.allclose(oracle.rmsnorm(1e3 * x, g, eps), oracle.rmsnorm(x, g, 0.0), rtol=1e-12)
+    # rows are normalised independently
+    two = oracle.rmsnorm(np.stack([np.full(d, 2.0), np.full(d, -0.5)]), np.ones(d), 0.0)
+    assert np.allclose(two, np.stack([np.ones(d), -np.ones(d)]), rtol=1e-15)
 
-    # swapped RoPE sign breaks the pairing special case
-    x = np.array([[[1.0, 0.0, 0.0, 0.0]]])
-    c, s = rope_cos_sin(np.array([1]), 4, 1e4)
-    half = 2
-    bad = np.concatenate([x[..., :half] * c[:, None] + x[..., half:] * s[:, None],
-                          x[..., half:] * c[:, None] - x[..., :half] * s[:, None]], axis=-1)
-    assert not np.allclose(bad[0, 0], [math.cos(1), 0, math.sin(1), 0])
 
-    # [MASK] not excluded: the mask-exclusion pin would see argmax == V-1
-    V, d = 64, 16
-    xx, head = rnd((7, d), 16), rnd((V, d), 17)
-    head[V - 1] = 50.0 * oracle.bf16(xx[0]) / np.linalg.norm(xx[0])
-    monkeypatch.setattr(np, "argmax", np.argmax)
-    y = oracle.rmsnorm(xx, np.ones(d), 1e-6)
-    assert np.argmax(y @ oracle.bf16(head).T, axis=1)[0] == V - 1
+# ---------------------------------------------------------------- bf16 rounding
 
-    # floor rule off: the 12-step schedule would not finish the canvas
-    R = 256
-    for s in range(12):
-        R -= commit_count(R, 0, Policy("threshold", tau=0.9, floor=False), s, 12)
-    assert R == 256
+def test_bf16_rounding_ties_and_edges():
+    # bf16 keeps 7 explicit mantissa bits: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
+    # and goes to the even neighbour 1; 1 + 3 * 2^-8 lies halfway between 1 + 2^-7 (odd)
+    # and 1 + 2^-6 (even)
+    cases = {
+        1.0 + 2.0 ** -8: 1.0,
+        1.0 + 3 * 2.0 ** -8: 1.0 + 2.0 ** -6,
+        -(1.0 + 2.0 ** -8): -1.0,
+        1.0 + 2.0 ** -8 + 2.0 ** -20: 1.0 + 2.0 ** -7,     # just above the tie: up
+        1.0 + 2.0 ** -8 - 2.0 ** -20: 1.0,                  # just below: down
+        2.0 ** -133: 2.0 ** -133,                           # smallest bf16 subnormal
+        3 * 2.0 ** -134: 2.0 ** -132,                       # subnormal tie, to even
+        2.0 ** -149: 0.0,                                   # below half the smallest subnormal
+        0.1: 0.10009765625,                                 # 0x3DCCCCCD -> 0x3DCD
+        65504.0: 65536.0,
+    }
+    got = oracle.bf16(np.array(list(cases), np.float32))
+    assert np.array_equal(got, np.array(list(cases.values()), np.float64))
+    assert np.isinf(oracle.bf16(np.array([3.4e38], np.float32))[0])   # above the bf16 maximum
+
+
+def test_bf16_rounding_matches_torch():
+    import torch
+    x = np.concatenate([uniform_f32(9, 1, 20000, -4, 4), uniform_f32(9, 2, 20000, -1e-3, 1e-3),
+                        (uniform_f32(9, 3, 5000, -1, 1) * np.float32(2.0 ** -130)).astype(np.float32)])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.bf16(x), ref)
+
+
+# ---------------------------------------------------------------- SwiGLU expert
+
+def test_swiglu_expert_closed_form():
+    # sigmoid(ln 3) = 3/4, so silu(ln 3) = 0.75 ln 3 and silu(-ln 3) = -0.25 ln 3
+    l3 = math.log(3.0)
+    y = np.array([[l3, -l3]])
+    wg, wu = np.eye(2), 2.0 * np.eye(2)
+    wd = np.array([[1.0, 0.0], [1.0, 1.0]])
+    # h = silu(Wg y) * (Wu y) = (0.75 l3 * 2 l3, -0.25 l3 * -2 l3) = (1.5, 0.5) l3^2
+    # out = Wd h = (1.5, 2.0) l3^2
+    out = swiglu_expert(y, wg, wu, wd)
+    assert np.allclose(out[0], np.array([1.5, 2.0]) * l3 * l3, rtol=1e-14, atol=0)
+
+
+def test_threshold_is_strictly_above_tau():
+    # "above" the threshold: a confidence equal to tau is not committed
+    conf = np.array([0.9, 0.95, 0.1], np.float32)
+    sel = commit_select(conf, np.ones(3, bool), Policy("threshold", tau=0.9, floor=False), 0, 48)
+    assert list(np.nonzero(sel)[0]) == [1]
