@@ -11,9 +11,15 @@ tokens. The 48 GB of weights exceed the 126 MB L2, so no flush is needed between
 steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep                  # the concurrency workload, B = 1 .. 64
+    python bench.py --routing uniform        # design point: every expert routed evenly
+    python bench.py --ingest-ncu FILE.csv    # record an ncu capture of the gate/up GEMM
 
 Prints one JSON line (rank 0). Under torchrun every rank runs its own replica
-(independent requests, weak scaling); the time is the max over ranks.
+(independent requests, weak scaling); the time is the max over ranks. The headline is
+timed with no kernel timing in the pass; the per-kernel breakdown and the roofline of
+the dominant kernel come from a second timed loop of the same step with CUDA-event
+nodes around the kernels inside the pass graph.
 """
 
 from __future__ import annotations
@@ -23,7 +29,6 @@ import datetime
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -38,8 +43,10 @@ METRIC = "committed tokens/s and denoise passes/s at batch 1; % of bf16 tensor-c
 TIMING_STRIDE = 6   # kernel timing brackets layers 0, 6, 12, ... of each pass
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
-GEMM_SOURCE = os.path.join(ROOT, "masked_block_diffusion_b200", "csrc", "gemm_tc.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "moe_gate_up_gemm_moe26b.md")
+CSRC = os.path.join(ROOT, "masked_block_diffusion_b200", "csrc")
+GEMM_SOURCES = [os.path.join(CSRC, f) for f in ("gemm_tc.cuh", "common.cuh", "engine.cu")]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "moe_gate_up_traffic.json")
+GATE_UP_KERNEL = "regex:gemm_tc_kernel.*EpiSwiGLU"
 
 
 def parse_args():
@@ -56,6 +63,11 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling)")
     ap.add_argument("--max-steps", type=int, default=0, help="override the step budget (profiling)")
     ap.add_argument("--timing-all", action="store_true", help="time every kernel group (diagnostic)")
+    ap.add_argument("--timing-steps", type=int, default=3, help="steps of the kernel-timing loop")
+    ap.add_argument("--routing", choices=["model", "uniform"], default="model",
+                    help="uniform: every canvas token routed evenly over all experts (design point)")
+    ap.add_argument("--sweep", action="store_true", help="concurrency sweep B = 1, 4, 8, 16, 32, 64")
+    ap.add_argument("--ingest-ncu", default="", help="ncu CSV of the gate/up GEMM launches to record")
     return ap.parse_args()
 
 
@@ -91,7 +103,8 @@ def workload_config(w, n_gpus, batch=None):
         "policy": (f"top-{w.k}" if w.policy == "topk" else f"threshold {w.tau} + step-budget floor"),
         "max_steps": w.max_steps,
         "parallelism": "replicas" if n_gpus == 1 else f"replicas x{n_gpus} (independent requests)",
-        "l2": "inputs larger than L2 (48 GB of weights streamed per pass)",
+        "l2": "inputs larger than L2, no flush: 48 GB of weights resident; each pass reads the routed "
+              "experts' weights (measured below as experts_routed_per_layer), the dense weights and the KV cache",
     }
 
 
@@ -109,28 +122,76 @@ def pass_flops(cfg, T, P, R):
     return cfg.n_layers * (lin + attn) + 2 * R * d * cfg.vocab
 
 
-def gate_up_bytes(cfg, T):
+def gate_up_bytes(cfg, T, routed=None):
     """Algorithmic HBM bytes of one grouped gate/up GEMM launch (one layer, T tokens):
-    every expert's gate and up rows (bf16), the gathered token rows as a bf16 hi/lo
-    pair, and the SwiGLU output written as a hi/lo pair."""
-    E = max(1, cfg.n_experts)
+    the gate and up rows of the routed experts (all experts if routed is None), the
+    gathered token rows and the SwiGLU output, activations at bf16 size."""
+    E = max(1, cfg.n_experts) if routed is None else routed
     k = 1 if cfg.dense else cfg.top_k
     N = T * k
-    return E * 2 * cfg.ffn_dim * cfg.d_model * 2 + N * cfg.d_model * 4 + N * cfg.ffn_dim * 4
+    return E * 2 * cfg.ffn_dim * cfg.d_model * 2 + N * cfg.d_model * 2 + N * cfg.ffn_dim * 2
 
 
-def recorded_traffic():
-    """Per-launch DRAM bytes of the gate/up GEMM from the committed ncu summary, if the
-    kernel source is unchanged since the capture; else None."""
+def sources_sha256():
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def parse_ncu_csv(path):
+    """Per launch of an `ncu --csv --print-units base` metrics log: {id: {metric: value}}
+    (units normalised to bytes and nanoseconds) and the kernel names."""
+    import csv
+    scale = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "ns": 1, "nsecond": 1, "usecond": 1e3,
+             "us": 1e3, "msecond": 1e6, "ms": 1e6, "second": 1e9}
+    rows = {}
+    names = {}
+    with open(path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for r in csv.DictReader(lines):
+        if "Metric Name" not in r:
+            continue
+        i = int(r["ID"])
+        v = float(str(r["Metric Value"]).replace(",", ""))
+        v *= scale.get(str(r.get("Metric Unit", "")).strip().lower(), 1)
+        rows.setdefault(i, {})[r["Metric Name"]] = v
+        names[i] = r["Kernel Name"]
+    return rows, names
+
+
+def ingest_ncu(path, workload, routing, command):
+    """Writes TRAFFIC_FILE from an ncu capture of the gate/up GEMM's canvas-pass launches
+    of `workload` under `routing`: mean DRAM bytes and duration per launch, with the hash
+    of the kernel's sources so that the benchmark reports the figure only while those
+    sources are unchanged."""
+    rows, names = parse_ncu_csv(path)
+    ids = sorted(i for i in rows if "EpiSwiGLU" in names[i])
+    if not ids:
+        raise SystemExit(f"{path}: no gate/up GEMM launch")
+    dram = [rows[i].get("dram__bytes_read.sum", 0.0) + rows[i].get("dram__bytes_write.sum", 0.0) for i in ids]
+    dur = [rows[i].get("gpu__time_duration.sum", 0.0) for i in ids]
+    rec = {"kernel": "grouped expert gate/up GEMM + SwiGLU", "launches": len(ids),
+           "dram_bytes_per_launch": statistics.mean(dram), "ns_per_launch_cold": statistics.mean(dur),
+           "workload": workload, "routing": routing, "sources_sha256": sources_sha256(), "command": command,
+           "csv": os.path.basename(path)}
+    os.makedirs(os.path.dirname(TRAFFIC_FILE), exist_ok=True)
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
+
+
+def recorded_traffic(workload, routing):
+    """Mean DRAM bytes per gate/up launch from the recorded ncu capture, if it was taken
+    on this workload and routing with the kernel sources unchanged since; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    txt = open(TRAFFIC_FILE).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    h = re.search(r"gemm_source_sha256:\s*([0-9a-f]+)", txt)
-    if not m or not h:
+    rec = json.load(open(TRAFFIC_FILE))
+    if (rec.get("sources_sha256") != sources_sha256() or rec.get("workload") != workload
+            or rec.get("routing") != routing):
         return None
-    cur = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
-    return float(m.group(1)) if h.group(1) == cur else None
+    return float(rec["dram_bytes_per_launch"])
 
 
 # ------------------------------------------------------------------ clocks
@@ -276,82 +337,119 @@ def prefill_flops(cfg, n):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args):
+def uniform_routing(cfg, T):
+    """Expert ids [n_layers][T][k] that give every expert T * k / E tokens: token t takes
+    experts (t * k + j) mod E, j < k (distinct for k <= E)."""
     import numpy as np
-    import torch
-    from masked_block_diffusion_b200 import Denoiser, DllmError, binding, make_policy
-    from synth import WORKLOADS, prompt_tokens
-    from synth.device import device_blob
+    k, E = cfg.top_k, cfg.n_experts
+    t = np.arange(T)[:, None] * k + np.arange(k)[None, :]
+    return np.broadcast_to((t % E)[None], (cfg.n_layers, T, k)).astype(np.int32)
 
-    world, rank, local = dist_setup()
-    w = resolve_workload(args)
-    cfg = w.model
-    C = cfg.canvas
-    Bq = args.batch or w.batch   # independent requests on this GPU
-    max_ctx = w.prefix + w.n_canvases * C
-    blob = device_blob(cfg)
-    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=Bq)
-    del blob
-    torch.cuda.synchronize()
-    torch.cuda.empty_cache()
-    h, st = den.h, den.stream
-    # requests of this rank: seeds prompt_seed + global request id
-    prompt_np = np.stack([prompt_tokens(cfg.vocab, w.prompt_seed + rank * Bq + r, w.prefix) for r in range(Bq)])
-    d_prompt = torch.from_numpy(prompt_np).cuda()
-    d_canvas = torch.empty((Bq, C), dtype=torch.int32, device="cuda")
-    torch.cuda.synchronize()
-    pol = make_policy(w.policy, w.k, w.tau, w.floor)
-    # the two grouped expert GEMMs are timed inside the graph (--timing-all: every kernel group)
-    # every TIMING_STRIDE-th layer is bracketed with events: few enough event nodes that
-    # the timed pass runs close to an untimed one, every kind still sampled each pass
-    binding.dllm_set_timing(h, ((1 << binding.DLLM_TIMING_KINDS) - 1 if args.timing_all
-                                else (1 << binding.DLLM_TIMING_GATE_UP) | (1 << binding.DLLM_TIMING_DOWN))
-                            | (TIMING_STRIDE << binding.DLLM_TIMING_STRIDE_SHIFT))
 
-    def step(gen_events=None):
-        for r in range(Bq):
-            binding.dllm_reset(h, r)
-            binding.dllm_prefill(h, r, d_prompt[r].data_ptr(), w.prefix)
+class Arm:
+    """One handle on the workload, with the step that every timed loop runs."""
+
+    def __init__(self, args, w, rank, max_batch):
+        import numpy as np
+        import torch
+        from masked_block_diffusion_b200 import Denoiser, binding, make_policy
+        from synth import prompt_tokens
+        from synth.device import device_blob
+        self.args, self.w, self.cfg, self.binding = args, w, w.model, binding
+        C = w.model.canvas
+        blob = device_blob(w.model)
+        self.den = Denoiser(w.model, blob, max_ctx=w.prefix + w.n_canvases * C, max_batch=max_batch)
+        del blob
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        self.h, self.st = self.den.h, self.den.stream
+        self.prompts = np.stack([prompt_tokens(w.model.vocab, w.prompt_seed + rank * max_batch + r, w.prefix)
+                                 for r in range(max_batch)])
+        self.d_prompt = torch.from_numpy(self.prompts).cuda()
+        self.d_canvas = torch.empty((max_batch, C), dtype=torch.int32, device="cuda")
+        self.pol = make_policy(w.policy, w.k, w.tau, w.floor)
+        torch.cuda.synchronize()
+
+    def step(self, B, gen_events=None):
+        """prefill B prompts, then per canvas: generate_block + append. Returns passes run."""
+        import torch
+        from masked_block_diffusion_b200 import DllmError
+        b, h, w = self.binding, self.h, self.w
+        for r in range(B):
+            b.dllm_reset(h, r)
+            b.dllm_prefill(h, r, self.d_prompt[r].data_ptr(), w.prefix)
         passes = 0
         for _ in range(w.n_canvases):
             if gen_events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
-                e0.record(st)
-            code, steps = binding.dllm_generate_block(h, Bq, w.max_steps, pol, d_canvas.data_ptr())
+                e0.record(self.st)
+            code, steps = b.dllm_generate_block(h, B, w.max_steps, self.pol, self.d_canvas.data_ptr())
             if code != 0:
-                raise DllmError(code, "dllm_generate_block", binding.dllm_last_error(h))
+                raise DllmError(code, "dllm_generate_block", b.dllm_last_error(h))
             if gen_events is not None:
                 e1 = torch.cuda.Event(enable_timing=True)
-                e1.record(st)
+                e1.record(self.st)
                 gen_events.append((e0, e1))
             passes += max(steps)
-            binding.dllm_append_kv(h, Bq, 0)
+            b.dllm_append_kv(h, B, 0)
         return passes
 
+    def timed(self, B, steps, world):
+        """Device time of `steps` steps (max over ranks), passes, generate-block time."""
+        import torch
+        gen_events = []
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        t0.record(self.st)
+        passes = 0
+        for _ in range(steps):
+            passes += self.step(B, gen_events)
+        t1.record(self.st)
+        self.st.synchronize()
+        elapsed = max_over_ranks(t0.elapsed_time(t1), world)
+        gen_ms = sum(a.elapsed_time(b) for a, b in gen_events)
+        return elapsed, passes, gen_ms
+
+
+def step_flops(cfg, w, B, passes_per_canvas):
+    C = cfg.canvas
+    return B * prefill_flops(cfg, w.prefix) + w.n_canvases * (
+        passes_per_canvas * pass_flops(cfg, C * B, w.prefix, C * B) + pass_flops(cfg, C * B, w.prefix, 0))
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    world, rank, local = dist_setup()
+    w = resolve_workload(args)
+    if args.sweep:
+        return run_sweep(args, w, world, rank)
+    cfg = w.model
+    C = cfg.canvas
+    Bq = args.batch or w.batch   # independent requests on this GPU
+    arm = Arm(args, w, rank, Bq)
+    b, h = arm.binding, arm.h
+    if args.routing == "uniform":
+        # every canvas pass (and append) routes each token to k experts chosen so that all
+        # E experts get T k / E tokens: the expert GEMMs stream every expert's weights
+        b.dllm_set_debug(h, True)
+        idx = np.ascontiguousarray(uniform_routing(cfg, C * Bq))
+        b.dllm_debug_force_routing(h, idx.ctypes.data, C * Bq)
+
+    # ---- headline: no kernel timing inside the pass graphs
+    b.dllm_set_timing(h, 0)
     for _ in range(args.warmup):
-        step()
-    st.synchronize()
-    barrier(world)
-    binding.dllm_timing_read(h, reset=True)
-    launches0 = binding.dllm_launch_count(h)
+        arm.step(Bq)
+    arm.st.synchronize()
+    launches0 = b.dllm_launch_count(h)
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
-    gen_events = []
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_stop = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    t_start.record(st)
-    passes = 0
-    for _ in range(args.steps):
-        passes += step(gen_events)
-    t_stop.record(st)
-    st.synchronize()
-    torch.cuda.synchronize()
+    elapsed_ms, passes, gen_ms = arm.timed(Bq, args.steps, world)
     clk = clocks.stop()
-    launches = binding.dllm_launch_count(h) - launches0
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop), world)
-    gen_ms = sum(a.elapsed_time(b) for a, b in gen_events)
-    kms, kn, kbytes = binding.dllm_timing_read(h, reset=True)
+    launches = b.dllm_launch_count(h) - launches0
     barrier(world)
 
     from masked_block_diffusion_b200.replicas import aggregate_rate
@@ -359,28 +457,49 @@ def run_ours(args):
     passes_per_canvas = passes / (args.steps * w.n_canvases)
     peaks, peak_src = load_peaks()
 
-    # dominant kernel: the grouped gate/up GEMM (expert weights streamed from HBM)
-    GU, DN = binding.DLLM_TIMING_GATE_UP, binding.DLLM_TIMING_DOWN
+    # ---- kernel breakdown: the same step, with event nodes around the grouped GEMMs (or
+    # every kernel group) of every TIMING_STRIDE-th layer inside the pass graphs
+    kinds = ((1 << b.DLLM_TIMING_KINDS) - 1 if args.timing_all
+             else (1 << b.DLLM_TIMING_GATE_UP) | (1 << b.DLLM_TIMING_DOWN))
+    b.dllm_set_timing(h, kinds | (TIMING_STRIDE << b.DLLM_TIMING_STRIDE_SHIFT))
+    arm.step(Bq)                                   # captures the graphs with their event nodes
+    b.dllm_timing_read(h, reset=True)
+    t_elapsed, t_passes, _ = arm.timed(Bq, max(1, args.timing_steps), world)
+    kms, kn, kbytes = b.dllm_timing_read(h, reset=True)
+    b.dllm_set_timing(h, 0)
+
+    GU, DN = b.DLLM_TIMING_GATE_UP, b.DLLM_TIMING_DOWN
     if kn[GU] == 0 or kms[GU] <= 0:
         raise RuntimeError("no gate/up GEMM launch was timed")
     gu_ms = kms[GU] / kn[GU]
     gu_bytes = kbytes[GU] / kn[GU]          # mean algorithmic bytes per launch (routed experts)
     achieved = kbytes[GU] / (kms[GU] / 1e3) / 1e9
     peak_hbm = float(peaks["hbm_gbs"])
+    act = Bq * C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 2
+    routed = (gu_bytes - act) / (2 * cfg.ffn_dim * cfg.d_model * 2)
+    traffic = recorded_traffic(w.name, args.routing)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_hbm, "unit": "GB/s",
-                "frac": round(achieved / peak_hbm, 4), "traffic": recorded_traffic(),
+                "frac": round(achieved / peak_hbm, 4), "traffic": round(traffic) if traffic else None,
                 "kernel": "grouped expert gate/up GEMM + SwiGLU (tcgen05, one launch per layer)",
-                "bytes_per_launch": round(gu_bytes), "bytes_per_launch_all_experts": gate_up_bytes(cfg, C * Bq),
+                "bytes_per_launch": round(gu_bytes),
+                "bytes_per_launch_all_experts": gate_up_bytes(cfg, C * Bq),
+                "bytes_note": ("algorithmic: bf16 weights of the experts each launch routed to + token rows in "
+                               "+ SwiGLU rows out at bf16 size; the kernel's (hi, lo) activation pairs are "
+                               "overhead, not work"),
+                "kernel_operand_bytes_per_launch": round(gu_bytes + act),
                 "avg_launch_ms": round(gu_ms, 5), "launches_timed": kn[GU],
-                "bytes_note": "weights of the experts each launch routed to + token pair rows + SwiGLU output",
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
+                "timing": (f"CUDA-event nodes inside the pass graph around every {TIMING_STRIDE}th layer's launch, "
+                           f"{max(1, args.timing_steps)} steps after the headline loop"),
+                "peak_source": (f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                                else "fallback 6650 GB/s")}
+    if traffic:
+        roofline["traffic_over_algorithmic"] = round(traffic / gu_bytes, 3)
     dn_ms = max(1e-9, kms[DN] / max(1, kn[DN]))
     dn_gbs = kbytes[DN] / max(1e-9, kms[DN] / 1e3) / 1e9
 
-    step_flops = Bq * prefill_flops(cfg, w.prefix) + w.n_canvases * (
-        passes_per_canvas * pass_flops(cfg, C * Bq, w.prefix, C * Bq) + pass_flops(cfg, C * Bq, w.prefix, 0))
+    flops = step_flops(cfg, w, Bq, passes_per_canvas)
     tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    step_tc = step_flops / (elapsed_ms / args.steps / 1e3) / (tc_peak * 1e12)
+    step_tc = flops / (elapsed_ms / args.steps / 1e3) / (tc_peak * 1e12)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -397,31 +516,34 @@ def run_ours(args):
         "roofline": roofline,
         "down_gemm": {"avg_launch_ms": round(dn_ms, 5), "achieved_gbs": round(dn_gbs, 1),
                       "bytes_per_launch": round(kbytes[DN] / max(1, kn[DN]))},
-        "experts_routed_per_layer": round((kbytes[GU] / kn[GU] - Bq * C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 4)
-                                          / (2 * cfg.ffn_dim * cfg.d_model * 2), 2),
+        "experts_routed_per_layer": round(routed, 2),
         "gpu_launches": int(launches),
         # mean bracketed launch time x launches per pass (n_layers, or 1 for the LM head)
-        "kernel_ms_per_pass": {binding.TIMING_NAMES[k]: round(kms[k] / kn[k] * (
-                                   1 if k == binding.DLLM_TIMING_HEAD else cfg.n_layers), 4)
-                               for k in range(binding.DLLM_TIMING_KINDS) if kn[k]},
+        "kernel_ms_per_pass": {b.TIMING_NAMES[k]: round(kms[k] / kn[k] * (
+                                   1 if k == b.DLLM_TIMING_HEAD else cfg.n_layers), 4)
+                               for k in range(b.DLLM_TIMING_KINDS) if kn[k]},
+        "timing_loop_ms_per_step": round(t_elapsed / max(1, args.timing_steps), 3),
         "timing_layer_stride": TIMING_STRIDE,
         "clocks": clk,
     }
+    if args.routing == "uniform":
+        out["routing"] = ("design point: every canvas token routed to k experts so that all experts get "
+                          "T k / E tokens (forced through the debug routing hook; debug copies of the router "
+                          "logits and residuals run in each layer)")
 
     if not args.no_e2e:
-        prompts = np.ascontiguousarray(prompt_np)
+        prompts = np.ascontiguousarray(arm.prompts[:Bq])
         toks = np.zeros((Bq, w.n_canvases * C), dtype=np.int32)
         stp = np.zeros((Bq * w.n_canvases,), dtype=np.int32)
-        binding.dllm_set_timing(h, 0)
         for _ in range(max(1, args.warmup)):
-            binding.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
-                                  toks.ctypes.data, stp.ctypes.data)
+            b.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, arm.pol,
+                            toks.ctypes.data, stp.ctypes.data)
         barrier(world)
         t0 = time.perf_counter()
         e_passes = 0
         for _ in range(args.steps):
-            binding.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, pol,
-                                  toks.ctypes.data, stp.ctypes.data)
+            b.dllm_generate(h, Bq, prompts.ctypes.data, w.prefix, w.n_canvases, w.max_steps, arm.pol,
+                            toks.ctypes.data, stp.ctypes.data)
             e_passes += int(stp.reshape(Bq, w.n_canvases).max(axis=0).sum())
         t1 = time.perf_counter()
         e_s = max_over_ranks(t1 - t0, world)
@@ -435,7 +557,53 @@ def run_ours(args):
         out["cpu_baseline"] = {"value": round(w.n_canvases * C / times[0][0], 5), "unit": UNIT, "cores": threads,
                                "kind": "oracle", "sample": sample,
                                "sample_seconds": round(times[0][1], 2)}
-    den.close()
+    arm.den.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_sweep(args, w, world, rank):
+    """The concurrency workload: B independent requests (prompt 4096 each, 12 fixed steps)
+    for B = 1, 4, 8, 16, 32, 64 on one handle; aggregate and per-request committed
+    tokens/s and the step's tensor-core fraction for each B, as one JSON record."""
+    import torch
+    from dataclasses import replace
+    from synth import WORKLOADS
+    if args.workload == "c3-moe26b-canvas":
+        w = WORKLOADS["c5-moe26b-batch"]
+        if args.layers:
+            w = replace(w, model=w.model.with_layers(args.layers), name=f"{w.name}-{args.layers}L")
+    cfg, C = w.model, w.model.canvas
+    batches = [B for B in w.batches if not args.batch or B <= args.batch]
+    arm = Arm(args, w, rank, max(batches))
+    peaks, peak_src = load_peaks()
+    tc_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    rows = []
+    for B in batches:
+        for _ in range(args.warmup):
+            arm.step(B)
+        elapsed_ms, passes, gen_ms = arm.timed(B, args.steps, world)
+        step_s = elapsed_ms / args.steps / 1e3
+        ppc = passes / (args.steps * w.n_canvases)
+        rows.append({"batch": B, "aggregate_tokens_per_s": round(world * B * C * w.n_canvases / step_s, 2),
+                     "per_request_tokens_per_s": round(C * w.n_canvases / step_s, 2),
+                     "ms_per_step": round(elapsed_ms / args.steps, 3),
+                     "denoise_ms_per_pass": round(gen_ms / max(1, passes), 3),
+                     "passes_per_canvas": ppc,
+                     "step_tc_frac": round(step_flops(cfg, w, B, ppc) / step_s / (tc_peak * 1e12), 4)})
+    clk = clocks.stop()
+    arm.den.close()
+    out = {"metric": "aggregate and per-request committed tokens/s over concurrent requests", "unit": UNIT,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+           "dtype": "bf16", "data": "synthetic (seeded random-init weights N(0,0.02), uniform prompt tokens)",
+           "config": workload_config(w, world, max(batches)), "sweep": rows, "clocks": clk,
+           "tc_peak": f"{tc_peak} TFLOP/s sustained bf16 ({peak_src})",
+           "step": "prefill of B prompts + 12 denoising passes over B canvases + append, all B in one batch"}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -474,6 +642,9 @@ def run_reference(args):
 
 def main():
     args = parse_args()
+    if args.ingest_ncu:
+        ingest_ncu(args.ingest_ncu, resolve_workload(args).name, args.routing, os.environ.get("NCU_COMMAND", ""))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

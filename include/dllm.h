@@ -26,8 +26,14 @@
  *     ordinary host memory owned by the caller. The handle owns its repacked weights, the
  *     KV cache, all scratch and its CUDA graphs.
  *   - All GPU work is ordered on the stream given to dllm_create. Calls return once the
- *     work is queued, except dllm_generate_block, dllm_generate and dllm_check, which
- *     synchronise that stream.
+ *     work is queued, except dllm_create, dllm_generate_block, dllm_generate, dllm_check,
+ *     dllm_set_debug / dllm_debug_* and dllm_set_wait_limit, which synchronise that
+ *     stream. dllm_prefill and dllm_generate with a host prompt copy it before returning.
+ *   - Device-side errors: every wait inside a kernel is bounded. A kernel that gives up
+ *     one records an error word on the device and returns; the context stays usable.
+ *     The pass that saw it commits nothing (remaining = -1, conf = NaN, argmax = -1),
+ *     later passes commit nothing either, and the next synchronising call (dllm_check,
+ *     dllm_generate_block, dllm_generate) returns DLLM_E_TIMEOUT and clears the word.
  *   - Canvas layout: int32 tokens [B][C] and uint8 mask [B][C] (1 = still [MASK]); request
  *     b of a batched call uses KV slot b. Masked positions hold mask_id.
  *   - Not thread-safe: one host thread per handle.
@@ -78,12 +84,19 @@ typedef struct {
  * TOPK: commit the min(k, R) most confident masked positions.
  * THRESHOLD: commit every masked position with conf > tau; with floor = 1 commit at
  * least max(1, ceil(R / (max_steps - step))) of the most confident ones, so that the
- * canvas completes within max_steps. Ties go to the lower position. */
+ * canvas completes within max_steps. Ties go to the lower position.
+ * t2t = 1 adds token-to-token editing (What changes, section 4.3, LLaDA2.1's T2T next
+ * to mask-to-token decoding): a position committed before the pass is re-written to the
+ * pass's argmax when that token differs from its own and conf > edit_tau; it stays
+ * committed, and R counts masked positions only. t2t = 0 (a zeroed struct): committed
+ * tokens never change. */
 typedef struct {
   int kind;
   int k;
   float tau;
   int floor;
+  int t2t;
+  float edit_tau;
 } dllm_policy;
 
 /* Creates a handle. `weights` is the blob in this order, every tensor row-major
@@ -109,6 +122,9 @@ int dllm_prefill(dllm_handle* h, int req, const int32_t* prompt, int n);
  * conf_out (device float [req_count][C]) and argmax_out (device int32 [req_count][C])
  * receive the pass's confidence and argmax of every position when not NULL.
  * remaining_out (device int32 [req_count]) receives the masked count after the commit.
+ * Returns once the pass is queued; it reads no device result, so a kernel that gave
+ * up a bounded wait shows as remaining_out = -1, conf_out = NaN and argmax_out = -1 of
+ * that pass (nothing committed), and as DLLM_E_TIMEOUT from the next dllm_check.
  * Errors: DLLM_E_INVAL, DLLM_E_STATE (slot without prefill), DLLM_E_CTX_FULL. */
 int dllm_denoise_step(dllm_handle* h, int req_count, int32_t* canvas, uint8_t* mask, const dllm_policy* policy,
                       int step, int max_steps, float* conf_out, int32_t* argmax_out, int32_t* remaining_out);
@@ -125,6 +141,15 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
  * generated canvases) to the KV cache: one bidirectional pass whose K/V are kept at
  * positions P..P+C-1; each request's prefix then grows by C. */
 int dllm_append_kv(dllm_handle* h, int req_count, const int32_t* canvas);
+
+/* Approximate append (What changes, section 5, "KV caching": Fast-dLLM's training-free,
+ * block-wise approximate KV cache): the K/V that each request's last canvas pass wrote
+ * at positions P..P+C-1 are kept as the finished canvas's cache entries, with no extra
+ * pass; each prefix grows by C. Those K/V were computed while the positions that pass
+ * committed were still [MASK], so later passes see a slightly different cache than after
+ * dllm_append_kv. Errors: DLLM_E_STATE (a slot without a canvas pass since its last
+ * prefill or append), DLLM_E_CTX_FULL, DLLM_E_INVAL. */
+int dllm_append_kv_approx(dllm_handle* h, int req_count);
 
 /* End to end with host buffers: for each request r < req_count, prefill
  * prompts[r][0..n_prompt-1], then n_canvases times generate a canvas and append it.
@@ -147,6 +172,14 @@ int dllm_check(dllm_handle* h);
 /* Kernel launches issued by the handle since creation (graph replays count their
  * kernels). */
 long long dllm_launch_count(const dllm_handle* h);
+
+/* Limit, in nanoseconds, of the pipeline waits inside the kernels (a stage waiting for
+ * its TMA copy, an MMA for its operands, an epilogue for its accumulator, a split-K
+ * rank for its peers); ns <= 0 restores the default of 2 s. The waits that let copies
+ * and MMAs already in flight land before a kernel exits keep the default. The limit is
+ * one value per device, shared by every handle on it; it exists so that the timeout
+ * path (DLLM_E_TIMEOUT, context intact) can be exercised. Synchronises the stream. */
+int dllm_set_wait_limit(dllm_handle* h, long long ns);
 
 /* Debug inspection of the last canvas pass (enable first; enabling drops captured
  * graphs). what: 0 = final residual x, fp32 [T][d]; 1 = router logits of `layer`,
@@ -173,8 +206,9 @@ int dllm_debug_force_routing(dllm_handle* h, const int32_t* idx, int T);
  * are summed per kind after each pass of dllm_generate_block. dllm_timing_read fills
  * total_ms[kind], launches[kind] and bytes[kind] (arrays of DLLM_TIMING_KINDS); bytes
  * are filled for the two grouped GEMMs: the launches' algorithmic HBM bytes, i.e. the
- * weights of the experts each layer routed to plus the token operand rows read and the
- * outputs written. If reset, the sums are zeroed. Changing the mask drops captured
+ * bf16 weights of the experts each layer routed to plus the token rows read and the
+ * results written, both counted at bf16 size (2 bytes per element). If reset, the sums
+ * are zeroed. Changing the mask drops captured
  * graphs. Kinds: grouped gate/up GEMM; grouped down GEMM; attention (+ split merge);
  * QKV GEMM; O GEMM; routing (pre-FFN RMSNorm, router, top-k, permute, gather);
  * combine of the expert outputs (with the next RMSNorm fused into it);
@@ -200,7 +234,9 @@ void dllm_destroy(dllm_handle* h);
 
 /* ---- single-operation entry points (the pass's kernels on caller buffers) ---------
  * All pointers are device memory, stream = cudaStream_t. They validate shapes, queue
- * the work and return; errors as above. */
+ * the work and return; errors as above. They return before the kernels run, so a
+ * kernel that gives up a bounded wait is reported in the outputs instead: the GEMM
+ * fills D with NaN, the LM heads write conf = NaN and argmax = -1 in every row. */
 
 /* D[M][N] (fp32, row-major) = A[M][K] * B[N][K]^T with bf16 A, B; the tcgen05 GEMM core.
  * K % 64 == 0, N % 128 == 0. */
@@ -220,11 +256,17 @@ int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, 
  * a fixed budget and forbids other cudaMalloc calls, or a path where an allocation's
  * implicit synchronisation or failure is not acceptable.
  * Arguments and results are those of dllm_op_lm_head_conf (caller-owned device buffers).
- * Scratch: one fixed device array inside the library (3 MiB), present on every GPU that
- * loads the library until the process exits. Limits: T <= 1024 rows, V <= 65536;
- * larger sizes return DLLM_E_INVAL and print the limit to stderr.
+ * Scratch: one fixed device array inside the library (3 MiB). The CUDA runtime reserves
+ * it on a device when it loads the library's module there, which it may do lazily, at
+ * the library's first call on that device (whichever entry point that is); from then on
+ * the device holds it until the process exits. A caller with a fixed device budget
+ * should therefore make one call into the library on each device before its own
+ * allocator takes the device. Limits: T <= 1024 rows, V <= 65536; larger sizes return
+ * DLLM_E_INVAL and print the limit to stderr.
  * The first call on a device looks up that array's device address (once per device,
- * with the device current); make that first call before any stream capture.
+ * with the device current) and keeps it; make that first call before any stream
+ * capture, and do not keep calling across a cudaDeviceReset of that device (the array
+ * may move when the module is loaded again).
  * Every call on a device shares the one array and it keeps the last call's contents:
  * calls that may overlap on the GPU (other streams, other host threads) race on it, so
  * order them on one stream. Calls no cudaMalloc, cudaFree or allocating library

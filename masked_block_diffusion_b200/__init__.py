@@ -93,6 +93,12 @@ class Denoiser:
         binding.dllm_append_kv(self.h, req_count, 0 if canvas is None else canvas.data_ptr())
         self._sync_out()
 
+    def append_kv_approx(self, req_count: int):
+        """Keeps the last canvas pass's K/V as the finished canvases' cache entries."""
+        self._sync_in()
+        binding.dllm_append_kv_approx(self.h, req_count)
+        self._sync_out()
+
     def generate(self, prompts: np.ndarray, n_canvases: int, max_steps: int, policy: dllm_policy):
         """End to end with host buffers: prompts int32 [B][n] -> tokens int32 [B][n_canvases*C]."""
         prompts = np.ascontiguousarray(prompts, dtype=np.int32)

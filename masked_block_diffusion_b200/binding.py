@@ -36,7 +36,7 @@ EXPORTS = [
     "dllm_generate", "dllm_reset", "dllm_prefix_len", "dllm_check", "dllm_launch_count",
     "dllm_set_debug", "dllm_debug_read", "dllm_debug_force_routing", "dllm_last_error", "dllm_destroy",
     "dllm_op_gemm_bf16", "dllm_op_lm_head_conf", "dllm_op_lm_head_conf_noalloc", "dllm_set_timing",
-    "dllm_timing_read",
+    "dllm_timing_read", "dllm_set_wait_limit", "dllm_append_kv_approx",
 ]
 DLLM_TIMING_GATE_UP = 0
 DLLM_TIMING_DOWN = 1
@@ -64,7 +64,8 @@ class dllm_config(ctypes.Structure):
 
 
 class dllm_policy(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int), ("k", ctypes.c_int), ("tau", ctypes.c_float), ("floor", ctypes.c_int)]
+    _fields_ = [("kind", ctypes.c_int), ("k", ctypes.c_int), ("tau", ctypes.c_float), ("floor", ctypes.c_int),
+                ("t2t", ctypes.c_int), ("edit_tau", ctypes.c_float)]
 
 
 class DllmError(RuntimeError):
@@ -108,6 +109,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dllm_op_lm_head_conf_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
         "dllm_set_timing": (_i, [_vp, _i]),
         "dllm_timing_read": (_i, [_vp, _vp, _vp, _vp, _i]),
+        "dllm_set_wait_limit": (_i, [_vp, ctypes.c_longlong]),
+        "dllm_append_kv_approx": (_i, [_vp, _i]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -128,9 +131,10 @@ def make_config(model, max_ctx: int, max_batch: int) -> dllm_config:
         weight_dtype=DLLM_WEIGHTS_F32 if model.weight_dtype == "f32" else DLLM_WEIGHTS_BF16)
 
 
-def make_policy(kind: str, k: int = 0, tau: float = 0.9, floor: bool = True) -> dllm_policy:
+def make_policy(kind: str, k: int = 0, tau: float = 0.9, floor: bool = True, t2t: bool = False,
+                edit_tau: float = 0.9) -> dllm_policy:
     return dllm_policy(kind=DLLM_POLICY_TOPK if kind == "topk" else DLLM_POLICY_THRESHOLD, k=int(k),
-                       tau=float(tau), floor=1 if floor else 0)
+                       tau=float(tau), floor=1 if floor else 0, t2t=1 if t2t else 0, edit_tau=float(edit_tau))
 
 
 def _check(code: int, where: str, handle=None):
@@ -171,6 +175,10 @@ def dllm_generate_block(h, req_count, max_steps, policy: dllm_policy, canvas_ptr
 
 def dllm_append_kv(h, req_count, canvas_ptr=0):
     _check(load().dllm_append_kv(h, req_count, _vp(canvas_ptr)), "dllm_append_kv", h)
+
+
+def dllm_append_kv_approx(h, req_count):
+    _check(load().dllm_append_kv_approx(h, req_count), "dllm_append_kv_approx", h)
 
 
 def dllm_generate(h, req_count, prompts_host_ptr, n_prompt, n_canvases, max_steps, policy: dllm_policy,
@@ -245,3 +253,8 @@ def dllm_op_lm_head_conf_noalloc(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, ar
     """The fused LM head on a fixed in-library scratch array (no device allocation)."""
     _check(load().dllm_op_lm_head_conf_noalloc(_vp(y_ptr), _vp(head_ptr), T, d, V, mask_id, _vp(conf_ptr),
                                                _vp(argmax_ptr), _vp(stream_ptr)), "dllm_op_lm_head_conf_noalloc")
+
+
+def dllm_set_wait_limit(h, ns: int):
+    """Pipeline-wait limit of the kernels on this device in ns (<= 0: the 2 s default)."""
+    _check(load().dllm_set_wait_limit(h, int(ns)), "dllm_set_wait_limit", h)

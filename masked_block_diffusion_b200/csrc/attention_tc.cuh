@@ -349,6 +349,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ---------------- TMA producer: K(j) and V(j) in order, each into its own ring
     const uint64_t pol = policy_evict_last();
     bool ok = true;
+    int k_issued = 0, v_issued = 0;   // K and V blocks whose loads were issued
     mbar_arrive_expect_tx(q_full, G::kQ);
     for (int a = 0; a < AT; ++a) tma_load_3d(sQ + a * 128 * 128, &tm_q, q_full, a * 64, g * grp, b * C + q0);
     for (int j = 0; j < nblk && ok; ++j) {
@@ -358,13 +359,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!mbar_wait(&k_empty[st], ph, abort_flag)) { ok = false; break; }
       mbar_arrive_expect_tx(&k_full[st], G::kKV);
       for (int a = 0; a < AT; ++a) tma_load_2d(sK + st * G::kKV + a * G::kKatom, &tm_k, &k_full[st], a * 64, row, pol);
+      k_issued = j + 1;
       if (!mbar_wait(&v_empty[st], ph, abort_flag)) { ok = false; break; }
       mbar_arrive_expect_tx(&v_full[st], G::kKV);
       for (int a = 0; a < AT; ++a) tma_load_2d(sV + st * G::kKV + a * G::kKatom, &tm_v, &v_full[st], a * 64, row, pol);
+      v_issued = j + 1;
     }
     if (!ok) {
       atomicExch(p.err, kDevTimeoutProducer);
       *abort_flag = 1;
+      // the loads already issued land before the CTA's shared memory goes away: the
+      // Q tile and the last fill of each K and V stage
+      mbar_drain(q_full, 0);
+      for (int jj = max(0, k_issued - ST); jj < k_issued; ++jj) mbar_drain(&k_full[jj % ST], (jj / ST) & 1);
+      for (int jj = max(0, v_issued - ST); jj < v_issued; ++jj) mbar_drain(&v_full[jj % ST], (jj / ST) & 1);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
@@ -420,8 +428,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       *abort_flag = 1;
     }
     umma_commit(drain);
-    unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
+    mbar_drain(drain, 0);
   } else if (warp >= 2) {
     softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_final,
                      reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);

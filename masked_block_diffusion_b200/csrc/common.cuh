@@ -26,6 +26,12 @@ enum DevError : int {
 // Upper bound of every spin wait on an mbarrier (global-timer nanoseconds).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Limit of the pipeline waits (mbar_wait, mbar_wait_cluster): kWaitLimitNs unless
+// dllm_set_wait_limit changed it for this device (tests of the timeout path). The drain
+// waits that let copies and MMAs already in flight land before a CTA exits always use
+// kWaitLimitNs, so a short pipeline limit never cuts them short.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
 DLLM_DEV float bf16_to_f32(bf16_t v) { return __uint_as_float(((uint32_t)v) << 16); }
 
 DLLM_DEV bf16_t f32_to_bf16(float f) {
@@ -82,16 +88,24 @@ DLLM_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete. Gives up after kWaitLimitNs, or as
+// Waits for the phase of `parity` to complete. Gives up after g_wait_limit_ns, or as
 // soon as another role of the CTA has raised *abort; returns false then.
 DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long limit = g_wait_limit_ns;
   unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit) return false;
   }
+}
+
+// Bounded wait (always kWaitLimitNs) for a phase that work already in flight will
+// complete: used on the abort paths before a CTA's shared memory or TMEM goes away.
+DLLM_DEV void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity) && global_ns() - t0 < kWaitLimitNs) {}
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch
@@ -149,13 +163,14 @@ DLLM_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait on a barrier that other CTAs of the cluster arrive on (acquire, cluster
-// scope); false after kWaitLimitNs or once *abort is raised.
+// scope); false after g_wait_limit_ns or once *abort is raised.
 DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const unsigned long long limit = g_wait_limit_ns;
   unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit) return false;
   }
 }
 

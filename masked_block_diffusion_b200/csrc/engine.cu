@@ -78,7 +78,11 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kMoeBN[4] = {32, 64, 128, 256};
+// Token-operand boxes of the grouped expert GEMMs: a chunk of up to kMoeChunk tokens is
+// loaded from boxes of these heights (its count rounded up to 16), so the MMA width
+// follows the chunk's token count.
+constexpr int kMoeBN[4] = {16, 32, 64, 128};
+constexpr int kMoeChunk = 128;
 
 struct LayerW {
   float* attn_norm = nullptr;
@@ -152,6 +156,7 @@ struct dllm_handle {
   bf16_t* hbuf_lo = nullptr;
   CUtensorMap tm_y, tm_ao, tm_xg[4], tm_h[4];
   CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
+  CUtensorMap* d_tok_maps = nullptr;   // device copies: [xg hi 16..128 | xg lo | h hi | h lo]
   CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // canvas passes use the tensor-core attention
@@ -164,6 +169,7 @@ struct dllm_handle {
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
+  std::vector<char> passed;  // per slot: a canvas pass wrote K/V at P..P+C-1 since the last prefill / append
   int32_t* d_P = nullptr;    // [max_batch]
   int32_t* d_slot = nullptr; // [max_batch] = 0..max_batch-1
   int32_t* d_pre_pos = nullptr;   // [1] = 0
@@ -250,14 +256,6 @@ int dalloc(dllm_handle* h, T** p, size_t count) {
   } while (0)
 
 int ceil_div(long a, long b) { return (int)((a + b - 1) / b); }
-
-int moe_bn_index(int N, int E) {
-  // token chunk width of the grouped GEMMs: 64, or 128 once the mean tokens per expert
-  // pass 64 (prefill, large batches). Routing is often far from uniform, and every chunk
-  // is its own work item, so a skewed expert costs more items rather than a long pole.
-  const double mean = (double)N / (double)E;
-  return mean <= 64.0 ? 1 : 2;
-}
 
 // Threads of a one-row-per-block kernel over d floats: one float4 column each (up to
 // 1024), so that all of a row's loads are in flight at once.
@@ -526,45 +524,46 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   return launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
 }
 
-// One grouped gate/up (or down) GEMM at chunk width BN with MPI weight tiles per work
-// item and ACC accumulator buffers (MPI * ACC * 2 BN TMEM columns <= 512).
-template <int BN, int MPI, int ACC>
-cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L, int bi) {
+// One grouped gate/up (or down) GEMM over chunks of up to kMoeChunk tokens, with MPI
+// weight tiles per work item and ACC accumulator buffers (MPI * ACC * 2 * kMoeChunk TMEM
+// columns <= 512). The MMA width of each chunk follows its token count.
+template <int MPI, int ACC>
+cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
+  constexpr int BN = kMoeChunk;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128, BN};
+  PersistentGroupedSched<MPI> s{h->d_tok_maps, h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128,
+                                BN};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[bi], d / 64, 1, s, e, nullptr,
-                                               &h->tm_xg_lo[bi]);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[3], d / 64, 1, s, e, nullptr,
+                                               &h->tm_xg_lo[3]);
 }
 
-template <int BN, int MPI, int ACC>
-cudaError_t moe_down(dllm_handle* h, const LayerW& L, int bi) {
+template <int MPI, int ACC>
+cudaError_t moe_down(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
+  constexpr int BN = kMoeChunk;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128, BN};
+  PersistentGroupedSched<MPI> s{h->d_tok_maps + 8, h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128,
+                                BN};
   EpiDown<BN> e{h->obuf, d};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[bi], F / 64, 1, s, e, nullptr,
-                                               &h->tm_h_lo[bi]);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[3], F / 64, 1, s, e, nullptr,
+                                               &h->tm_h_lo[3]);
 }
 
-// Grouped expert GEMMs of one layer. Chunk width 64 tokens while the mean tokens per
-// expert stay below 64 (canvas passes), else 128 (prefill, large batches). At width 64,
-// down takes two weight tiles per work item (its 22 m tiles leave enough items to spread
-// over the SMs) and gate/up one (with 11 m tiles, pairs would leave too few items per
-// layer to balance).
-cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int N, int l, uint32_t timed) {
-  const int bi = moe_bn_index(N, h->E);
+// Grouped expert GEMMs of one layer. gate/up: one weight tile per item, two accumulator
+// buffers; down: two weight tiles per item sharing the token chunk (its 22 m tiles leave
+// enough items to spread over the SMs), or one with DLLM_MOE_PAIR=0.
+cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int l, uint32_t timed) {
   cudaError_t r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-  r = bi >= 2 ? moe_gate_up<128, 1, 2>(h, L, 2) : moe_gate_up<64, 1, 2>(h, L, 1);
+  r = moe_gate_up<1, 2>(h, L);
   if (r != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  r = bi >= 2 ? moe_down<128, 1, 2>(h, L, 2)
-              : (h->moe_pair ? moe_down<64, 2, 2>(h, L, 1) : moe_down<64, 1, 2>(h, L, 1));
+  r = h->moe_pair ? moe_down<2, 1>(h, L) : moe_down<1, 2>(h, L);
   if (r != cudaSuccess) return r;
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
@@ -625,13 +624,13 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       h->launches++;
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
-                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeBN[moe_bn_index(N, h->E)],
+                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeChunk,
                 timed ? h->routed_stat + l : nullptr));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(std::min(1024, (d / 8 + 31) / 32 * 32)), 0, h->y, h->y_lo,
                 h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
-    CK(moe_gemms(h, L, N, l, timed));
+    CK(moe_gemms(h, L, l, timed));
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
     const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
     if (next_gain)
@@ -672,10 +671,11 @@ int run_canvas_pass(dllm_handle* h, int B, int mode) {
     CK((launch_gemm<256, 3, 1, kSplitA>(h, dim3(mt * nvt), h->tm_y, h->tm_head, d / 64, 0, s, e, &h->tm_y_lo)));
   }
   CK(launch_k(h, lm_merge_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->lm_m, h->lm_s, h->lm_i, T, nvt,
-              h->conf, h->argmax));
+              h->conf, h->argmax, (const int*)h->d_err));
   const int threads = ceil_div(C, 32) * 32;
   CK(launch_k(h, commit_kernel, dim3(B), dim3(threads), C * (sizeof(float) + 1), h->canvas, h->mask, h->conf,
-              h->argmax, C, h->d_policy, h->d_step, h->d_remaining, nullptr, nullptr));
+              h->argmax, C, h->d_policy, h->d_step, h->d_remaining, nullptr, nullptr,
+              (const int*)h->d_err));
   h->launches += 2;
   CK(tmark(h, tm, DLLM_TIMING_HEAD, 0, 1));
   CK(cudaGetLastError());
@@ -721,22 +721,29 @@ int check_requests(dllm_handle* h, int B) {
   return DLLM_OK;
 }
 
-int upload_P(dllm_handle* h) {
-  std::vector<int32_t> v(h->P.size());
-  for (size_t i = 0; i < v.size(); ++i) v[i] = h->P[i] < 0 ? 0 : h->P[i];
-  CK(cudaMemcpyAsync(h->d_P, v.data(), sizeof(int32_t) * v.size(), cudaMemcpyHostToDevice, h->st));
-  CK(cudaStreamSynchronize(h->st));   // v is a local: keep the copy inside its lifetime
+// Device copies of small host state (prefix lengths, slot ids, policy, step counters)
+// are written by one-block kernels that take the values as arguments: no host staging
+// buffer has to outlive the call, so no call synchronises for them.
+int set_ints(dllm_handle* h, int32_t* dst, int n, int v, bool add) {
+  CK(launch_k(h, set_ints_kernel, dim3(1), dim3(64), 0, dst, n, v, add ? 1 : 0));
+  h->launches++;
   return DLLM_OK;
 }
 
-int upload_policy(dllm_handle* h, const dllm_policy* p, int max_steps) {
+int check_policy(dllm_handle* h, const dllm_policy* p, int max_steps) {
   if (!p) return fail(h, DLLM_E_INVAL, "policy is NULL");
   if (p->kind != DLLM_POLICY_TOPK && p->kind != DLLM_POLICY_THRESHOLD) return fail(h, DLLM_E_INVAL, "policy kind");
   if (p->kind == DLLM_POLICY_TOPK && p->k < 1) return fail(h, DLLM_E_INVAL, "top-k policy needs k >= 1");
   if (max_steps < 1) return fail(h, DLLM_E_INVAL, "max_steps < 1");
-  PolicyDev pd{p->kind == DLLM_POLICY_TOPK ? 0 : 1, p->k, p->tau, p->floor, max_steps};
-  CK(cudaMemcpyAsync(h->d_policy, &pd, sizeof(pd), cudaMemcpyHostToDevice, h->st));
-  CK(cudaStreamSynchronize(h->st));
+  return DLLM_OK;
+}
+
+// The policy, and the step counter of requests 0..n_steps-1 (n_steps = 0: counters kept).
+int stage_step(dllm_handle* h, const dllm_policy* p, int max_steps, int step, int n_steps) {
+  const PolicyDev pd{p->kind == DLLM_POLICY_TOPK ? 0 : 1, p->k, p->tau, p->floor, max_steps, p->t2t ? 1 : 0,
+                     p->edit_tau};
+  CK(launch_k(h, stage_step_kernel, dim3(1), dim3(64), 0, pd, step, n_steps, h->d_policy, h->d_step));
+  h->launches++;
   return DLLM_OK;
 }
 
@@ -751,8 +758,8 @@ int check_device_error(dllm_handle* h) {
 }
 
 // After a timed pass over T tokens: adds each grouped GEMM launch's event time and its
-// algorithmic bytes (weights of the experts the layer routed to, the token operand
-// pair read, the output written).
+// algorithmic bytes (weights of the experts the layer routed to, the token rows read
+// and the results written, both at bf16 size).
 void accumulate_timing(dllm_handle* h, int T) {
   const int L = h->c.n_layers;
   std::vector<int32_t> nr(L);
@@ -773,8 +780,10 @@ void accumulate_timing(dllm_handle* h, int T) {
       }
       h->t_ms[kind] += ms;
       h->t_n[kind] += 1;
-      if (kind == DLLM_TIMING_GATE_UP) h->t_bytes[kind] += nr[l] * 2 * F * d * 2 + N * d * 4 + N * F * 4;
-      if (kind == DLLM_TIMING_DOWN) h->t_bytes[kind] += nr[l] * d * F * 2 + N * F * 4 + N * d * 4;
+      // the method's bytes: the routed experts' bf16 weights, the bf16 token rows in and
+      // the bf16 results out (the (hi, lo) pairs and fp32 outputs are the kernels' own)
+      if (kind == DLLM_TIMING_GATE_UP) h->t_bytes[kind] += nr[l] * 2 * F * d * 2 + N * d * 2 + N * F * 2;
+      if (kind == DLLM_TIMING_DOWN) h->t_bytes[kind] += nr[l] * d * F * 2 + N * F * 2 + N * d * 2;
     }
   }
 }
@@ -1002,6 +1011,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
 
   // ---- request state
   h->P.assign(c.max_batch, -1);
+  h->passed.assign(c.max_batch, 0);
   DA(h->d_P, c.max_batch);
   DA(h->d_slot, c.max_batch);
   DA(h->d_pre_pos, 1);
@@ -1054,6 +1064,18 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     }
   }
   if (!ok) return fail(h, DLLM_E_CUDA, "cuTensorMapEncodeTiled failed");
+  {
+    // the grouped GEMMs read their token-operand maps from device memory
+    CUtensorMap maps[16];
+    for (int i = 0; i < 4; ++i) {
+      maps[i] = h->tm_xg[i];
+      maps[4 + i] = h->tm_xg_lo[i];
+      maps[8 + i] = h->tm_h[i];
+      maps[12 + i] = h->tm_h_lo[i];
+    }
+    DA(h->d_tok_maps, 16);
+    CK(cudaMemcpy(h->d_tok_maps, maps, sizeof(maps), cudaMemcpyHostToDevice));
+  }
   CK(cudaFuncSetAttribute(reinterpret_cast<const void*>(router_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
                           kRouterTok * d * (int)sizeof(float)));
   CK(cudaStreamSynchronize(h->st));
@@ -1079,14 +1101,15 @@ int prefill_impl(dllm_handle* h, int req, const int32_t* prompt, int n, bool pro
   if (n + c.canvas > c.max_ctx) return fail(h, DLLM_E_CTX_FULL, "prompt + canvas exceeds max_ctx");
   CK(cudaMemcpyAsync(h->d_tokens, prompt, sizeof(int32_t) * n,
                      prompt_on_host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, h->st));
-  const int32_t s = req;
-  CK(cudaMemcpyAsync(h->d_pre_slot, &s, sizeof(int32_t), cudaMemcpyHostToDevice, h->st));
+  int r = set_ints(h, h->d_pre_slot, 1, req, false);
+  if (r) return r;
   CK(launch_k(h, embed_kernel, dim3(n), dim3(128), 0, h->emb, h->d_tokens, nullptr, c.mask_id, c.d_model, h->x));
   h->launches++;
-  int r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, false, 0u, nullptr);
+  r = run_layers(h, n, 1, n, h->d_pre_pos, h->d_pre_slot, 1, 1, false, 0u, nullptr);
   if (r) return r;
   h->P[req] = n;
-  return upload_P(h);
+  h->passed[req] = 0;
+  return set_ints(h, h->d_P + req, 1, n, false);
 }
 
 }  // namespace
@@ -1139,15 +1162,14 @@ int dllm_denoise_step(dllm_handle* h, int req_count, int32_t* canvas, uint8_t* m
   int r = check_requests(h, req_count);
   if (r) return r;
   if (step < 0) return fail(h, DLLM_E_INVAL, "step < 0");
-  if ((r = upload_policy(h, policy, max_steps))) return r;
+  if ((r = check_policy(h, policy, max_steps))) return r;
   const int C = h->c.canvas, B = req_count;
-  std::vector<int32_t> steps(B, step);
-  CK(cudaMemcpyAsync(h->d_step, steps.data(), sizeof(int32_t) * B, cudaMemcpyHostToDevice, h->st));
+  if ((r = stage_step(h, policy, max_steps, step, B))) return r;
   CK(cudaMemcpyAsync(h->canvas, canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
   CK(cudaMemcpyAsync(h->mask, mask, (size_t)B * C, cudaMemcpyDeviceToDevice, h->st));
-  CK(cudaStreamSynchronize(h->st));   // `steps` is a local
   if ((r = replay_pass(h, B, 0))) return r;
   h->last_B = B;
+  for (int b = 0; b < B; ++b) h->passed[b] = 1;
   CK(cudaMemcpyAsync(canvas, h->canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
   CK(cudaMemcpyAsync(mask, h->mask, (size_t)B * C, cudaMemcpyDeviceToDevice, h->st));
   if (conf_out) CK(cudaMemcpyAsync(conf_out, h->conf, sizeof(float) * B * C, cudaMemcpyDeviceToDevice, h->st));
@@ -1163,8 +1185,9 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
   if (!h) return DLLM_E_INVAL;
   int r = check_requests(h, req_count);
   if (r) return r;
-  if ((r = upload_policy(h, policy, max_steps))) return r;
+  if ((r = check_policy(h, policy, max_steps))) return r;
   const int C = h->c.canvas, B = req_count;
+  if ((r = stage_step(h, policy, max_steps, 0, 0))) return r;
   CK(launch_k(h, canvas_init_kernel, dim3(ceil_div((long)B * C, 256)), dim3(256), 0, h->canvas, h->mask, B * C,
               h->c.mask_id, h->d_step, B));
   h->launches++;
@@ -1173,13 +1196,20 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
   bool all_done = false;
   for (; s < max_steps && !all_done; ++s) {
     if ((r = replay_pass(h, B, 0))) return r;
+    for (int b = 0; b < B; ++b) h->passed[b] = 1;
     CK(cudaMemcpyAsync(h->h_remaining, h->d_remaining, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, h->st));
     CK(cudaStreamSynchronize(h->st));
     if (h->timing) accumulate_timing(h, B * C);
     all_done = true;
+    bool aborted = false;
     for (int b = 0; b < B; ++b) {
       if (h->h_remaining[b] == 0 && done_at[b] < 0) done_at[b] = s + 1;
       if (h->h_remaining[b] != 0) all_done = false;
+      if (h->h_remaining[b] < 0) aborted = true;   // a kernel of the pass gave up a bounded wait
+    }
+    if (aborted) {
+      ++s;
+      break;
     }
   }
   h->last_B = B;
@@ -1199,8 +1229,25 @@ int dllm_append_kv(dllm_handle* h, int req_count, const int32_t* canvas) {
   const int C = h->c.canvas, B = req_count;
   if (canvas) CK(cudaMemcpyAsync(h->canvas, canvas, sizeof(int32_t) * B * C, cudaMemcpyDeviceToDevice, h->st));
   if ((r = replay_pass(h, B, 1))) return r;
-  for (int b = 0; b < B; ++b) h->P[b] += C;
-  return upload_P(h);
+  for (int b = 0; b < B; ++b) {
+    h->P[b] += C;
+    h->passed[b] = 0;
+  }
+  return set_ints(h, h->d_P, B, C, true);
+}
+
+int dllm_append_kv_approx(dllm_handle* h, int req_count) {
+  if (!h) return DLLM_E_INVAL;
+  int r = check_requests(h, req_count);
+  if (r) return r;
+  for (int b = 0; b < req_count; ++b)
+    if (!h->passed[b]) return fail(h, DLLM_E_STATE, "slot " + std::to_string(b) + " has no canvas pass to keep");
+  // the K/V that the last canvas pass wrote at P..P+C-1 stay where they are
+  for (int b = 0; b < req_count; ++b) {
+    h->P[b] += h->c.canvas;
+    h->passed[b] = 0;
+  }
+  return set_ints(h, h->d_P, req_count, h->c.canvas, true);
 }
 
 int dllm_generate(dllm_handle* h, int req_count, const int32_t* prompts, int n_prompt, int n_canvases, int max_steps,
@@ -1232,7 +1279,8 @@ int dllm_reset(dllm_handle* h, int req) {
   if (!h) return DLLM_E_INVAL;
   if (req < 0 || req >= h->c.max_batch) return fail(h, DLLM_E_INVAL, "req out of range");
   h->P[req] = -1;
-  return upload_P(h);
+  h->passed[req] = 0;
+  return set_ints(h, h->d_P + req, 1, 0, false);
 }
 
 int dllm_prefix_len(const dllm_handle* h, int req) {
@@ -1248,6 +1296,14 @@ int dllm_check(dllm_handle* h) {
 }
 
 long long dllm_launch_count(const dllm_handle* h) { return h ? h->launches : -1; }
+
+int dllm_set_wait_limit(dllm_handle* h, long long ns) {
+  if (!h) return DLLM_E_INVAL;
+  const unsigned long long v = ns > 0 ? (unsigned long long)ns : kWaitLimitNs;
+  CK(cudaStreamSynchronize(h->st));
+  CK(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+  return DLLM_OK;
+}
 
 int dllm_set_debug(dllm_handle* h, int on) {
   if (!h) return DLLM_E_INVAL;
@@ -1368,6 +1424,10 @@ int dllm_op_gemm_bf16(const uint16_t* A, const uint16_t* B, float* D, int M, int
   DenseSched s{M, mt, 128};
   EpiStoreF32<128> e{D, N, N};
   cudaError_t r = launch_gemm<128, 4, 1, kSplitNone>(h, dim3(mt * (N / 128)), ta, tb, K / 64, 0, s, e);
+  if (r == cudaSuccess) {
+    poison_on_error_kernel<<<148, 256, 0, tmp.st>>>(err, D, (long)M * N);
+    r = cudaGetLastError();
+  }
   cudaFreeAsync(err, tmp.st);
   tmp.d_err = nullptr;
   if (r != cudaSuccess) return DLLM_E_CUDA;
@@ -1397,7 +1457,7 @@ int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, 
   EpiLMHead<256> e{pm, ps, pi, nvt, mask_id};
   cudaError_t r = launch_gemm<256, 4, 1, kSplitNone>(h, dim3(mt * nvt), ta, tb, d / 64, 0, s, e);
   if (r == cudaSuccess) {
-    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax);
+    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax, err);
     r = cudaGetLastError();
   }
   cudaFreeAsync(pm, tmp.st);
@@ -1486,7 +1546,7 @@ extern "C" int dllm_op_lm_head_conf_noalloc(const uint16_t* y, const uint16_t* h
   EpiLMHead<256> e{pm, ps, pi, nvt, mask_id};
   cudaError_t r = launch_gemm<256, 4, 1, kSplitNone>(h, dim3(mt * nvt), ta, tb, d / 64, 0, s, e);
   if (r == cudaSuccess) {
-    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax);
+    lm_merge_kernel<<<ceil_div((long)T * 32, 256), 256, 0, tmp.st>>>(pm, ps, pi, T, nvt, conf, argmax, err);
     r = cudaGetLastError();
   }
   tmp.d_err = nullptr;

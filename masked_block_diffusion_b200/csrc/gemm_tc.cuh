@@ -21,13 +21,20 @@ struct Tile {
   int n_valid;   // columns of the tile inside the problem
   int mt, nt;    // dense: (m tile, n tile); grouped: (m tile inside the expert, expert)
   int m_count = 1;   // m tiles of this work item (128 rows apart, sharing the B tile)
+  int n_cols = 0;    // accumulator columns computed (per operand half); 0 = the full BN
 };
+
+// Columns of the tile an epilogue reads: the full BN, or the rounded-up valid columns
+// of a grouped tile whose MMA width follows its token count.
+template <int BN>
+DLLM_DEV int tile_cols(const Tile& t) { return t.n_cols > 0 ? t.n_cols : BN; }
 
 // One output tile per CTA over an M x N problem; m tiles vary fastest so that the CTAs
 // sharing a weight tile run close together (the second read hits L2).
 struct DenseSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = 1;
+  static constexpr bool kDynN = false;
   static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
@@ -53,6 +60,7 @@ template <int KS>
 struct DenseSplitKSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = KS;
+  static constexpr bool kDynN = false;
   static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
@@ -83,12 +91,20 @@ struct DenseSplitKSched {
 // The routing tables are copied into shared memory once per CTA (stage(), run by every
 // thread before the roles split), so that finding an item's expert is a short search in
 // shared memory instead of a chain of dependent global loads on the producer's path.
+//
+// The MMA width follows each chunk's token count (kDynN): a chunk of n tokens loads only
+// n16 = n rounded up to 16 rows of the token pair, composed from boxes of 128, 64, 32
+// and 16 rows (tok_maps: [hi 16, 32, 64, 128 | lo 16, 32, 64, 128], tensor maps in
+// global memory), stacked as [hi n16 rows | lo n16 rows], and one MMA of N = 2 n16 reads
+// both. An expert with few tokens then costs its weight bytes and little else.
 template <int MPI>
 struct PersistentGroupedSched {
   static constexpr int kMaxRouted = 256;
   static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
   static constexpr int kKSplit = 1;
+  static constexpr bool kDynN = true;
   static constexpr int kMPerItem = MPI;
+  const CUtensorMap* tok_maps;   // 8 token-operand maps (see above), device memory
   const int* offsets;        // [E+1] token ranges per expert
   const int* routed;         // [E] experts with at least one token, ascending
   const int* n_routed;       // [1]
@@ -151,6 +167,7 @@ struct PersistentGroupedSched {
     t.b_row = off + chunk * BN;
     t.m_valid = 128;
     t.n_valid = min(BN, cnt - chunk * BN);
+    t.n_cols = (t.n_valid + 15) & ~15;
     return t;
   }
 };
@@ -340,6 +357,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
+    if constexpr (Sched::kDynN)
+      for (int i = 0; i < 8; ++i) tma_prefetch_desc(sched.tok_maps + i);
     const uint64_t pol_first = policy_evict_first();
     const uint64_t pol_last = policy_evict_last();
     const uint64_t pol_a = a_stream_first ? pol_first : pol_last;
@@ -352,12 +371,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       const Tile t = sched.tile(j);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], L::kStageBytes - (MPI - t.m_count) * L::kAtile);
-        for (int u = 0; u < t.m_count; ++u)
-          tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
-        if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
-        tma_load_2d(sB + stage * L::kBStage, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
-        if (SPLIT == kSplitB) tma_load_2d(sB2 + stage * L::kBStage, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
+        if constexpr (Sched::kDynN) {
+          static_assert(SPLIT == kSplitB && BN == 128, "dynamic N: stacked token pair, up to 128 rows");
+          const int n16 = t.n_cols;
+          mbar_arrive_expect_tx(&full[stage], t.m_count * L::kAtile + 2 * n16 * 128);
+          for (int u = 0; u < t.m_count; ++u)
+            tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
+          // [hi n16 rows | lo n16 rows], each half from boxes of 128 / 64 / 32 / 16 rows
+          uint8_t* dst = sB + stage * L::kBStage;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            int off = 0;
+#pragma unroll
+            for (int bi = 3; bi >= 0; --bi) {
+              const int rows = 16 << bi;
+              if ((n16 - off) & rows) {
+                tma_load_2d(dst + (half * n16 + off) * 128, sched.tok_maps + half * 4 + bi, &full[stage], kb * 64,
+                            t.b_row + off, pol_b);
+                off += rows;
+              }
+            }
+          }
+        } else {
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes - (MPI - t.m_count) * L::kAtile);
+          for (int u = 0; u < t.m_count; ++u)
+            tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
+          if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
+          tma_load_2d(sB + stage * L::kBStage, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
+          if (SPLIT == kSplitB)
+            tma_load_2d(sB2 + stage * L::kBStage, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
+        }
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -370,8 +413,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       for (int i = 0; i < min(issued, STAGES); ++i) {
         s = (s + STAGES - 1) % STAGES;
         if (s == STAGES - 1) p ^= 1;
-        unsigned long long t0 = global_ns();
-        while (!mbar_try_wait(&full[s], p) && global_ns() - t0 < kWaitLimitNs) {}
+        mbar_drain(&full[s], p);
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -384,7 +426,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       const uint32_t acc_phase = (j / ACC_BUFS) & 1;
       if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const int mc = MPI > 1 ? sched.tile(j).m_count : 1;
+      int mc = 1;
+      uint32_t idesc = kIdesc;
+      if constexpr (MPI > 1 || Sched::kDynN) {
+        const Tile tj = sched.tile(j);
+        mc = tj.m_count;
+        if constexpr (Sched::kDynN) idesc = idesc_bf16_f32(128, 2 * tj.n_cols);
+      }
       const uint32_t d_tmem = tmem_base + acc * MPI * kCols;
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -394,15 +442,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc,
+          umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc,
                     (kb != kb_begin || kk != 0) ? 1u : 0u);
           if (SPLIT == kSplitA)
-            umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), kIdesc, 1);
+            umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc, 1);
 #pragma unroll
           for (int u = 1; u < MPI; ++u)
             if (u < mc)
               umma_bf16(d_tmem + u * kCols, sdesc_k_sw128(a0 + u * L::kAtile + kk * 32), sdesc_k_sw128(b0 + kk * 32),
-                        kIdesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
+                        idesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -415,8 +463,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     }
     // wait for every MMA issued by this thread before TMEM is released
     umma_commit(drain);
-    unsigned long long t0 = global_ns();
-    while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {}
+    mbar_drain(drain, 0);
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
@@ -439,12 +486,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         t.a_row += u * 128;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (acc * MPI + u) * kCols;
         if constexpr (SPLIT == kSplitB) {
-          // D = D_hi + D_lo, into the first BN columns the epilogue reads
+          // D = D_hi + D_lo, into the first columns the epilogue reads (the lo half starts
+          // at the tile's column count: BN, or n16 for a dynamic-width tile)
+          const int ncols = tile_cols<BN>(t);
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 16) {
+          for (int c = 0; c < ncols; c += 16) {
             float hi[16], lo[16];
             tmem_ld16(taddr + c, hi);
-            tmem_ld16(taddr + BN + c, lo);
+            tmem_ld16(taddr + ncols + c, lo);
 #pragma unroll
             for (int i = 0; i < 16; ++i) hi[i] += lo[i];
             tmem_st16(taddr + c, hi);
@@ -637,8 +686,9 @@ struct EpiSwiGLU {
   DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t* smem) const {
     float* us = reinterpret_cast<float*>(smem);
     const int f = t.mt * 64 + (r & 63);
+    const int ncols = tile_cols<BN>(t);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = 0; c < ncols; c += 16) {
       float v[16];
       tmem_ld16(taddr + c, v);
       if (r >= 64) {
@@ -706,8 +756,9 @@ struct EpiDown {
   int d;
   DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
     const int dd = t.mt * 128 + r;
+    const int ncols = tile_cols<BN>(t);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = 0; c < ncols; c += 16) {
       float v[16];
       tmem_ld16(taddr + c, v);
 #pragma unroll

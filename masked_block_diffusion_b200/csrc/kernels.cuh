@@ -444,14 +444,23 @@ DLLM_DEV void lse_combine(float& m, float& s, int& i, float m2, float s2, int i2
 }
 
 // conf[t] = 1 / sum_v exp(l_v - max), argmax[t] = lowest id reaching the max.
-// One warp per row over the row's vocabulary-tile partials.
+// One warp per row over the row's vocabulary-tile partials. If a kernel before this one
+// gave up a bounded wait (*err != 0), the partials are incomplete: every row gets
+// conf = NaN and argmax = -1 instead.
 __global__ void lm_merge_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
                                 const int32_t* __restrict__ pi, int rows, int n_tiles, float* __restrict__ conf,
-                                int32_t* __restrict__ argmax) {
+                                int32_t* __restrict__ argmax, const int* __restrict__ err) {
   pdl_begin();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= rows) return;
+  if (err && *err) {
+    if (lane == 0) {
+      conf[t] = __int_as_float(0x7fc00000);
+      argmax[t] = -1;
+    }
+    return;
+  }
   float m = -INFINITY, s = 0.f;
   int i = 0x7fffffff;
   for (int j = lane; j < n_tiles; j += 32) {
@@ -479,18 +488,28 @@ struct PolicyDev {
   float tau;
   int floor;
   int max_steps;
+  int t2t;        // token-to-token editing of committed positions
+  float edit_tau;
 };
 
 // One CTA per request (C <= 1024 positions). Commits the n most confident masked
 // positions (fp32 conf, ties to the lower position): top-k: n = min(k, R);
 // threshold: n = max(#{conf > tau}, n_min) with the step-budget floor
 // n_min = max(1, ceil(R / (S_max - s))), capped at R. Writes the committed token,
-// clears the mask bit, stores R - n and advances the request's step counter.
+// clears the mask bit, stores R - n and advances the request's step counter. With T2T
+// editing on, a position committed before this pass is re-written to the pass's argmax
+// when that token differs and conf > edit_tau (the mask and R are left alone). If a
+// kernel of the pass gave up a bounded wait (*err != 0), nothing is committed or edited
+// and the remaining count is -1.
 __global__ void commit_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict__ mask, const float* __restrict__ conf,
                               const int32_t* __restrict__ argmax, int C, const PolicyDev* __restrict__ pol,
                               int32_t* __restrict__ step, int32_t* __restrict__ remaining, float* __restrict__ conf_out,
-                              int32_t* __restrict__ argmax_out) {
+                              int32_t* __restrict__ argmax_out, const int* __restrict__ err) {
   pdl_begin();
+  if (*err) {
+    if (threadIdx.x == 0) remaining[blockIdx.x] = -1;
+    return;
+  }
   extern __shared__ uint8_t smc[];
   float* sc = reinterpret_cast<float*>(smc);
   uint8_t* sm = smc + C * sizeof(float);
@@ -533,10 +552,40 @@ __global__ void commit_kernel(int32_t* __restrict__ canvas, uint8_t* __restrict_
       mask[o] = 0;
     }
   }
+  if (i < C && !mi && P.t2t) {
+    const int a = argmax[o];
+    if (a != canvas[o] && ci > P.edit_tau) canvas[o] = a;
+  }
   if (i == 0) {
     remaining[b] = R - n;
     step[b] = s + 1;
   }
+}
+
+// The step's policy and, for n_steps > 0, the step counters of requests 0..n_steps-1.
+// The values arrive as kernel arguments, so the caller keeps no host buffer alive and
+// the call needs no synchronisation.
+__global__ void stage_step_kernel(PolicyDev pd, int step, int n_steps, PolicyDev* __restrict__ pol,
+                                  int32_t* __restrict__ steps) {
+  pdl_begin();
+  if (threadIdx.x == 0) *pol = pd;
+  for (int i = threadIdx.x; i < n_steps; i += blockDim.x) steps[i] = step;
+}
+
+// dst[i] = v (add = 0) or dst[i] += v (add = 1) for i < n: prefix lengths and slot ids
+// set without a host staging buffer.
+__global__ void set_ints_kernel(int32_t* __restrict__ dst, int n, int v, int add) {
+  pdl_begin();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = add ? dst[i] + v : v;
+}
+
+// After a single GEMM: if a kernel gave up a bounded wait, D is incomplete; fill it
+// with NaN so that a caller who cannot wait for an error code still sees it.
+__global__ void poison_on_error_kernel(const int* __restrict__ err, float* __restrict__ d, long n) {
+  pdl_begin();
+  if (!*err) return;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    d[i] = __int_as_float(0x7fc00000);
 }
 
 // Fresh all-[MASK] canvases and zeroed step counters.

@@ -21,11 +21,12 @@ from .model import (
     lm_head_conf,
     commit_count,
     commit_select,
+    edit_select,
     sequence_forward,
 )
 
 __all__ = [
     "Policy", "OracleModel", "bf16", "rmsnorm", "rope_cos_sin", "apply_rope", "attention",
     "router_topk", "swiglu_expert", "moe_ffn", "lm_head_conf", "commit_count",
-    "commit_select", "sequence_forward",
+    "commit_select", "edit_select", "sequence_forward",
 ]

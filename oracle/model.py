@@ -52,7 +52,17 @@ Readings where the pages are silent (all listed in the design notes):
    attention output, SwiGLU output) are kept exact here; the kernels carry them as a
    bf16 (hi, lo) pair, more precisely than bf16 operands. Residual stream, router and
    softmax statistics are fp64; router and LM-head logits are rounded to fp32 before
-   the top-k / argmax decision, and conf to fp32 before commit ranking.
+   the top-k / argmax decision, and conf to fp32 before commit ranking;
+11. token-to-token editing (What changes, section 4.3, LLaDA2.1: the model may revise
+   tokens it already wrote; the pages give no rule, so the plainest one that mirrors
+   the threshold commit): with T2T on, a position committed before the pass is
+   re-written to the pass's argmax when that token differs from its own and the pass's
+   confidence there is above edit_tau; a re-written position stays committed, and the
+   masked count is the commit's alone;
+12. approximate append (What changes, section 5 "KV caching": Fast-dLLM's
+   training-free, block-wise approximate cache): the finished canvas's K/V are taken
+   from its last denoising pass, computed while the positions that pass committed
+   were still [MASK], instead of from one more pass over the finished canvas.
 
 Parity pins (tests/test_oracle_pins.py), one or more per function: RMSNorm against
 closed forms (constant and +-a rows, a hand-worked row, scale invariance); bf16
@@ -61,8 +71,9 @@ attention against brute force and closed forms; RoPE against a hand-worked pairi
 case and relative-position invariance; the SwiGLU expert against a closed form at
 sigmoid(ln 3) = 3/4; MoE top-k against brute force over all subsets and the k = E
 reduction; LM-head confidence against a zero-gain closed form and log-sum-exp; commit
-schedule, strict threshold and sampler invariants; the KV-cache pass against an
-uncached block-causal sequence forward. tests/test_oracle_mutations.py plants a
+schedule, strict threshold, T2T edit rule and sampler invariants; the KV-cache pass
+against an uncached block-causal sequence forward; the approximate append against the
+last pass's own K/V and the exact append at a canvas without a final commit. tests/test_oracle_mutations.py plants a
 plausible mistake in each function in turn and checks that a pin fails. Values
 produced for random weights beyond those properties are "parity unpinned": no page
 prints a worked example.
@@ -99,6 +110,9 @@ def bf16_store(w) -> np.ndarray:
     if not np.any(u & np.uint32(0xFFFF)):
         return w                      # already bf16-exact: no copy
     return bf16(w).astype(np.float32)
+
+
+_bf16_store = bf16_store
 
 
 # --------------------------------------------------------------------------------------
@@ -225,6 +239,8 @@ class Policy:
     k: int = 1
     tau: float = 0.9
     floor: bool = True
+    t2t: bool = False        # token-to-token editing of committed positions (reading 11)
+    edit_tau: float = 0.9    # a committed token is re-written when the pass's conf exceeds it
 
 
 def commit_count(R: int, n_above: int, policy: Policy, step: int, s_max: int) -> int:
@@ -259,6 +275,22 @@ def commit_select(conf: np.ndarray, mask: np.ndarray, policy: Policy, step: int,
     return sel
 
 
+def edit_select(conf: np.ndarray, argmax: np.ndarray, canvas: np.ndarray, mask: np.ndarray,
+                policy: Policy) -> np.ndarray:
+    """Boolean [C]: the committed positions this pass re-writes (T2T, reading 11).
+
+    A position committed before the pass is re-written to the pass's argmax when that
+    token differs from the one it holds and the pass's confidence there (fp32) is above
+    edit_tau. Masked positions are the commit's business, never the edit's.
+    """
+    if not policy.t2t:
+        return np.zeros(np.asarray(mask).shape[0], dtype=bool)
+    conf32 = np.asarray(conf, dtype=np.float32)
+    committed = ~np.asarray(mask, dtype=bool)
+    differs = np.asarray(argmax) != np.asarray(canvas)
+    return committed & differs & (conf32 > np.float32(policy.edit_tau))
+
+
 # --------------------------------------------------------------------------------------
 # the model
 
@@ -267,16 +299,25 @@ class _Request:
         self.k = [None] * n_layers      # per layer [P][Hkv][hd] (bf16 values)
         self.v = [None] * n_layers
         self.P = 0
+        self.last_k = None              # K/V of the request's last canvas pass (per layer)
+        self.last_v = None
 
 
 class OracleModel:
     """The denoiser over named weights (float32 arrays, e.g. from synth.gen_weights)."""
 
-    def __init__(self, cfg, weights: Dict[str, np.ndarray]):
+    def __init__(self, cfg, weights: Dict[str, np.ndarray], f64_matrices: bool = False):
+        """f64_matrices keeps every matrix as float64 (the same bf16 values) instead of
+        float32, so that the products do not convert their operands on every call: faster
+        for repeated passes, twice the memory, identical results."""
         self.cfg = cfg
         c = cfg
         # every matrix enters its products as a bf16 operand (reading 10); norm gains
         # stay as given
+        if f64_matrices:
+            bf16_store = lambda w: _bf16_store(w).astype(np.float64)   # noqa: E731
+        else:
+            bf16_store = _bf16_store
         self.emb = bf16_store(weights["emb"])
         self.layers = []
         for l in range(c.n_layers):
@@ -372,32 +413,51 @@ class OracleModel:
     def denoise_pass(self, req: int, canvas: np.ndarray, mask: np.ndarray,
                      rec: Optional[dict] = None):
         """One pass: conf [C] (fp32) and argmax [C] for every canvas position."""
-        x, _, _ = self._canvas_forward(req, canvas, mask, rec)
+        x, ks, vs = self._canvas_forward(req, canvas, mask, rec)
+        st = self.requests[req]
+        st.last_k, st.last_v = ks, vs
         out = lm_head_conf(x, self.final_norm, self.head, self.cfg.mask_id, self.cfg.rms_eps,
                            return_logits=rec is not None)
         if rec is not None:
             conf, arg, logits = out
-            srt = np.sort(logits, axis=1)
-            rec["logit_margin"] = srt[:, -1] - srt[:, -2]
+            top2 = np.partition(logits, -2, axis=1)[:, -2:]      # the two largest, either order
+            rec["logit_margin"] = np.abs(top2[:, 1] - top2[:, 0])
             rec["final_x"] = x
             return conf, arg
         return out
 
-    def append(self, req: int, canvas: np.ndarray):
-        """Bidirectional pass over the finished canvas; its K/V join the cache (reading 6)."""
+    def append(self, req: int, canvas: np.ndarray, rec: Optional[dict] = None):
+        """Bidirectional pass over the finished canvas; its K/V join the cache (reading 6).
+
+        rec, if given, receives the pass's per-layer records (as in denoise_pass).
+        """
         st = self.requests[req]
         C = np.asarray(canvas).size
-        _, ks, vs = self._canvas_forward(req, canvas, np.zeros(C, dtype=bool))
+        _, ks, vs = self._canvas_forward(req, canvas, np.zeros(C, dtype=bool), rec)
         for l in range(self.cfg.n_layers):
             st.k[l] = np.concatenate([st.k[l], ks[l]], axis=0) if st.k[l] is not None else ks[l]
             st.v[l] = np.concatenate([st.v[l], vs[l]], axis=0) if st.v[l] is not None else vs[l]
         st.P += C
 
+    def append_approx(self, req: int):
+        """Approximate append (Fast-dLLM-style reuse, reading 12): the finished canvas's
+        K/V are those its last denoising pass computed, taken as they are; no extra pass."""
+        st = self.requests[req]
+        if st.last_k is None:
+            raise ValueError("no canvas pass to reuse")
+        C = st.last_k[0].shape[0]
+        for l in range(self.cfg.n_layers):
+            st.k[l] = np.concatenate([st.k[l], st.last_k[l]], axis=0) if st.k[l] is not None else st.last_k[l]
+            st.v[l] = np.concatenate([st.v[l], st.last_v[l]], axis=0) if st.v[l] is not None else st.last_v[l]
+        st.P += C
+        st.last_k = st.last_v = None
+
     def generate_block(self, req: int, policy: Policy, s_max: int, trace: bool = False):
         """Denoise one all-[MASK] canvas until no position is masked or S_max passes ran.
 
         Returns (canvas, steps, trace list). Each trace entry holds the pass's input
-        canvas/mask, conf, argmax, the commit set and the masked count after it.
+        canvas/mask, conf, argmax, the commit set, the edit set (T2T) and the masked
+        count after it.
         """
         c = self.cfg
         C = c.canvas
@@ -410,10 +470,11 @@ class OracleModel:
             rec = {} if trace else None
             conf, arg = self.denoise_pass(req, canvas, mask, rec)
             sel = commit_select(conf, mask, policy, s, s_max)
+            edit = edit_select(conf, arg, canvas, mask, policy)
             if trace:
                 tr.append(dict(step=s, canvas=canvas.copy(), mask=mask.copy(), conf=conf,
-                               argmax=arg, commit=sel.copy(), rec=rec))
-            canvas = np.where(sel, arg, canvas)
+                               argmax=arg, commit=sel.copy(), edit=edit.copy(), rec=rec))
+            canvas = np.where(sel | edit, arg, canvas)
             mask = mask & ~sel
             steps += 1
             if trace:

@@ -10,7 +10,9 @@ within 2e-2 of the row's largest magnitude.
 
 from __future__ import annotations
 
+import functools
 import math
+import os
 
 import numpy as np
 import torch
@@ -23,10 +25,16 @@ MARGIN = 1e-3
 REL = 2e-2
 
 
+@functools.lru_cache(maxsize=1)
+def cached_weights(cfg):
+    """The seeded weights of cfg, generated once for the tests that share a model."""
+    return gen_weights(cfg, threads=os.cpu_count() or 8)
+
+
 def build_pair(cfg, prefix: int, prompt_seed: int, max_ctx: int, max_batch: int = 1):
-    W = gen_weights(cfg)
+    W = cached_weights(cfg)
     blob = blob_from_weights(cfg, W)
-    orc = OracleModel(cfg, W)
+    orc = OracleModel(cfg, W, f64_matrices=cfg.d_model >= 2048)
     den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=max_batch)
     del blob
     prompt = prompt_tokens(cfg.vocab, prompt_seed, prefix)
@@ -62,8 +70,9 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
     """Replays every oracle step on the GPU and checks the decisions and values."""
     C = cfg.canvas
     stats = stats if stats is not None else {"route_pinned": 0, "route_total": 0, "arg_pinned": 0,
-                                             "arg_total": 0, "commit_pinned": 0, "steps": 0}
-    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor)
+                                             "arg_total": 0, "commit_pinned": 0, "steps": 0, "edits": 0,
+                                             "edit_pinned": 0}
+    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor, policy.t2t, policy.edit_tau)
     den.set_debug(True)
     for e in orc_trace:
         rec = e["rec"]
@@ -120,9 +129,23 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
         if commit_margin(e["conf"], old_mask, n, policy) > MARGIN:
             assert np.array_equal(gpu_commit, e["commit"]), f"step {e['step']}: commit set differs"
             stats["commit_pinned"] += 1
-        # committed positions hold the pass's argmax; earlier commits are untouched (M2T)
+        # newly committed positions hold the pass's argmax
         assert np.array_equal(new_canvas[gpu_commit], arg[gpu_commit])
-        assert np.array_equal(new_canvas[~old_mask], e["canvas"][~old_mask])
+        # earlier commits: untouched (M2T); with T2T, re-written exactly where the oracle
+        # edits, wherever that decision is pinned (argmax margin, and the log-confidence
+        # margin to edit_tau, above 1e-3), and only ever to the pass's argmax
+        committed = ~old_mask
+        gpu_edit = committed & (new_canvas != e["canvas"])
+        if policy.t2t:
+            pinned = committed & lm_sel & (np.abs(np.log(e["conf"].astype(np.float64))
+                                                  - math.log(policy.edit_tau)) > MARGIN)
+            bad = np.nonzero(pinned & (gpu_edit != e["edit"]))[0]
+            assert bad.size == 0, f"step {e['step']}: edit set differs at {bad[:8]}"
+            assert np.array_equal(new_canvas[gpu_edit], arg[gpu_edit])
+            stats["edits"] += int(gpu_edit.sum())
+            stats["edit_pinned"] += int((pinned & e["edit"]).sum())
+        else:
+            assert not gpu_edit.any(), f"step {e['step']}: a committed token changed"
         assert not np.any(new_mask & ~old_mask)
         stats["steps"] += 1
     if not cfg.dense:
@@ -132,7 +155,7 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
 
 
 def check_generate_invariants(cfg, den: Denoiser, policy: Policy, s_max: int, expect_steps=None):
-    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor)
+    pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor, policy.t2t, policy.edit_tau)
     code, canvas, steps = den.generate_block(1, s_max, pol)
     assert code == 0, code
     c = canvas.cpu().numpy()[0]

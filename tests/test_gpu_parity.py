@@ -5,6 +5,8 @@ and the 26B model's layer shapes (E = 128, top-8, F = 704, head_dim 176, V = 655
 with two layers. Every oracle step is replayed on the GPU from the oracle's canvas.
 """
 
+import math
+
 import numpy as np
 import pytest
 
@@ -110,8 +112,231 @@ def test_parity_batched_requests_small_moe():
     den.close()
 
 
-def test_parity_moe26b_shapes_two_layers():
-    # full-width layers of the 26B model; threshold 0.9 + floor, 12-step budget
-    stats, steps, gsteps, agree = run_workload("c4-moe26b-1024out", n_layers=2, prefix=1024)
-    assert steps == 12 and gsteps == 12
+def _append_both(orc, den, cfg, canvas):
+    """Appends the oracle's finished canvas on both sides; the GPU's append pass runs on
+    the oracle's experts of that pass, so that a near-tie cannot move the cached K/V."""
+    import torch
+    rec = {}
+    orc.append(0, canvas, rec)
+    t = torch.from_numpy(canvas.astype(np.int32)[None]).cuda()
+    if cfg.dense:
+        den.append_kv(1, t)
+        return
+    den.set_debug(True)
+    den.force_routing(np.stack(rec["topk_idx"]))
+    den.append_kv(1, t)
+    den.force_routing(None)
+    den.set_debug(False)
+
+
+def test_parity_moe26b_four_canvas_chain():
+    """The 1024-token workload of the 26B model on two full-width layers: prompt 4096,
+    four canvases of 256, threshold 0.9 with the floor, 12 steps each, the finished
+    canvas appended after each, so the prefix grows 4096 -> 5120 and attention reads up
+    to 5120 keys over its key-range splits. Every one of the 48 steps is compared."""
+    w = WORKLOADS["c4-moe26b-1024out"]
+    cfg = w.model.with_layers(2)
+    C, P, S = cfg.canvas, w.prefix, w.max_steps
+    orc, den, _ = build_pair(cfg, P, w.prompt_seed, P + w.n_canvases * C)
+    pol = Policy(w.policy, k=w.k, tau=w.tau, floor=w.floor)
+    stats = None
+    try:
+        for ci in range(w.n_canvases):
+            canvas, steps, trace = orc.generate_block(0, pol, S, trace=True)
+            assert steps == S
+            stats = compare_trace(cfg, trace, den, pol, S, stats)
+            _append_both(orc, den, cfg, canvas)
+            assert den.prefix_len(0) == P + (ci + 1) * C
+    finally:
+        den.close()
+    assert stats["steps"] == w.n_canvases * S
     assert stats["route_pinned"] > 0.9 * stats["route_total"]
+    assert stats["arg_pinned"] > 0.9 * stats["arg_total"]
+
+
+def _threshold_between(conf, lo, hi):
+    """A tau strictly between two adjacent confidences of ranks lo..hi (descending), at
+    the widest log gap there; returns (tau, number of confidences above it)."""
+    c = np.sort(np.asarray(conf, np.float64))[::-1]
+    gaps = np.log(c[lo:hi]) - np.log(c[lo + 1:hi + 1])
+    i = lo + int(np.argmax(gaps))
+    return float(np.float32(math.sqrt(c[i] * c[i + 1]))), i + 1
+
+
+@pytest.mark.parametrize("name,layers", [("c1-tiny-dense", None), ("c2-small-moe", 2)])
+def test_threshold_branch_decides_the_commits(name, layers):
+    """tau is set between the step-0 confidences of the oracle's own pass, so that more
+    positions pass it than the step-budget floor asks for: the threshold itself decides
+    the commit set. Every step of the trace is replayed on the GPU and its commit set
+    compared wherever the log-confidence margin to tau and to the cut exceeds 1e-3."""
+    w = WORKLOADS[name]
+    cfg = w.model if layers is None else w.model.with_layers(layers)
+    C, S = cfg.canvas, 8
+    P = min(w.prefix, 512)
+    orc, den, _ = build_pair(cfg, P, w.prompt_seed + 3, P + 2 * C)
+    try:
+        conf0, _ = orc.denoise_pass(0, np.full(C, cfg.mask_id), np.ones(C, bool))
+        n_min = -(-C // S)
+        tau, n_above = _threshold_between(conf0, n_min + 2, C // 2)
+        assert n_above > n_min
+        pol = Policy("threshold", tau=tau, floor=True)
+        _, steps, trace = orc.generate_block(0, pol, S, trace=True)
+        assert int(trace[0]["commit"].sum()) == n_above
+        stats = compare_trace(cfg, trace, den, pol, S)
+        assert stats["commit_pinned"] >= 1
+        gpu_canvas, gpu_steps = check_generate_invariants(cfg, den, pol, S)
+    finally:
+        den.close()
+
+
+def _partial_canvas(cfg, seed):
+    """A canvas in mid-denoising: about 40% of the positions committed to seeded tokens."""
+    from synth import prompt_tokens, uniform_f32
+    C = cfg.canvas
+    committed = uniform_f32(seed, 1, C) > 0.2
+    tokens = prompt_tokens(cfg.vocab, seed, C).astype(np.int64)
+    mask = ~committed
+    return np.where(mask, cfg.mask_id, tokens), mask
+
+
+def _batched_parity(cfg, B, prompt_lens, step, s_max, seed0):
+    """One batched pass over B independent requests (own prompts, prefix lengths and
+    mid-denoising canvases) against the oracle run on each request alone: hidden state,
+    conf, argmax and the commit set of every request."""
+    import torch
+    from masked_block_diffusion_b200 import Denoiser, make_policy
+    from oracle import OracleModel, commit_select
+    from parity_util import MARGIN, REL, cached_weights, commit_margin
+    from synth import blob_from_weights, prompt_tokens
+
+    C = cfg.canvas
+    W = cached_weights(cfg)
+    orc = OracleModel(cfg, W, f64_matrices=cfg.d_model >= 2048)
+    den = Denoiser(cfg, blob_from_weights(cfg, W), max_ctx=max(prompt_lens) + C, max_batch=B)
+    pol = Policy("threshold", tau=0.9, floor=True)
+    refs = []
+    try:
+        den.set_debug(True)
+        for r in range(B):
+            p = prompt_tokens(cfg.vocab, seed0 + r, prompt_lens[r])
+            rec = {}
+            orc.prefill(r, p, rec)
+            den.force_routing(np.stack(rec["topk_idx"]))
+            den.prefill(r, p)
+            canvas, mask = _partial_canvas(cfg, seed0 + 500 + r)
+            rec = {}
+            conf, arg = orc.denoise_pass(r, canvas, mask, rec)
+            commit = commit_select(conf, mask, pol, step, s_max)
+            refs.append(dict(canvas=canvas, mask=mask, conf=conf, argmax=arg, commit=commit, rec=rec))
+        den.force_routing(np.concatenate([np.stack(e["rec"]["topk_idx"]) for e in refs], axis=1))
+        cv = torch.from_numpy(np.stack([e["canvas"] for e in refs]).astype(np.int32)).cuda()
+        mk = torch.from_numpy(np.stack([e["mask"] for e in refs]).astype(np.uint8)).cuda()
+        conf, arg, rem = den.denoise_step(cv, mk, make_policy("threshold", 0, 0.9, True), step, s_max)
+        x_gpu = den.debug_read(0, 0, (B * C, cfg.d_model), np.float32).astype(np.float64)
+        conf, arg, rem = conf.cpu().numpy(), arg.cpu().numpy(), rem.cpu().numpy()
+        new_mask = mk.cpu().numpy().astype(bool)
+        new_canvas = cv.cpu().numpy()
+        pinned_commits = 0
+        for r, e in enumerate(refs):
+            xr = e["rec"]["final_x"]
+            err = np.abs(x_gpu[r * C:(r + 1) * C] - xr).max(axis=1) / np.abs(xr).max(axis=1)
+            assert err.max() <= REL, f"request {r}: hidden rel err {err.max():.3g}"
+            assert np.all(np.abs(conf[r] / e["conf"] - 1.0) <= REL), f"request {r}: conf"
+            sel = e["rec"]["logit_margin"] > MARGIN
+            assert np.array_equal(arg[r][sel], e["argmax"][sel]), f"request {r}: argmax"
+            n = int(e["commit"].sum())
+            gpu_commit = e["mask"] & ~new_mask[r]
+            assert int(gpu_commit.sum()) == n and rem[r] == int(e["mask"].sum()) - n
+            if commit_margin(e["conf"], e["mask"], n, pol) > MARGIN:
+                assert np.array_equal(gpu_commit, e["commit"]), f"request {r}: commit set"
+                pinned_commits += 1
+            assert np.array_equal(new_canvas[r][gpu_commit], arg[r][gpu_commit])
+            assert np.array_equal(new_canvas[r][~e["mask"]], e["canvas"][~e["mask"]])
+        assert pinned_commits >= B // 2
+        den.force_routing(None)
+        den.set_debug(False)
+    finally:
+        den.close()
+
+
+def test_parity_batched_moe26b_eight_requests():
+    """Eight requests of the concurrency workload on the 26B model's layer shapes (two
+    layers), prompts of different lengths, in one batched pass."""
+    cfg = WORKLOADS["c5-moe26b-batch"].model.with_layers(2)
+    _batched_parity(cfg, 8, [256 + 40 * r for r in range(8)], step=3, s_max=12, seed0=2550)
+
+
+def test_parity_batched_small_moe_sixty_four_requests():
+    """64 requests in one pass (16,384 tokens, 65,536 expert assignments): the large
+    permute and the wider expert-chunk path, on the small MoE model's shapes."""
+    cfg = WORKLOADS["c2-small-moe"].model.with_layers(2)
+    _batched_parity(cfg, 64, [96 + 8 * (r % 16) for r in range(64)], step=5, s_max=12, seed0=2700)
+
+
+def _edit_tau_for(orc, cfg, trace):
+    """An edit threshold that the trace's committed positions straddle: the median
+    confidence of those whose argmax differs from their token, moved to the widest
+    nearby log gap."""
+    c = []
+    for e in trace[1:]:
+        committed = ~e["mask"]
+        diff = committed & (e["argmax"] != e["canvas"])
+        c.extend(e["conf"][diff].astype(np.float64).tolist())
+    c = np.sort(np.array(c))
+    assert c.size >= 8, "too few committed positions whose argmax differs"
+    lo, hi = c.size // 4, 3 * c.size // 4
+    gaps = np.log(c[lo + 1:hi + 1]) - np.log(c[lo:hi])
+    i = lo + int(np.argmax(gaps))
+    return float(np.float32(math.sqrt(c[i] * c[i + 1])))
+
+
+@pytest.mark.parametrize("name,layers", [("c1-tiny-dense", None), ("c2-small-moe", 2)])
+def test_t2t_editing_matches_the_oracle(name, layers):
+    """Token-to-token editing: committed positions whose argmax changes with confidence
+    above edit_tau are re-written. The threshold is chosen from the oracle's own M2T
+    trace so that edits happen; the T2T trace is then replayed step by step and the edit
+    sets compared wherever pinned."""
+    w = WORKLOADS[name]
+    cfg = w.model if layers is None else w.model.with_layers(layers)
+    C = cfg.canvas
+    S = 8
+    k = C // S
+    P = min(w.prefix, 512)
+    orc, den, _ = build_pair(cfg, P, w.prompt_seed + 5, P + 2 * C)
+    try:
+        _, _, m2t = orc.generate_block(0, Policy("topk", k=k), S, trace=True)
+        pol = Policy("topk", k=k, t2t=True, edit_tau=_edit_tau_for(orc, cfg, m2t))
+        _, steps, trace = orc.generate_block(0, pol, S, trace=True)
+        assert sum(int(e["edit"].sum()) for e in trace) > 0
+        stats = compare_trace(cfg, trace, den, pol, S)
+        assert stats["edit_pinned"] > 0
+        check_generate_invariants(cfg, den, pol, S, expect_steps=steps)
+    finally:
+        den.close()
+
+
+def test_approximate_append_matches_the_oracle():
+    """Two canvases with the approximate append between them (the last pass's K/V kept,
+    no append pass): every step of the second canvas is compared with the oracle doing
+    the same."""
+    import torch
+    w = WORKLOADS["c2-small-moe"]
+    cfg = w.model.with_layers(2)
+    C, S = cfg.canvas, w.max_steps
+    pol = Policy(w.policy, k=w.k)
+    orc, den, _ = build_pair(cfg, 512, w.prompt_seed + 9, 512 + 3 * C)
+    try:
+        from masked_block_diffusion_b200 import DllmError, binding
+        with pytest.raises(DllmError) as e:          # no canvas pass yet: nothing to keep
+            den.append_kv_approx(1)
+        assert e.value.code == binding.DLLM_E_STATE
+        _, _, trace1 = orc.generate_block(0, pol, S, trace=True)
+        compare_trace(cfg, trace1, den, pol, S)      # the GPU's last pass is the oracle's last
+        orc.append_approx(0)
+        den.append_kv_approx(1)
+        assert den.prefix_len(0) == 512 + C
+        _, _, trace2 = orc.generate_block(0, pol, S, trace=True)
+        stats = compare_trace(cfg, trace2, den, pol, S)
+        assert stats["steps"] == S
+    finally:
+        den.close()

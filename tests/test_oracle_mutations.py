@@ -255,6 +255,35 @@ def append_keeps_prefix_length(self, req, canvas):
     st.P = P
 
 
+def edit_select_masked_too(conf, argmax, canvas, mask, policy):   # edits masked positions as well
+    if not policy.t2t:
+        return np.zeros(np.asarray(mask).shape[0], dtype=bool)
+    return (np.asarray(argmax) != np.asarray(canvas)) & (np.asarray(conf, np.float32) > np.float32(policy.edit_tau))
+
+
+def edit_select_at_or_above(conf, argmax, canvas, mask, policy):   # conf >= edit_tau
+    if not policy.t2t:
+        return np.zeros(np.asarray(mask).shape[0], dtype=bool)
+    committed = ~np.asarray(mask, bool)
+    return committed & (np.asarray(argmax) != np.asarray(canvas)) & (
+        np.asarray(conf, np.float32) >= np.float32(policy.edit_tau))
+
+
+def edit_select_ignores_token(conf, argmax, canvas, mask, policy):   # re-writes even an equal token
+    if not policy.t2t:
+        return np.zeros(np.asarray(mask).shape[0], dtype=bool)
+    return ~np.asarray(mask, bool) & (np.asarray(conf, np.float32) > np.float32(policy.edit_tau))
+
+
+def append_approx_from_masked(self, req):   # K/V of the canvas as if every position were [MASK]
+    st = self.requests[req]
+    C = st.last_k[0].shape[0]
+    _, ks, vs = om.OracleModel.__dict__["_canvas_forward"](self, req, np.full(C, self.cfg.mask_id),
+                                                          np.ones(C, bool))
+    st.last_k, st.last_v = ks, vs
+    om.OracleModel.__dict__["_orig_append_approx"](self, req)
+
+
 # ---------------------------------------------------------------- which pins guard what
 
 P = pins
@@ -296,6 +325,11 @@ CASES = [
      [lambda: P.test_cached_passes_equal_block_causal_sequence(P.MICRO)]),
     ("OracleModel.append", append_keeps_prefix_length,
      [lambda: P.test_cached_passes_equal_block_causal_sequence(P.MICRO_DENSE)]),
+    ("edit_select", edit_select_masked_too, [P.test_edit_select_rule]),
+    ("edit_select", edit_select_at_or_above, [P.test_edit_select_rule]),
+    ("edit_select", edit_select_ignores_token, [P.test_edit_select_rule, P.test_generate_block_t2t_invariants]),
+    ("OracleModel.append_approx", append_approx_from_masked,
+     [lambda: P.test_approximate_append_equals_exact_append_on_a_finished_pass(P.MICRO)]),
 ]
 
 

@@ -374,3 +374,73 @@ def test_threshold_is_strictly_above_tau():
     conf = np.array([0.9, 0.95, 0.1], np.float32)
     sel = commit_select(conf, np.ones(3, bool), Policy("threshold", tau=0.9, floor=False), 0, 48)
     assert list(np.nonzero(sel)[0]) == [1]
+
+
+# ---------------------------------------------------------------- T2T editing and approximate append
+
+def test_edit_select_rule():
+    M = 63
+    canvas = np.array([5, 7, M, 3, 9])
+    mask = np.array([0, 0, 1, 0, 0], bool)
+    argmax = np.array([5, 8, 9, 4, 2])
+    conf = np.array([0.95, 0.95, 0.99, 0.5, 0.9], np.float32)
+    on = Policy("topk", k=1, t2t=True, edit_tau=0.9)
+    # 0: same token; 1: edited; 2: masked (the commit's business); 3: below tau;
+    # 4: exactly at tau (not above)
+    assert list(oracle.edit_select(conf, argmax, canvas, mask, on)) == [False, True, False, False, False]
+    assert not oracle.edit_select(conf, argmax, canvas, mask, Policy("topk", k=1)).any()
+
+
+def test_generate_block_t2t_invariants():
+    cfg = MICRO
+    m = OracleModel(cfg, gen_weights(cfg))
+    m.prefill(0, prompt_tokens(cfg.vocab, 2000, 12))
+    pol = Policy("topk", k=2, t2t=True, edit_tau=0.02)
+    canvas, steps, tr = m.generate_block(0, pol, 4, trace=True)
+    assert steps == 4 and not np.any(canvas == cfg.mask_id)
+    edits = 0
+    prev_R = cfg.canvas
+    for e in tr:
+        assert int(e["mask"].sum()) == prev_R
+        nxt = canvas if e is tr[-1] else tr[tr.index(e) + 1]["canvas"]
+        committed = ~e["mask"]
+        changed = committed & (nxt != e["canvas"])
+        # a committed position changes only to the pass's argmax, with conf above edit_tau
+        assert np.array_equal(changed, e["edit"])
+        assert np.all(nxt[changed] == e["argmax"][changed])
+        assert np.all(e["conf"][changed] > np.float32(pol.edit_tau))
+        assert not np.any(nxt[committed] == cfg.mask_id)        # no mask comes back
+        assert e["commit"].sum() == min(pol.k, prev_R)          # the commit count is unchanged
+        edits += int(changed.sum())
+        prev_R = e["remaining"]
+    assert edits > 0
+
+
+@pytest.mark.parametrize("cfg", [MICRO, MICRO_DENSE])
+def test_approximate_append_equals_exact_append_on_a_finished_pass(cfg):
+    """When the last denoising pass already saw the finished canvas (nothing masked),
+    its K/V are exactly what the append pass computes: the approximate and exact caches
+    agree. In general they differ by what the last commit changed."""
+    W = gen_weights(cfg)
+    a, b = OracleModel(cfg, W), OracleModel(cfg, W)
+    p = prompt_tokens(cfg.vocab, 2005, 10)
+    a.prefill(0, p)
+    b.prefill(0, p)
+    fin = prompt_tokens(cfg.vocab, 2006, cfg.canvas).astype(np.int64)
+    a.denoise_pass(0, fin, np.zeros(cfg.canvas, bool))
+    a.append_approx(0)
+    b.append(0, fin)
+    assert a.requests[0].P == b.requests[0].P == 10 + cfg.canvas
+    for l in range(cfg.n_layers):
+        assert np.array_equal(a.requests[0].k[l], b.requests[0].k[l])
+        assert np.array_equal(a.requests[0].v[l], b.requests[0].v[l])
+    # after a pass with masked positions, the approximate cache is not the exact one
+    a2, b2 = OracleModel(cfg, W), OracleModel(cfg, W)
+    a2.prefill(0, p)
+    b2.prefill(0, p)
+    mask = np.zeros(cfg.canvas, bool)
+    mask[::2] = True
+    a2.denoise_pass(0, np.where(mask, cfg.mask_id, fin), mask)
+    a2.append_approx(0)
+    b2.append(0, fin)
+    assert not np.array_equal(a2.requests[0].k[0][10:], b2.requests[0].k[0][10:])
