@@ -67,6 +67,10 @@ def parse_args():
     ap.add_argument("--routing", choices=["model", "uniform"], default="model",
                     help="uniform: every canvas token routed evenly over all experts (design point)")
     ap.add_argument("--sweep", action="store_true", help="concurrency sweep B = 1, 4, 8, 16, 32, 64")
+    ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: expert weights as FP8 E4M3 with power-of-two 128x128 tile scales")
+    ap.add_argument("--append", choices=["exact", "approx"], default="exact",
+                    help="approx: keep the last denoising pass's K/V instead of an append pass")
     ap.add_argument("--ingest-ncu", default="", help="ncu CSV of the gate/up GEMM launches to record")
     return ap.parse_args()
 
@@ -358,7 +362,8 @@ class Arm:
         self.args, self.w, self.cfg, self.binding = args, w, w.model, binding
         C = w.model.canvas
         blob = device_blob(w.model)
-        self.den = Denoiser(w.model, blob, max_ctx=w.prefix + w.n_canvases * C, max_batch=max_batch)
+        self.den = Denoiser(w.model, blob, max_ctx=w.prefix + w.n_canvases * C, max_batch=max_batch,
+                            expert_fp8=args.experts == "fp8")
         del blob
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
@@ -391,7 +396,10 @@ class Arm:
                 e1.record(self.st)
                 gen_events.append((e0, e1))
             passes += max(steps)
-            b.dllm_append_kv(h, B, 0)
+            if self.args.append == "approx":
+                b.dllm_append_kv_approx(h, B)
+            else:
+                b.dllm_append_kv(h, B, 0)
         return passes
 
     def timed(self, B, steps, world):
@@ -476,13 +484,15 @@ def run_ours(args):
     achieved = kbytes[GU] / (kms[GU] / 1e3) / 1e9
     peak_hbm = float(peaks["hbm_gbs"])
     act = Bq * C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 2
-    routed = (gu_bytes - act) / (2 * cfg.ffn_dim * cfg.d_model * 2)
+    wbytes = 1 if args.experts == "fp8" else 2
+    routed = (gu_bytes - act) / (2 * cfg.ffn_dim * cfg.d_model * wbytes)
     traffic = recorded_traffic(w.name, args.routing)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_hbm, "unit": "GB/s",
                 "frac": round(achieved / peak_hbm, 4), "traffic": round(traffic) if traffic else None,
                 "kernel": "grouped expert gate/up GEMM + SwiGLU (tcgen05, one launch per layer)",
                 "bytes_per_launch": round(gu_bytes),
-                "bytes_per_launch_all_experts": gate_up_bytes(cfg, C * Bq),
+                "bytes_per_launch_all_experts": gate_up_bytes(cfg, C * Bq) // (2 // wbytes) if wbytes == 2
+                else gate_up_bytes(cfg, C * Bq) - cfg.n_experts * 2 * cfg.ffn_dim * cfg.d_model,
                 "bytes_note": ("algorithmic: bf16 weights of the experts each launch routed to + token rows in "
                                "+ SwiGLU rows out at bf16 size; the kernel's (hi, lo) activation pairs are "
                                "overhead, not work"),
@@ -526,6 +536,11 @@ def run_ours(args):
         "timing_layer_stride": TIMING_STRIDE,
         "clocks": clk,
     }
+    if args.experts == "fp8":
+        out["dtype"] = "bf16 (expert weights fp8 e4m3, power-of-two 128x128 tile scales)"
+        out["roofline"]["bytes_note"] += "; FP8 experts: weight bytes are 1 per element"
+    if args.append == "approx":
+        out["append"] = "approximate: the last denoising pass's K/V kept, no append pass"
     if args.routing == "uniform":
         out["routing"] = ("design point: every canvas token routed to k experts so that all experts get "
                           "T k / E tokens (forced through the debug routing hook; debug copies of the router "

@@ -60,6 +60,9 @@ extern "C" {
 #define DLLM_WEIGHTS_F32 0
 #define DLLM_WEIGHTS_BF16 1
 
+#define DLLM_EXPERTS_BF16 0
+#define DLLM_EXPERTS_FP8 1
+
 #define DLLM_POLICY_TOPK 0
 #define DLLM_POLICY_THRESHOLD 1
 
@@ -78,6 +81,13 @@ typedef struct {
   float rms_eps;   /* 1e-6 */
   float rope_theta;/* 10000 */
   int weight_dtype;/* DLLM_WEIGHTS_F32 or DLLM_WEIGHTS_BF16 */
+  /* DLLM_EXPERTS_BF16 (0): expert weights as given. DLLM_EXPERTS_FP8 (1): at create, every
+   * expert matrix (Wg, Wu, Wd) is stored as FP8 E4M3 with one power-of-two scale 2^e per
+   * 128 x 128 tile of the matrix, e the least integer with the tile's max |w| <= 448 * 2^e,
+   * codes rounded to nearest even (What changes, section 4.2 "Speed": the measured setting
+   * runs FP8). The kernels expand each staged tile to bf16 exactly, so the pass computes on
+   * the FP8 values; expert bytes per pass halve. Needs ffn_dim and d_model multiples of 128. */
+  int expert_format;
 } dllm_config;
 
 /* Commit policy (What changes, section 2 and section 5).
@@ -241,6 +251,13 @@ void dllm_destroy(dllm_handle* h);
 /* D[M][N] (fp32, row-major) = A[M][K] * B[N][K]^T with bf16 A, B; the tcgen05 GEMM core.
  * K % 64 == 0, N % 128 == 0. */
 int dllm_op_gemm_bf16(const uint16_t* A, const uint16_t* B, float* D, int M, int N, int K, void* stream);
+
+/* The FP8 block quantiser that dllm_create applies to expert matrices with
+ * DLLM_EXPERTS_FP8: w (bf16 [rows][cols], row-major) -> q (E4M3 codes [rows][cols]) and
+ * exps (int8 [ceil(rows/128)][ceil(cols/128)]): per 128 x 128 tile, e = the least integer
+ * with max |w| <= 448 * 2^e (0 for an all-zero tile), q = nearest E4M3 (ties to even) of
+ * w * 2^-e. cols % 16 == 0. */
+int dllm_op_quantize_fp8(const uint16_t* w, int rows, int cols, uint8_t* q, int8_t* exps, void* stream);
 
 /* The fused LM head (What changes, section 2: commit the most confident positions):
  * for each of the T rows of y (bf16 [T][d]) against head (bf16 [V][d]), argmax over

@@ -25,14 +25,14 @@ class Denoiser:
     tensors synchronise the handle's stream first, so results are ready to use.
     """
 
-    def __init__(self, model, weights, max_ctx: int, max_batch: int = 1):
+    def __init__(self, model, weights, max_ctx: int, max_batch: int = 1, expert_fp8: bool = False):
         import torch
         self.torch = torch
         self.model = model
         self.C = model.canvas
         self.max_batch = max_batch
         self.stream = torch.cuda.Stream()
-        self.cfg = make_config(model, max_ctx, max_batch)
+        self.cfg = make_config(model, max_ctx, max_batch, expert_fp8)
         if isinstance(weights, np.ndarray):
             buf = np.ascontiguousarray(weights)
             ptr, nbytes, on_dev = buf.ctypes.data, buf.nbytes, False

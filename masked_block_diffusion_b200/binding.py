@@ -27,6 +27,8 @@ ERROR_NAMES = {0: "DLLM_OK", -1: "DLLM_E_INVAL", -2: "DLLM_E_OOM", -3: "DLLM_E_C
 
 DLLM_WEIGHTS_F32 = 0
 DLLM_WEIGHTS_BF16 = 1
+DLLM_EXPERTS_BF16 = 0
+DLLM_EXPERTS_FP8 = 1
 DLLM_POLICY_TOPK = 0
 DLLM_POLICY_THRESHOLD = 1
 
@@ -36,7 +38,7 @@ EXPORTS = [
     "dllm_generate", "dllm_reset", "dllm_prefix_len", "dllm_check", "dllm_launch_count",
     "dllm_set_debug", "dllm_debug_read", "dllm_debug_force_routing", "dllm_last_error", "dllm_destroy",
     "dllm_op_gemm_bf16", "dllm_op_lm_head_conf", "dllm_op_lm_head_conf_noalloc", "dllm_set_timing",
-    "dllm_timing_read", "dllm_set_wait_limit", "dllm_append_kv_approx",
+    "dllm_timing_read", "dllm_set_wait_limit", "dllm_append_kv_approx", "dllm_op_quantize_fp8",
 ]
 DLLM_TIMING_GATE_UP = 0
 DLLM_TIMING_DOWN = 1
@@ -59,7 +61,7 @@ class dllm_config(ctypes.Structure):
         ("top_k", ctypes.c_int), ("ffn_dim", ctypes.c_int), ("vocab", ctypes.c_int),
         ("mask_id", ctypes.c_int), ("canvas", ctypes.c_int), ("max_ctx", ctypes.c_int),
         ("max_batch", ctypes.c_int), ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
-        ("weight_dtype", ctypes.c_int),
+        ("weight_dtype", ctypes.c_int), ("expert_format", ctypes.c_int),
     ]
 
 
@@ -111,6 +113,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dllm_timing_read": (_i, [_vp, _vp, _vp, _vp, _i]),
         "dllm_set_wait_limit": (_i, [_vp, ctypes.c_longlong]),
         "dllm_append_kv_approx": (_i, [_vp, _i]),
+        "dllm_op_quantize_fp8": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -120,9 +123,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-def make_config(model, max_ctx: int, max_batch: int) -> dllm_config:
+def make_config(model, max_ctx: int, max_batch: int, expert_fp8: bool = False) -> dllm_config:
     """dllm_config from a model description with the fields of synth.ModelConfig."""
     return dllm_config(
+        expert_format=DLLM_EXPERTS_FP8 if expert_fp8 else DLLM_EXPERTS_BF16,
         n_layers=model.n_layers, d_model=model.d_model, n_heads=model.n_heads,
         n_kv_heads=model.n_kv_heads, head_dim=model.head_dim, n_experts=model.n_experts,
         top_k=model.top_k, ffn_dim=model.ffn_dim, vocab=model.vocab, mask_id=model.vocab - 1,
@@ -258,3 +262,9 @@ def dllm_op_lm_head_conf_noalloc(y_ptr, head_ptr, T, d, V, mask_id, conf_ptr, ar
 def dllm_set_wait_limit(h, ns: int):
     """Pipeline-wait limit of the kernels on this device in ns (<= 0: the 2 s default)."""
     _check(load().dllm_set_wait_limit(h, int(ns)), "dllm_set_wait_limit", h)
+
+
+def dllm_op_quantize_fp8(w_ptr, rows, cols, q_ptr, exps_ptr, stream_ptr):
+    """FP8 E4M3 codes and per-128x128-tile scale exponents of a bf16 matrix (device buffers)."""
+    _check(load().dllm_op_quantize_fp8(_vp(w_ptr), rows, cols, _vp(q_ptr), _vp(exps_ptr), _vp(stream_ptr)),
+           "dllm_op_quantize_fp8")

@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #define DLLM_DEV __device__ __forceinline__
@@ -52,6 +54,21 @@ DLLM_DEV void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
 }
 
 DLLM_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// ---------------------------------------------------------------- FP8 E4M3
+
+// Nearest E4M3 code of x (ties to even; |x| <= 448 here, so saturation never acts).
+DLLM_DEV uint8_t f32_to_e4m3(float x) {
+  return (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Two E4M3 codes (low byte first) times 2^e as a bf16 pair (low half first). Exact: an
+// E4M3 value has 4 significant bits and the scale is a power of two.
+DLLM_DEV uint32_t e4m3x2_to_bf16x2(uint16_t two, float scale) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x * scale, f.y * scale);
+}
 
 DLLM_DEV unsigned long long global_ns() {
   unsigned long long t;
@@ -324,6 +341,9 @@ DLLM_DEV void tmem_st32_nowait(uint32_t taddr, const uint32_t (&v)[32]) {
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
+
+// Tensor-memory address of row `lane_row` (a multiple of 32) at column `col`.
+DLLM_DEV uint32_t tmem_at(uint32_t base, int lane_row, int col) { return base + ((uint32_t)lane_row << 16) + col; }
 
 // 16 consecutive 32-bit TMEM columns of this thread's lane (no wait).
 DLLM_DEV void tmem_st16_nowait(uint32_t taddr, const uint32_t (&v)[16]) {

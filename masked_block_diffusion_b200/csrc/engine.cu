@@ -81,6 +81,21 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, ui
 // Token-operand boxes of the grouped expert GEMMs: a chunk of up to kMoeChunk tokens is
 // loaded from boxes of these heights (its count rounded up to 16), so the MMA width
 // follows the chunk's token count.
+// 2-D uint8 tensor map over [rows][cols] FP8 codes, box = 64 columns x box_rows, 64-byte
+// swizzle (the converter warps read each row's four 16-byte chunks at chunk ^ ((row >> 1) & 3)).
+bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || cols % 16 || box_rows == 0 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr int kMoeBN[4] = {16, 32, 64, 128};
 constexpr int kMoeChunk = 128;
 
@@ -92,7 +107,14 @@ struct LayerW {
   bf16_t* wr = nullptr;     // [E][d]
   bf16_t* wgu = nullptr;    // [E][2F][d]: per 128-row block, 64 gate rows then the 64 matching up rows
   bf16_t* wd = nullptr;     // [E][d][F]
-  CUtensorMap tm_wqkv, tm_wo, tm_wo128, tm_wgu, tm_wd, tm_wr;
+  // FP8 experts (expert_format = DLLM_EXPERTS_FP8): the same layouts as E4M3 codes, and the
+  // scale exponents of each 128 x 128 tile of the original Wg / Wu ([E][2][F/128][d/128])
+  // and Wd ([E][d/128][F/128]), tile counts rounded up
+  uint8_t* wgu8 = nullptr;
+  uint8_t* wd8 = nullptr;
+  int8_t* egu = nullptr;
+  int8_t* ed = nullptr;
+  CUtensorMap tm_wqkv, tm_wo, tm_wo128, tm_wgu, tm_wd, tm_wr, tm_wgu8, tm_wd8;
   CUtensorMap tm_k, tm_v;   // this layer's K / V cache as [slot][Hkv][max_ctx] rows of hd
 };
 
@@ -167,6 +189,7 @@ struct dllm_handle {
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
   int router_ks = 8;        // largest K split of the router GEMM
   bool pdl = true;          // programmatic dependent launch between the kernels of a pass
+  bool w8 = false;          // FP8 expert weights
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
   std::vector<char> passed;  // per slot: a canvas pass wrote K/V at P..P+C-1 since the last prefill / append
@@ -313,7 +336,7 @@ cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const 
     // split-K: clusters of kKSplit consecutive CTAs share one output tile
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(gemm_threads<Sched>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = h->st;
     cudaLaunchAttribute at[2];
@@ -331,8 +354,8 @@ cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const 
     if (r != cudaSuccess) return r;
     return cudaGetLastError();
   }
-  r = launch_k(h, kern, grid, dim3(192), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e,
-               h->d_err);
+  r = launch_k(h, kern, grid, dim3(gemm_threads<Sched>()), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks,
+               a_first, s, e, h->d_err);
   h->launches++;
   if (r != cudaSuccess) return r;
   return cudaGetLastError();
@@ -553,17 +576,43 @@ cudaError_t moe_down(dllm_handle* h, const LayerW& L) {
                                                &h->tm_h_lo[3]);
 }
 
+// The FP8-weight variants: one weight tile per item and one accumulator, the rest of
+// tensor memory holding the converted bf16 A stages.
+cudaError_t moe_gate_up_w8(dllm_handle* h, const LayerW& L) {
+  const auto& c = h->c;
+  const int F = c.ffn_dim, d = c.d_model;
+  constexpr int BN = kMoeChunk;
+  constexpr int STAGES = 4;
+  PersistentGroupedSched<1, true> s{h->d_tok_maps, h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F,
+                                    2 * F / 128, BN, L.egu, 1, (F + 127) / 128, (d + 127) / 128};
+  EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
+  return launch_gemm<BN, STAGES, 1, kSplitB>(h, dim3(h->num_sms), L.tm_wgu8, h->tm_xg[3], d / 64, 1, s, e, nullptr,
+                                             &h->tm_xg_lo[3]);
+}
+
+cudaError_t moe_down_w8(dllm_handle* h, const LayerW& L) {
+  const auto& c = h->c;
+  const int F = c.ffn_dim, d = c.d_model;
+  constexpr int BN = kMoeChunk;
+  constexpr int STAGES = 4;
+  PersistentGroupedSched<1, true> s{h->d_tok_maps + 8, h->offsets, h->routed, h->n_routed, h->chunk_prefix, d,
+                                    d / 128, BN, L.ed, 0, d / 128, (F + 127) / 128};
+  EpiDown<BN> e{h->obuf, d};
+  return launch_gemm<BN, STAGES, 1, kSplitB>(h, dim3(h->num_sms), L.tm_wd8, h->tm_h[3], F / 64, 1, s, e, nullptr,
+                                             &h->tm_h_lo[3]);
+}
+
 // Grouped expert GEMMs of one layer. gate/up: one weight tile per item, two accumulator
 // buffers; down: two weight tiles per item sharing the token chunk (its 22 m tiles leave
 // enough items to spread over the SMs), or one with DLLM_MOE_PAIR=0.
 cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int l, uint32_t timed) {
   cudaError_t r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-  r = moe_gate_up<1, 2>(h, L);
+  r = h->w8 ? moe_gate_up_w8(h, L) : moe_gate_up<1, 2>(h, L);
   if (r != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  r = h->moe_pair ? moe_down<2, 1>(h, L) : moe_down<1, 2>(h, L);
+  r = h->w8 ? moe_down_w8(h, L) : h->moe_pair ? moe_down<2, 1>(h, L) : moe_down<1, 2>(h, L);
   if (r != cudaSuccess) return r;
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
@@ -782,8 +831,9 @@ void accumulate_timing(dllm_handle* h, int T) {
       h->t_n[kind] += 1;
       // the method's bytes: the routed experts' bf16 weights, the bf16 token rows in and
       // the bf16 results out (the (hi, lo) pairs and fp32 outputs are the kernels' own)
-      if (kind == DLLM_TIMING_GATE_UP) h->t_bytes[kind] += nr[l] * 2 * F * d * 2 + N * d * 2 + N * F * 2;
-      if (kind == DLLM_TIMING_DOWN) h->t_bytes[kind] += nr[l] * d * F * 2 + N * F * 2 + N * d * 2;
+      const double wb = h->w8 ? 1.0 : 2.0;   // weight bytes per element (FP8 or bf16)
+      if (kind == DLLM_TIMING_GATE_UP) h->t_bytes[kind] += nr[l] * 2 * F * d * wb + N * d * 2 + N * F * 2;
+      if (kind == DLLM_TIMING_DOWN) h->t_bytes[kind] += nr[l] * d * F * wb + N * F * 2 + N * d * 2;
     }
   }
 }
@@ -810,6 +860,9 @@ int validate(const dllm_config* c, std::string* why) {
   if (c->canvas < 1 || c->canvas > 1024) return bad("canvas in [1, 1024]");
   if (c->max_batch < 1 || c->max_ctx < c->canvas + 1) return bad("max_batch >= 1 and max_ctx > canvas");
   if (c->weight_dtype != DLLM_WEIGHTS_F32 && c->weight_dtype != DLLM_WEIGHTS_BF16) return bad("weight_dtype");
+  if (c->expert_format != DLLM_EXPERTS_BF16 && c->expert_format != DLLM_EXPERTS_FP8) return bad("expert_format");
+  if (c->expert_format == DLLM_EXPERTS_FP8 && c->n_experts > 0 && (c->ffn_dim % 128 || c->d_model % 128))
+    return bad("FP8 experts need ffn_dim and d_model multiples of 128");
   return DLLM_OK;
 }
 
@@ -888,6 +941,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
   if (const char* m = getenv("DLLM_ROUTER_KS")) h->router_ks = atoi(m);
+  h->w8 = !h->dense && c.expert_format == DLLM_EXPERTS_FP8;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
   // ---- weights
@@ -901,9 +955,20 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     DA(L.wqkv, (size_t)(qd + 2 * kvd) * d);
     DA(L.wo, (size_t)d * qd);
     if (!h->dense) DA(L.wr, (size_t)h->E * d);
-    DA(L.wgu, (size_t)h->E * 2 * F * d);
-    DA(L.wd, (size_t)h->E * d * F);
+    if (h->w8) {
+      DA(L.wgu8, (size_t)h->E * 2 * F * d);
+      DA(L.wd8, (size_t)h->E * d * F);
+      DA(L.egu, (size_t)h->E * 2 * ((F + 127) / 128) * ((d + 127) / 128));
+      DA(L.ed, (size_t)h->E * (d / 128) * ((F + 127) / 128));
+    } else {
+      DA(L.wgu, (size_t)h->E * 2 * F * d);
+      DA(L.wd, (size_t)h->E * d * F);
+    }
   }
+  // FP8 experts: each expert matrix is unpacked to bf16 here (original layout), then
+  // quantised into its packed FP8 place
+  bf16_t* w8_src = nullptr;
+  if (h->w8) DA(w8_src, (size_t)F * d);
   uint8_t* staging = nullptr;
   if (!on_device) {
     const size_t sizes[] = {(size_t)V * d, (size_t)qd * d, (size_t)kvd * d, (size_t)F * d, (size_t)h->E * d};
@@ -928,6 +993,18 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
       if ((r = pack_tensor(h, br, staging, L.wr, h->E, d, BIG, 0, 0))) return r;
     for (int e = 0; e < h->E; ++e) {
       const long gu0 = (long)e * 2 * F;
+      if (h->w8) {
+        const int nrbF = (F + 127) / 128, ncbD = (d + 127) / 128, nrbD = d / 128, ncbF = (F + 127) / 128;
+        for (int which = 0; which < 2; ++which) {   // gate rows, then up rows
+          if ((r = pack_tensor(h, br, staging, w8_src, F, d, BIG, 0, 0))) return r;
+          CK(launch_k(h, quantize_e4m3_blocks_kernel, dim3(ncbD, nrbF), dim3(256), 0, w8_src, F, d, L.wgu8,
+                      L.egu + (size_t)(e * 2 + which) * nrbF * ncbD, 64L, 128L, gu0 + 64 * which));
+        }
+        if ((r = pack_tensor(h, br, staging, w8_src, d, F, BIG, 0, 0))) return r;
+        CK(launch_k(h, quantize_e4m3_blocks_kernel, dim3(ncbF, nrbD), dim3(256), 0, w8_src, d, F, L.wd8,
+                    L.ed + (size_t)e * nrbD * ncbF, BIG, 0L, (long)e * d));
+        continue;
+      }
       if ((r = pack_tensor(h, br, staging, L.wgu, F, d, 64, 128, gu0))) return r;        // gate rows
       if ((r = pack_tensor(h, br, staging, L.wgu, F, d, 64, 128, gu0 + 64))) return r;   // up rows
       if ((r = pack_tensor(h, br, staging, L.wd, d, F, BIG, 0, (long)e * d))) return r;
@@ -1054,8 +1131,13 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     ok &= make_tmap(&L.tm_wo, L.wo, d, qd, 64);
     ok &= make_tmap(&L.tm_wo128, L.wo, d, qd, 128);
     if (h->router_tc) ok &= make_tmap(&L.tm_wr, L.wr, h->E, d, 32);
-    ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
-    ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);
+    if (h->w8) {
+      ok &= make_tmap_u8(&L.tm_wgu8, L.wgu8, (uint64_t)h->E * 2 * F, d, 128);
+      ok &= make_tmap_u8(&L.tm_wd8, L.wd8, (uint64_t)h->E * d, F, 128);
+    } else {
+      ok &= make_tmap(&L.tm_wgu, L.wgu, (uint64_t)h->E * 2 * F, d, 128);
+      ok &= make_tmap(&L.tm_wd, L.wd, (uint64_t)h->E * d, F, 128);
+    }
     if (h->attn_tc) {
       const size_t l = &L - h->L.data();
       const uint64_t kv_rows = (uint64_t)c.max_batch * Hkv * c.max_ctx;
@@ -1466,6 +1548,14 @@ int dllm_op_lm_head_conf(const uint16_t* y, const uint16_t* head, int T, int d, 
   cudaFreeAsync(err, tmp.st);
   tmp.d_err = nullptr;
   return r == cudaSuccess ? DLLM_OK : DLLM_E_CUDA;
+}
+
+int dllm_op_quantize_fp8(const uint16_t* w, int rows, int cols, uint8_t* q, int8_t* exps, void* stream) {
+  if (!w || !q || !exps || rows < 1 || cols < 16 || cols % 16) return DLLM_E_INVAL;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  quantize_e4m3_blocks_kernel<<<dim3((cols + 127) / 128, (rows + 127) / 128), 256, 0, st>>>(
+      w, rows, cols, q, exps, 1L << 40, 0L, 0L);
+  return cudaGetLastError() == cudaSuccess ? DLLM_OK : DLLM_E_CUDA;
 }
 
 }  // extern "C"

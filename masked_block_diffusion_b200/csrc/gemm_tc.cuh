@@ -35,6 +35,7 @@ struct DenseSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = 1;
   static constexpr bool kDynN = false;
+  static constexpr bool kW8 = false;
   static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
@@ -61,6 +62,7 @@ struct DenseSplitKSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = KS;
   static constexpr bool kDynN = false;
+  static constexpr bool kW8 = false;
   static constexpr int kMPerItem = 1;
   int M, n_mtiles, BN;
   DLLM_DEV void stage(int*) {}
@@ -97,12 +99,20 @@ struct DenseSplitKSched {
 // and 16 rows (tok_maps: [hi 16, 32, 64, 128 | lo 16, 32, 64, 128], tensor maps in
 // global memory), stacked as [hi n16 rows | lo n16 rows], and one MMA of N = 2 n16 reads
 // both. An expert with few tokens then costs its weight bytes and little else.
-template <int MPI>
+//
+// W8: the weights are FP8 E4M3 with one power-of-two scale 2^e per 128 x 128 tile of
+// each original expert matrix (exps, int8). Converter warps turn each staged FP8 tile
+// into bf16 (exact) straight into tensor memory, where the MMA reads its A operand, so
+// the bf16 copy never touches shared memory. exp_interleave = 1 for the gate/up layout
+// (each 128-row tile: 64 gate rows, then the matching 64 up rows), 0 for down; exps is
+// [E][2 if interleaved][exp_nrb][exp_ncb].
+template <int MPI, bool W8 = false>
 struct PersistentGroupedSched {
   static constexpr int kMaxRouted = 256;
   static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
   static constexpr int kKSplit = 1;
   static constexpr bool kDynN = true;
+  static constexpr bool kW8 = W8;
   static constexpr int kMPerItem = MPI;
   const CUtensorMap* tok_maps;   // 8 token-operand maps (see above), device memory
   const int* offsets;        // [E+1] token ranges per expert
@@ -112,6 +122,15 @@ struct PersistentGroupedSched {
   int rows_per_expert;
   int m_tiles;
   int BN;
+  const int8_t* exps = nullptr;
+  int exp_interleave = 0, exp_nrb = 0, exp_ncb = 0;
+  // scale exponent of row r of m tile u of tile t at k block kb (64 columns)
+  DLLM_DEV int exponent(const Tile& t, int u, int r, int kb) const {
+    const int mt = t.mt + u;
+    const int cb = kb >> 1;
+    if (exp_interleave) return exps[((t.nt * 2 + (r >> 6)) * exp_nrb + (mt >> 1)) * exp_ncb + cb];
+    return exps[(t.nt * exp_nrb + mt) * exp_ncb + cb];
+  }
   // shared-memory copies, per routed expert r: token offset and count (set by stage())
   const int* s_off = nullptr;
   const int* s_cnt = nullptr;
@@ -176,6 +195,15 @@ __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
 }
 
+// tcgen05.alloc takes a power of two of at least 32 columns.
+__host__ __device__ constexpr int tmem_alloc_cols(int n) {
+  return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
+}
+
+// Threads of a GEMM CTA: producer, MMA, 4 epilogue warps, and for W8 4 converter warps.
+template <class Sched>
+__host__ __device__ constexpr int gemm_threads() { return Sched::kW8 ? 320 : 192; }
+
 // Operand splitting. Weights are bf16; an activation operand can be carried as a pair
 // of bf16 tensors (hi = bf16(v), lo = bf16(v - hi)) so that products keep about 16
 // mantissa bits of the activation. kSplitNone: plain. kSplitA: A is a (hi, lo) pair and
@@ -186,7 +214,8 @@ enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
 
 template <int BN, int STAGES, int SPLIT, class Epi, class Sched = DenseSched>
 struct GemmSmem {
-  static constexpr int kAtile = 128 * 64 * 2;              // one 128-row A tile of a k block
+  // one 128-row A tile of a k block: bf16, or FP8 bytes for a W8 schedule
+  static constexpr int kAtile = Sched::kW8 ? 128 * 64 : 128 * 64 * 2;
   static constexpr int kA = Sched::kMPerItem * kAtile;     // the item's A tiles
   static constexpr int kB = BN * 64 * 2;
   static constexpr int kA2 = SPLIT == kSplitA ? kA : 0;
@@ -280,7 +309,7 @@ DLLM_DEV bool splitk_reduce(int krank, uint32_t taddr, int r, uint8_t* part_smem
 }
 
 template <int BN, int STAGES, int ACC_BUFS, int SPLIT, class Sched, class Epi>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(gemm_threads<Sched>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a2,
                const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_b2,
                int k_blocks, int a_stream_first, Sched sched_in, Epi epi, int* err) {
@@ -291,8 +320,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   constexpr int MPI = Sched::kMPerItem;                   // accumulators per work item
   static_assert(MPI == 1 || SPLIT != kSplitA, "several m tiles per item share B only");
   constexpr int kCols = tmem_cols_for(kAccN);
-  constexpr int kTmemCols = kCols * ACC_BUFS * MPI;
-  static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+  constexpr bool W8 = Sched::kW8;
+  static_assert(!W8 || (SPLIT == kSplitB && Sched::kDynN), "FP8 weights: grouped expert tiles only");
+  constexpr int kAccCols = kCols * ACC_BUFS * MPI;
+  constexpr int kACol = kAccCols;                        // W8: bf16 A stages, 32 columns per tile
+  constexpr int kTmemCols = tmem_alloc_cols(kAccCols + (W8 ? STAGES * MPI * 32 : 0));
+  static_assert(kAccCols + (W8 ? STAGES * MPI * 32 : 0) <= 512, "TMEM has 512 columns");
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, kAccN);
   constexpr int KS = Sched::kKSplit;
   static_assert(KS == 1 || BN * 128 * 4 <= STAGES * L::kStageBytes, "split-K partial fits the stage buffers");
@@ -309,7 +342,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   uint64_t* acc_empty = acc_full + ACC_BUFS;
   uint64_t* drain = acc_empty + ACC_BUFS;
   uint64_t* peer_ready = drain + 1;   // split-K: rank 0 learns that the peers' partials are in place
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* conv_full = drain + 2;    // W8: the stage's bf16 A tiles are in tensor memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv_full + (W8 ? STAGES : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* epi_smem = smem + L::kEpiOff;
   Sched sched = sched_in;
@@ -328,6 +362,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     }
     mbar_init(drain, 1);
     if (KS > 1) mbar_init(peer_ready, 128 * (KS - 1));
+    if (W8)
+      for (int s = 0; s < STAGES; ++s) mbar_init(&conv_full[s], 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tma_a);
@@ -435,22 +471,34 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       }
       const uint32_t d_tmem = tmem_base + acc * MPI * kCols;
       for (int kb = kb_begin; kb < kb_end; ++kb) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(W8 ? &conv_full[stage] : &full[stage], phase, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + stage * L::kA);
         const uint32_t b0 = smem_u32(sB + stage * L::kBStage);
         const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
+        if constexpr (W8) {
+          // A: the converted bf16 tile in tensor memory (8 columns per 16 k)
+          const uint32_t at = tmem_base + kACol + stage * MPI * 32;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc,
-                    (kb != kb_begin || kk != 0) ? 1u : 0u);
-          if (SPLIT == kSplitA)
-            umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc, 1);
+          for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-          for (int u = 1; u < MPI; ++u)
-            if (u < mc)
-              umma_bf16(d_tmem + u * kCols, sdesc_k_sw128(a0 + u * L::kAtile + kk * 32), sdesc_k_sw128(b0 + kk * 32),
-                        idesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
+            for (int u = 0; u < MPI; ++u)
+              if (u < mc)
+                umma_bf16_ts(d_tmem + u * kCols, at + u * 32 + kk * 8, sdesc_k_sw128(b0 + kk * 32), idesc,
+                             (kb != kb_begin || kk != 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc,
+                      (kb != kb_begin || kk != 0) ? 1u : 0u);
+            if (SPLIT == kSplitA)
+              umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc, 1);
+#pragma unroll
+            for (int u = 1; u < MPI; ++u)
+              if (u < mc)
+                umma_bf16(d_tmem + u * kCols, sdesc_k_sw128(a0 + u * L::kAtile + kk * 32), sdesc_k_sw128(b0 + kk * 32),
+                          idesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -464,6 +512,49 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     // wait for every MMA issued by this thread before TMEM is released
     umma_commit(drain);
     mbar_drain(drain, 0);
+  } else if (W8 && warp >= 6) {
+    // ---------------- converters (W8): FP8 tile -> bf16 in tensor memory, one row per thread
+    if constexpr (W8) {
+      const int q = warp & 3;
+      const int r = q * 32 + lane;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const Tile t = sched.tile(j);
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) { ok = false; break; }
+          for (int u = 0; u < t.m_count; ++u) {
+            // the FP8 tile was stored with the 64-byte swizzle: 16-byte chunk c of row r
+            // sits at chunk c ^ ((r >> 1) & 3) of its 64-byte row
+            const uint8_t* row = sA + stage * L::kA + u * L::kAtile + r * 64;
+            uint4 v[4];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + ((c ^ ((r >> 1) & 3)) << 4));
+            const float sc = ldexpf(1.0f, sched.exponent(t, u, r, kb));
+            uint32_t o[32];
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                o[c * 8 + 2 * i] = e4m3x2_to_bf16x2((uint16_t)(w[i] & 0xFFFFu), sc);
+                o[c * 8 + 2 * i + 1] = e4m3x2_to_bf16x2((uint16_t)(w[i] >> 16), sc);
+              }
+            }
+            tmem_st32_nowait(tmem_at(tmem_base + kACol + (stage * MPI + u) * 32, q * 32, 0), o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&conv_full[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        atomicExch(err, kDevTimeoutProducer);
+        *abort_flag = 1;
+      }
+    }
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter this warp may access

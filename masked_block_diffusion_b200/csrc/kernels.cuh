@@ -599,6 +599,46 @@ __global__ void canvas_init_kernel(int32_t* canvas, uint8_t* mask, int n, int ma
   if (i < B) step[i] = 0;
 }
 
+// ---------------------------------------------------------------- FP8 expert weights
+
+// One CTA per 128 x 128 tile (bi, bj) = (blockIdx.y, blockIdx.x) of a bf16 matrix src
+// [rows][cols]: the tile's scale exponent e is the least integer with max|w| <= 448 * 2^e
+// (0 for an all-zero tile), stored at exps[bi * gridDim.x + bj]; every element becomes the
+// E4M3 code of w * 2^-e (round to nearest even), written to dst row
+// (i / group) * group_stride + i % group + row_offset (the same row map as
+// pack_rows_kernel), dst rows cols bytes long.
+__global__ void __launch_bounds__(256) quantize_e4m3_blocks_kernel(const bf16_t* __restrict__ src, int rows, int cols,
+                                                                   uint8_t* __restrict__ dst, int8_t* __restrict__ exps,
+                                                                   long group, long group_stride, long row_offset) {
+  pdl_begin();
+  const int r0 = blockIdx.y * 128, c0 = blockIdx.x * 128;
+  const int nr = min(128, rows - r0), nc = min(128, cols - c0);
+  float amax = 0.f;
+  for (int i = threadIdx.x; i < nr * nc; i += blockDim.x) {
+    const int r = i / nc, c = i % nc;
+    amax = fmaxf(amax, fabsf(bf16_to_f32(src[(long)(r0 + r) * cols + c0 + c])));
+  }
+  __shared__ float red[8];
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
+  int e = 0;
+  if (amax > 0.f) {
+    e = (int)ceilf(log2f(amax / 448.0f));
+    while (amax > ldexpf(448.0f, e)) ++e;
+    while (amax <= ldexpf(448.0f, e - 1)) --e;
+  }
+  if (threadIdx.x == 0) exps[blockIdx.y * gridDim.x + blockIdx.x] = (int8_t)e;
+  const float inv = ldexpf(1.0f, -e);
+  for (int i = threadIdx.x; i < nr * nc; i += blockDim.x) {
+    const long r = r0 + i / nc, c = c0 + i % nc;
+    const long drow = (r / group) * group_stride + (r % group) + row_offset;
+    dst[drow * cols + c] = f32_to_e4m3(bf16_to_f32(src[r * cols + c]) * inv);
+  }
+}
+
 // ---------------------------------------------------------------- weight packing
 
 // dst row ((i / group) * group_stride + i % group + row_offset) = bf16(src row i).

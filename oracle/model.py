@@ -62,7 +62,13 @@ Readings where the pages are silent (all listed in the design notes):
 12. approximate append (What changes, section 5 "KV caching": Fast-dLLM's
    training-free, block-wise approximate cache): the finished canvas's K/V are taken
    from its last denoising pass, computed while the positions that pass committed
-   were still [MASK], instead of from one more pass over the finished canvas.
+   were still [MASK], instead of from one more pass over the finished canvas;
+13. FP8 expert weights (What changes, section 4.2 "Speed": the measured setting runs
+   FP8; DiffusionGemma names NVFP4 as the next step): optionally, the expert matrices
+   Wg, Wu, Wd are held as FP8 E4M3 with one power-of-two scale 2^e per 128 x 128 tile
+   of each matrix, e the least integer with the tile's max |w| <= 448 * 2^e, values
+   rounded to nearest (ties to even); the pass then runs on those values exactly as on
+   bf16 weights (they are bf16-exact).
 
 Parity pins (tests/test_oracle_pins.py), one or more per function: RMSNorm against
 closed forms (constant and +-a rows, a hand-worked row, scale invariance); bf16
@@ -113,6 +119,62 @@ def bf16_store(w) -> np.ndarray:
 
 
 _bf16_store = bf16_store
+
+
+# --------------------------------------------------------------------------------------
+# FP8 expert weights (reading 13)
+
+def e4m3_values() -> np.ndarray:
+    """The non-negative finite values of FP8 E4M3 in code order: 1 sign bit, 4 exponent
+    bits with bias 7, 3 mantissa bits, no infinities, code 0x7F is NaN. Code c = 8 e + m
+    is m / 8 * 2^-6 for e = 0 (subnormal) and (1 + m / 8) * 2^(e - 7) otherwise; the
+    largest finite value is 448."""
+    vals = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        vals.append(m / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest E4M3 value to x (|x| <= 448), ties to the even code, sign kept."""
+    v = e4m3_values()
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    i = np.clip(np.searchsorted(v, a), 1, v.size - 1)      # v[i - 1] < a <= v[i]
+    lo, hi = v[i - 1], v[i]
+    up = (hi - a < a - lo) | ((hi - a == a - lo) & (i % 2 == 0))
+    return np.sign(x) * np.where(up, hi, lo)
+
+
+def fp8_block_exponents(w: np.ndarray, block: int = 128) -> np.ndarray:
+    """Per block x block tile of w (edge tiles smaller): the least integer e with
+    max|w| <= 448 * 2^e over the tile (0 for an all-zero tile)."""
+    w = np.asarray(w, dtype=np.float64)
+    R, Cn = w.shape
+    ex = np.zeros(((R + block - 1) // block, (Cn + block - 1) // block), dtype=np.int64)
+    for bi in range(ex.shape[0]):
+        for bj in range(ex.shape[1]):
+            amax = float(np.max(np.abs(w[bi * block:(bi + 1) * block, bj * block:(bj + 1) * block])))
+            if amax == 0.0:
+                continue
+            e = int(math.ceil(math.log2(amax / 448.0)))
+            while amax > math.ldexp(448.0, e):
+                e += 1
+            while amax <= math.ldexp(448.0, e - 1):
+                e -= 1
+            ex[bi, bj] = e
+    return ex
+
+
+def fp8_block_dequant(w: np.ndarray, block: int = 128) -> np.ndarray:
+    """The values an FP8 E4M3 copy of w holds with one power-of-two scale 2^e per
+    block x block tile (e from fp8_block_exponents): q = e4m3_round(w / 2^e), returned
+    as q * 2^e in float32 (exact: 4 significant bits times a power of two)."""
+    w = np.asarray(w, dtype=np.float64)
+    ex = fp8_block_exponents(w, block)
+    s = np.repeat(np.repeat(np.ldexp(1.0, ex), block, axis=0), block, axis=1)[:w.shape[0], :w.shape[1]]
+    return (e4m3_round(w / s) * s).astype(np.float32)
 
 
 # --------------------------------------------------------------------------------------
@@ -306,10 +368,13 @@ class _Request:
 class OracleModel:
     """The denoiser over named weights (float32 arrays, e.g. from synth.gen_weights)."""
 
-    def __init__(self, cfg, weights: Dict[str, np.ndarray], f64_matrices: bool = False):
+    def __init__(self, cfg, weights: Dict[str, np.ndarray], f64_matrices: bool = False,
+                 expert_fp8: bool = False):
         """f64_matrices keeps every matrix as float64 (the same bf16 values) instead of
         float32, so that the products do not convert their operands on every call: faster
-        for repeated passes, twice the memory, identical results."""
+        for repeated passes, twice the memory, identical results. expert_fp8 replaces the
+        expert matrices (Wg, Wu, Wd of every MoE expert) by their FP8 block-scaled values
+        (reading 13); everything else is unchanged."""
         self.cfg = cfg
         c = cfg
         # every matrix enters its products as a bf16 operand (reading 10); norm gains
@@ -336,9 +401,10 @@ class OracleModel:
                                   bf16_store(weights[p + "wd"]))]
             else:
                 lw["wr"] = bf16_store(weights[p + "wr"])
-                lw["experts"] = [(bf16_store(weights[p + f"experts.{e}.wg"]),
-                                  bf16_store(weights[p + f"experts.{e}.wu"]),
-                                  bf16_store(weights[p + f"experts.{e}.wd"]))
+                ex = (lambda w: bf16_store(fp8_block_dequant(_bf16_store(w)))) if expert_fp8 else bf16_store
+                lw["experts"] = [(ex(weights[p + f"experts.{e}.wg"]),
+                                  ex(weights[p + f"experts.{e}.wu"]),
+                                  ex(weights[p + f"experts.{e}.wd"]))
                                  for e in range(c.n_experts)]
             self.layers.append(lw)
         self.final_norm = np.asarray(weights["final_norm"], np.float64)

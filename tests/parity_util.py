@@ -31,11 +31,11 @@ def cached_weights(cfg):
     return gen_weights(cfg, threads=os.cpu_count() or 8)
 
 
-def build_pair(cfg, prefix: int, prompt_seed: int, max_ctx: int, max_batch: int = 1):
+def build_pair(cfg, prefix: int, prompt_seed: int, max_ctx: int, max_batch: int = 1, expert_fp8: bool = False):
     W = cached_weights(cfg)
     blob = blob_from_weights(cfg, W)
-    orc = OracleModel(cfg, W, f64_matrices=cfg.d_model >= 2048)
-    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=max_batch)
+    orc = OracleModel(cfg, W, f64_matrices=cfg.d_model >= 2048, expert_fp8=expert_fp8)
+    den = Denoiser(cfg, blob, max_ctx=max_ctx, max_batch=max_batch, expert_fp8=expert_fp8)
     del blob
     prompt = prompt_tokens(cfg.vocab, prompt_seed, prefix)
     rec = {}

@@ -97,3 +97,30 @@ def test_lm_head_conf_full_size_sampled():
     sel = margin > 1e-3
     assert np.array_equal(arg[sel], ra[sel])
     assert np.all(np.abs(conf / rc - 1) < 2e-2)
+
+
+def test_fp8_block_quantiser_matches_the_oracle_bit_for_bit():
+    """dllm_op_quantize_fp8 (the quantiser dllm_create applies to expert matrices) against
+    the oracle's definition: the same tile exponents and the same E4M3 codes, on a matrix
+    whose tiles have ragged edges, a large outlier and an all-zero tile."""
+    import oracle.model as om
+    rows, cols = 300, 400
+    w = (uniform_f32(47, 1, rows * cols, -1, 1) * np.float32(0.05)).reshape(rows, cols)
+    w[140, 7] = 2.5
+    w[256:, 384:] = 0.0
+    w = bf16_bits_to_f32(f32_to_bf16_bits(w))
+    W = dev_bf16(w)
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device="cuda")
+    ex = torch.zeros((3, 4), dtype=torch.int8, device="cuda")
+    binding.dllm_op_quantize_fp8(W.data_ptr(), rows, cols, q.data_ptr(), ex.data_ptr(),
+                                 torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    ex_ref = om.fp8_block_exponents(w.astype(np.float64))
+    assert np.array_equal(ex.cpu().numpy().astype(np.int64), ex_ref)
+    codes = q.cpu().numpy()
+    vals = om.e4m3_values()
+    mag = vals[codes & 0x7F]
+    sign = np.where(codes & 0x80, -1.0, 1.0)
+    s = np.ldexp(1.0, np.repeat(np.repeat(ex_ref, 128, 0), 128, 1)[:rows, :cols])
+    assert np.all((codes & 0x7F) != 0x7F)                       # no NaN code
+    assert np.array_equal(sign * mag * s, om.fp8_block_dequant(w.astype(np.float64)).astype(np.float64))

@@ -340,3 +340,24 @@ def test_approximate_append_matches_the_oracle():
         assert stats["steps"] == S
     finally:
         den.close()
+
+
+@pytest.mark.parametrize("name,layers,prefix", [("c2-small-moe", 2, 512), ("c3-moe26b-canvas", 2, 512)])
+def test_fp8_experts_match_the_oracle(name, layers, prefix):
+    """Expert weights held as FP8 E4M3 with power-of-two 128 x 128 tile scales: the GPU's
+    pass (FP8 tiles expanded to bf16 in tensor memory) against the oracle running on the
+    same FP8 values, step by step."""
+    w = WORKLOADS[name]
+    cfg = w.model.with_layers(layers)
+    C = cfg.canvas
+    S = 8
+    pol = Policy("topk", k=C // S)
+    orc, den, _ = build_pair(cfg, prefix, w.prompt_seed + 13, prefix + 2 * C, expert_fp8=True)
+    try:
+        _, steps, trace = orc.generate_block(0, pol, S, trace=True)
+        stats = compare_trace(cfg, trace[:4], den, pol, S)
+        assert stats["route_pinned"] > 0.9 * stats["route_total"]
+        assert stats["arg_pinned"] > 0.9 * stats["arg_total"]
+        check_generate_invariants(cfg, den, pol, S, expect_steps=steps)
+    finally:
+        den.close()

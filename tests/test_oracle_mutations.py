@@ -284,6 +284,34 @@ def append_approx_from_masked(self, req):   # K/V of the canvas as if every posi
     om.OracleModel.__dict__["_orig_append_approx"](self, req)
 
 
+def fp8_exponents_plus_one(w, block=128):     # a scale twice the least one
+    return om.__dict__["_orig_fp8_block_exponents"](w, block) + 1
+
+
+def fp8_exponents_per_row(w, block=128):      # the first row's scale for its whole tile
+    w = np.asarray(w, np.float64)
+    ex = om.__dict__["_orig_fp8_block_exponents"](w, block)
+    for bi in range(ex.shape[0]):
+        ex[bi] = om.__dict__["_orig_fp8_block_exponents"](w[bi * block:bi * block + 1], block)[0]
+    return ex
+
+
+def e4m3_truncate(x):                         # rounds toward zero
+    v = om.e4m3_values()
+    x = np.asarray(x, np.float64)
+    i = np.searchsorted(v, np.abs(x), side="right") - 1
+    return np.sign(x) * v[i]
+
+
+def e4m3_ties_up(x):                          # ties away from zero instead of to the even code
+    v = om.e4m3_values()
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    i = np.clip(np.searchsorted(v, a), 1, v.size - 1)
+    lo, hi = v[i - 1], v[i]
+    return np.sign(x) * np.where(hi - a <= a - lo, hi, lo)
+
+
 # ---------------------------------------------------------------- which pins guard what
 
 P = pins
@@ -328,6 +356,10 @@ CASES = [
     ("edit_select", edit_select_masked_too, [P.test_edit_select_rule]),
     ("edit_select", edit_select_at_or_above, [P.test_edit_select_rule]),
     ("edit_select", edit_select_ignores_token, [P.test_edit_select_rule, P.test_generate_block_t2t_invariants]),
+    ("fp8_block_exponents", fp8_exponents_plus_one, [P.test_fp8_block_scales_and_round_trip]),
+    ("fp8_block_exponents", fp8_exponents_per_row, [P.test_fp8_block_scales_and_round_trip]),
+    ("e4m3_round", e4m3_truncate, [P.test_e4m3_rounding_ties_and_torch, P.test_fp8_block_scales_and_round_trip]),
+    ("e4m3_round", e4m3_ties_up, [P.test_e4m3_rounding_ties_and_torch]),
     ("OracleModel.append_approx", append_approx_from_masked,
      [lambda: P.test_approximate_append_equals_exact_append_on_a_finished_pass(P.MICRO)]),
 ]

@@ -444,3 +444,84 @@ def test_approximate_append_equals_exact_append_on_a_finished_pass(cfg):
     a2.append_approx(0)
     b2.append(0, fin)
     assert not np.array_equal(a2.requests[0].k[0][10:], b2.requests[0].k[0][10:])
+
+
+# ---------------------------------------------------------------- FP8 expert weights
+
+def test_e4m3_value_set():
+    v = oracle.model.e4m3_values()
+    assert v.size == 127 and v[0] == 0.0 and v[-1] == 448.0
+    assert v[1] == 2.0 ** -9 and v[8] == 2.0 ** -6            # smallest subnormal, smallest normal
+    assert np.all(np.diff(v) > 0)
+    # one binade holds 8 values, equally spaced by a 1/8 of its lower end
+    b = v[(v >= 1.0) & (v < 2.0)]
+    assert np.allclose(b, 1.0 + np.arange(8) / 8.0)
+
+
+def test_e4m3_rounding_ties_and_torch():
+    import torch
+    cases = {0.53125: 0.5,            # halfway between 0.5 (code 48) and 0.5625 (49): even code
+             0.59375: 0.625,          # halfway between 0.5625 (49) and 0.625 (50)
+             -0.59375: -0.625,
+             3 * 2.0 ** -10: 2.0 ** -8,   # subnormal tie between codes 1 and 2
+             440.0: 448.0, 0.0: 0.0, 17.0: 16.0, 17.5: 18.0}
+    got = oracle.model.e4m3_round(np.array(list(cases)))
+    assert np.array_equal(got, np.array(list(cases.values())))
+    x = np.concatenate([uniform_f32(11, 1, 20000, -448, 448), uniform_f32(11, 2, 20000, -0.05, 0.05)])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.model.e4m3_round(x.astype(np.float64)), ref)
+
+
+def test_fp8_block_scales_and_round_trip():
+    om = oracle.model
+    # 200 x 300: tiles of 128 x 128 with a 72-row and a 44-column edge
+    w = rnd((200, 300), 40, scale=0.05)
+    w[130:140, 10] = 3.0                  # one tile with a large entry
+    ex = om.fp8_block_exponents(w)
+    assert ex.shape == (2, 3)
+    for bi in range(2):
+        for bj in range(3):
+            t = w[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]
+            amax = np.abs(t).max()
+            # the least power of two that brings the tile's largest entry within 448
+            assert 224.0 < amax / 2.0 ** ex[bi, bj] <= 448.0
+    assert ex[1, 0] > ex[0, 0]            # the large entry sets only its own tile's scale
+    d = om.fp8_block_dequant(w)
+    s = np.ldexp(1.0, np.repeat(np.repeat(ex, 128, 0), 128, 1)[:200, :300])
+    q = d.astype(np.float64) / s
+    # the stored values are E4M3 numbers times the tile scale, and bf16-exact
+    assert np.array_equal(np.abs(q), om.e4m3_round(np.abs(q)))
+    assert np.array_equal(d.astype(np.float64), oracle.bf16(d))
+    # round trip: relative error <= 2^-4 in the normal range, absolute <= 2^-10 * s below it
+    err = np.abs(d - w)
+    normal = np.abs(w) / s >= 2.0 ** -6
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(w[normal]))
+    assert np.all(err[~normal] <= 2.0 ** -10 * s[~normal])
+    # a tile whose entries are E4M3 numbers times a power of two is held exactly
+    exact = np.ldexp(om.e4m3_values()[80:120], -12)
+    assert np.array_equal(om.fp8_block_dequant(exact[None, :]).astype(np.float64), exact[None, :])
+    assert np.all(om.fp8_block_dequant(np.zeros((4, 4))) == 0.0)
+
+
+def test_fp8_expert_model_runs_on_the_dequantised_experts():
+    cfg = MICRO
+    W = gen_weights(cfg)
+    m8 = OracleModel(cfg, W, expert_fp8=True)
+    m = OracleModel(cfg, W)
+    wg = W["layers.0.experts.1.wg"]
+    assert np.array_equal(m8.layers[0]["experts"][1][0], oracle.model.fp8_block_dequant(wg))
+    assert np.array_equal(m8.layers[0]["wq"], m.layers[0]["wq"])      # only the experts change
+    # the FP8 model's pass equals the bf16 model's pass on weights replaced by their FP8 values
+    W2 = dict(W)
+    for l in range(cfg.n_layers):
+        for e in range(cfg.n_experts):
+            for n in ("wg", "wu", "wd"):
+                key = f"layers.{l}.experts.{e}.{n}"
+                W2[key] = oracle.model.fp8_block_dequant(W[key])
+    m2 = OracleModel(cfg, W2)
+    p = prompt_tokens(cfg.vocab, 2007, 9)
+    m8.prefill(0, p)
+    m2.prefill(0, p)
+    c8, a8 = m8.denoise_pass(0, np.full(cfg.canvas, cfg.mask_id), np.ones(cfg.canvas, bool))
+    c2, a2 = m2.denoise_pass(0, np.full(cfg.canvas, cfg.mask_id), np.ones(cfg.canvas, bool))
+    assert np.array_equal(c8, c2) and np.array_equal(a8, a2)
