@@ -86,7 +86,7 @@ typedef struct {
    * 128 x 128 tile of the matrix, e the least integer with the tile's max |w| <= 448 * 2^e,
    * codes rounded to nearest even (What changes, section 4.2 "Speed": the measured setting
    * runs FP8). The kernels expand each staged tile to bf16 exactly, so the pass computes on
-   * the FP8 values; expert bytes per pass halve. Needs ffn_dim and d_model multiples of 128. */
+   * the FP8 values; expert bytes per pass halve. */
   int expert_format;
 } dllm_config;
 

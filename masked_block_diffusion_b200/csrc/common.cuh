@@ -31,8 +31,10 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 // Limit of the pipeline waits (mbar_wait, mbar_wait_cluster): kWaitLimitNs unless
 // dllm_set_wait_limit changed it for this device (tests of the timeout path). The drain
 // waits that let copies and MMAs already in flight land before a CTA exits always use
-// kWaitLimitNs, so a short pipeline limit never cuts them short.
-__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+// kWaitLimitNs, so a short pipeline limit never cuts them short. Constant memory: a
+// wait that does not succeed at once reads it, and a global load there would put a
+// memory round trip on every such wait of the pipelines.
+__constant__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 DLLM_DEV float bf16_to_f32(bf16_t v) { return __uint_as_float(((uint32_t)v) << 16); }
 
@@ -53,6 +55,16 @@ DLLM_DEV void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
   lo = pack_bf16x2(a - bf16_to_f32(ha), b - bf16_to_f32(hb));
 }
 
+// The same split with a third term: hi + mid + lo carries all 24 bits of an fp32 value.
+DLLM_DEV void split3_bf16x2(float a, float b, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  const bf16_t ha = f32_to_bf16(a), hb = f32_to_bf16(b);
+  hi = (uint32_t)ha | ((uint32_t)hb << 16);
+  const float ra = a - bf16_to_f32(ha), rb = b - bf16_to_f32(hb);
+  const bf16_t ma = f32_to_bf16(ra), mb = f32_to_bf16(rb);
+  mid = (uint32_t)ma | ((uint32_t)mb << 16);
+  lo = pack_bf16x2(ra - bf16_to_f32(ma), rb - bf16_to_f32(mb));
+}
+
 DLLM_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 // ---------------------------------------------------------------- FP8 E4M3
@@ -67,7 +79,8 @@ DLLM_DEV uint8_t f32_to_e4m3(float x) {
 DLLM_DEV uint32_t e4m3x2_to_bf16x2(uint16_t two, float scale) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
   const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-  return pack_bf16x2(f.x * scale, f.y * scale);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 DLLM_DEV unsigned long long global_ns() {

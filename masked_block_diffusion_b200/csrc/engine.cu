@@ -22,6 +22,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "common.cuh"
@@ -31,6 +33,15 @@
 using namespace dllm;
 
 namespace {
+
+// NVTX range for the duration of a scope: entry points and, when kernels are launched
+// eagerly (graph capture, DLLM_NO_GRAPH), each layer. A no-op unless a profiler attaches.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -78,9 +89,6 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Token-operand boxes of the grouped expert GEMMs: a chunk of up to kMoeChunk tokens is
-// loaded from boxes of these heights (its count rounded up to 16), so the MMA width
-// follows the chunk's token count.
 // 2-D uint8 tensor map over [rows][cols] FP8 codes, box = 64 columns x box_rows, 64-byte
 // swizzle (the converter warps read each row's four 16-byte chunks at chunk ^ ((row >> 1) & 3)).
 bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -96,8 +104,15 @@ bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Token-operand boxes of the grouped expert GEMMs: a chunk of up to 64 or 128 tokens is
+// loaded from boxes of these heights (its count rounded up to 16), so the MMA width
+// follows the chunk's token count.
 constexpr int kMoeBN[4] = {16, 32, 64, 128};
-constexpr int kMoeChunk = 128;
+
+// Chunk width of the grouped expert GEMMs: 64 tokens while the mean per expert stays at
+// or below 64 (a batch-1 canvas: experts are few and uneven, and more, smaller items
+// spread better over the SMs), else 128 (prefill, large batches: fewer weight-tile reads).
+int moe_chunk(int N, int E) { return (double)N / (double)E <= 64.0 ? 64 : 128; }
 
 struct LayerW {
   float* attn_norm = nullptr;
@@ -173,22 +188,18 @@ struct dllm_handle {
   int32_t* argmax = nullptr;
   // lo halves of the activation operands carried as (hi, lo) bf16 pairs
   bf16_t* y_lo = nullptr;
+  bf16_t* y_lo2 = nullptr;   // third term of the attention norm's output (the QKV operand)
   bf16_t* ao_lo = nullptr;
   bf16_t* xg_lo = nullptr;
   bf16_t* hbuf_lo = nullptr;
-  CUtensorMap tm_y, tm_ao, tm_xg[4], tm_h[4];
-  CUtensorMap tm_y_lo, tm_ao_lo, tm_xg_lo[4], tm_h_lo[4];
-  CUtensorMap* d_tok_maps = nullptr;   // device copies: [xg hi 16..128 | xg lo | h hi | h lo]
+  CUtensorMap tm_y, tm_xg[4], tm_h[4];
+  CUtensorMap tm_y_lo, tm_y_lo2, tm_xg_lo[4], tm_h_lo[4];
+  TokMaps tok_xg, tok_h;     // the grouped GEMMs' token-operand maps: boxes of 16..128 rows, hi then lo
   CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
-  bool attn_tc = false;     // canvas passes use the tensor-core attention
-  bool oproj_swap = true;   // O projection with swapped operands (weights as M, stacked token halves as N)
-  bool qkv_splitk = true;   // QKV projection on few tiles: K split over CTA pairs
-  bool prefill_tc = true;   // causal prefill attention on the tensor cores too
+  bool attn_tc = false;     // attention on the tensor cores (the GQA group divides a 128-row query tile)
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
   bool router_tc = false;   // router logits on the tensor cores (experts a multiple of 32)
-  int router_ks = 8;        // largest K split of the router GEMM
-  bool pdl = true;          // programmatic dependent launch between the kernels of a pass
   bool w8 = false;          // FP8 expert weights
 
   std::vector<int> P;        // prefix length per slot (-1 = no prefill yet)
@@ -302,8 +313,8 @@ int attn_splits(const dllm_handle* h, int B) {
 
 // ------------------------------------------------------------------ launch helpers
 
-// Launches kern on the handle's stream; with h->pdl the launch carries programmatic
-// stream serialisation, so the kernel may start while its predecessor drains (every
+// Launches kern on the handle's stream; the launch carries programmatic stream
+// serialisation, so the kernel may start while its predecessor drains (every
 // kernel of the pass waits for its predecessor with griddepcontrol.wait before its first
 // global-memory access).
 template <typename... KArgs, typename... Args>
@@ -317,7 +328,7 @@ cudaError_t launch_k(dllm_handle* h, void (*kern)(KArgs...), dim3 grid, dim3 blo
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = h->pdl ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -325,7 +336,11 @@ cudaError_t launch_k(dllm_handle* h, void (*kern)(KArgs...), dim3 grid, dim3 blo
 template <int BN, int STAGES, int ACC, int SPLIT, class Sched, class Epi>
 cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const CUtensorMap& tb, int kblocks,
                         int a_first, const Sched& s, const Epi& e, const CUtensorMap* ta2 = nullptr,
-                        const CUtensorMap* tb2 = nullptr) {
+                        const CUtensorMap* tb2 = nullptr, const TokMaps* tok = nullptr,
+                        const CUtensorMap* ta3 = nullptr) {
+  static const TokMaps no_tok{};   // the token maps of a dynamic-width schedule, or the third A term
+  TokMaps tk = tok ? *tok : no_tok;
+  if (ta3) tk.m[0] = *ta3;
   auto kern = gemm_tc_kernel<BN, STAGES, ACC, SPLIT, Sched, Epi>;
   constexpr int smem = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>::kTotal;
   static_assert(smem <= 232448, "shared memory per CTA");
@@ -347,36 +362,40 @@ cudaError_t launch_gemm(dllm_handle* h, dim3 grid, const CUtensorMap& ta, const 
     at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = h->pdl ? 2 : 1;
+    cfg.numAttrs = 2;
     if (grid.x % Sched::kKSplit || kblocks < Sched::kKSplit) return cudaErrorInvalidValue;
-    r = cudaLaunchKernelEx(&cfg, kern, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks, a_first, s, e, h->d_err);
+    r = cudaLaunchKernelEx(&cfg, kern, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, tk, kblocks, a_first, s, e, h->d_err);
     h->launches++;
     if (r != cudaSuccess) return r;
     return cudaGetLastError();
   }
-  r = launch_k(h, kern, grid, dim3(gemm_threads<Sched>()), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, kblocks,
-               a_first, s, e, h->d_err);
+  r = launch_k(h, kern, grid, dim3(gemm_threads<Sched>()), smem, ta, ta2 ? *ta2 : ta, tb, tb2 ? *tb2 : tb, tk,
+               kblocks, a_first, s, e, h->d_err);
   h->launches++;
   if (r != cudaSuccess) return r;
   return cudaGetLastError();
 }
 
+// The QKV projection reads the attention norm's output as three bf16 terms (all of its
+// fp32 bits, three MMAs per k step): Q, K and V are rounded to bf16 right after, and a
+// 16-bit operand would move that rounding often enough to shift attention over
+// thousands of cached keys measurably (router logits by up to 2e-3 at a 4096-token prefix).
 template <int HD>
 cudaError_t qkv_gemm_hd(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, int T, const int* pos0,
                         const int* slot, int tok_per_req) {
   const auto& c = h->c;
   EpiQKV<HD> e{h->q, kc, vc, h->rope_cos, h->rope_sin, pos0, slot, tok_per_req, c.n_heads, c.n_kv_heads, c.max_ctx};
   const int mt = ceil_div(T, 128);
-  constexpr int STAGES = HD > 128 ? 4 : 5;
-  if (h->qkv_splitk && mt * h->qkv_heads * 2 <= 2 * h->num_sms) {
+  constexpr int STAGES = HD > 128 ? 3 : 4;
+  if (mt * h->qkv_heads * 2 <= 2 * h->num_sms) {
     // few tiles (one canvas): split K over CTA pairs so that about twice as many SMs stream
     DenseSplitKSched<2> s{T, mt, HD};
-    return launch_gemm<HD, STAGES, 1, kSplitA>(h, dim3(mt * h->qkv_heads * 2), h->tm_y, L.tm_wqkv, c.d_model / 64, 0,
-                                               s, e, &h->tm_y_lo);
+    return launch_gemm<HD, STAGES, 1, kSplitA3>(h, dim3(mt * h->qkv_heads * 2), h->tm_y, L.tm_wqkv, c.d_model / 64, 0,
+                                                s, e, &h->tm_y_lo, nullptr, nullptr, &h->tm_y_lo2);
   }
   DenseSched s{T, mt, HD};
-  return launch_gemm<HD, STAGES, 1, kSplitA>(h, dim3(mt * h->qkv_heads), h->tm_y, L.tm_wqkv, c.d_model / 64, 0, s, e,
-                                             &h->tm_y_lo);
+  return launch_gemm<HD, STAGES, 1, kSplitA3>(h, dim3(mt * h->qkv_heads), h->tm_y, L.tm_wqkv, c.d_model / 64, 0, s, e,
+                                              &h->tm_y_lo, nullptr, nullptr, &h->tm_y_lo2);
 }
 
 cudaError_t qkv_gemm(dllm_handle* h, const LayerW& L, bf16_t* kc, bf16_t* vc, int T, const int* pos0,
@@ -474,7 +493,7 @@ cudaError_t attention(dllm_handle* h, bf16_t* kc, bf16_t* vc, int T, int nreq, i
                       const int* slot, int causal, int splits, const LayerW* L = nullptr) {
   // tensor cores: the bidirectional canvas pass, and (one key range per query tile) the
   // causal prompt prefill
-  if (h->attn_tc && L && (!causal || (h->prefill_tc && splits == 1))) {
+  if (h->attn_tc && L && (!causal || splits == 1)) {
     if (h->c.head_dim == 176)
       return attention_tc_hd<176>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits);
     return attention_tc_hd<64>(h, *L, T, nreq, tok_per_req, pos0, slot, causal, splits);
@@ -519,100 +538,99 @@ cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T) {
   const int mt = ceil_div(T, 128);
   const int tiles = mt * (h->E / 32);
   const int kb = h->c.d_model / 64;
-  const int cap = h->router_ks;   // largest split allowed (1, 2, 4 or 8)
-  if (cap >= 8 && tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
-  if (cap >= 4 && tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
-  if (cap >= 2 && tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
+  if (tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
+  if (tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
+  if (tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
   return router_gemm_ks<1>(h, L, T, mt, tiles);
 }
 
-// Attention output projection with the residual add, x += ao * Wo^T. By default the
-// operands are swapped: weight rows (output features) are M and 64-token chunks N, with
-// the token operand's (hi, lo) halves stacked into one N = 128 MMA, so each weight tile
-// is read from shared memory once per k step. Otherwise tokens are M and the (hi, lo)
-// pair is the A operand (two MMAs per k step).
+// Attention output projection with the residual add, x += ao * Wo^T, operands swapped:
+// weight rows (output features) are M and 64-token chunks N, with the token operand's
+// (hi, lo) halves stacked into one N = 128 MMA, so each weight tile is read from shared
+// memory once per k step (measured faster than tokens as M with two MMAs per k step:
+// 0.73 vs 0.91 ms per 26B canvas pass).
 cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int kb = c.n_heads * c.head_dim / 64;
-  if (h->oproj_swap) {
-    EpiResidualT<64> et{h->x, d, T};
-    DenseSched s{d, d / 128, 64};
-    return launch_gemm<64, 6, 1, kSplitB>(h, dim3((d / 128) * ceil_div(T, 64)), L.tm_wo128, h->tm_ao64, kb, 1, s, et,
-                                          nullptr, &h->tm_ao64_lo);
-  }
-  EpiResidual<64> e{h->x, d};
-  const int mt = ceil_div(T, 128);
-  DenseSched s{T, mt, 64};
-  return launch_gemm<64, 5, 1, kSplitA>(h, dim3(mt * (d / 64)), h->tm_ao, L.tm_wo, kb, 0, s, e, &h->tm_ao_lo);
+  EpiResidualT<64> et{h->x, d, T};
+  DenseSched s{d, d / 128, 64};
+  return launch_gemm<64, 6, 1, kSplitB>(h, dim3((d / 128) * ceil_div(T, 64)), L.tm_wo128, h->tm_ao64, kb, 1, s, et,
+                                        nullptr, &h->tm_ao64_lo);
 }
 
-// One grouped gate/up (or down) GEMM over chunks of up to kMoeChunk tokens, with MPI
-// weight tiles per work item and ACC accumulator buffers (MPI * ACC * 2 * kMoeChunk TMEM
-// columns <= 512). The MMA width of each chunk follows its token count.
-template <int MPI, int ACC>
+// One grouped gate/up (or down) GEMM over chunks of up to BN tokens, with MPI weight
+// tiles per work item and ACC accumulator buffers (MPI * ACC * 2 * BN TMEM columns <= 512).
+// The MMA width of each chunk follows its token count.
+template <int BN, int MPI, int ACC>
 cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int BN = kMoeChunk;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->d_tok_maps, h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128,
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128,
                                 BN};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
   return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[3], d / 64, 1, s, e, nullptr,
-                                               &h->tm_xg_lo[3]);
+                                               &h->tm_xg_lo[3], &h->tok_xg);
 }
 
-template <int MPI, int ACC>
+template <int BN, int MPI, int ACC>
 cudaError_t moe_down(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int BN = kMoeChunk;
   constexpr int STAGES = (192 * 1024) / (MPI * 16384 + 2 * BN * 128);
-  PersistentGroupedSched<MPI> s{h->d_tok_maps + 8, h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128,
+  PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128,
                                 BN};
   EpiDown<BN> e{h->obuf, d};
   return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[3], F / 64, 1, s, e, nullptr,
-                                               &h->tm_h_lo[3]);
+                                               &h->tm_h_lo[3], &h->tok_h);
 }
 
-// The FP8-weight variants: one weight tile per item and one accumulator, the rest of
-// tensor memory holding the converted bf16 A stages.
+// The FP8-weight variants: one weight tile per item; tensor memory holds the accumulators
+// and the converted bf16 A stages (32 columns each).
+template <int BN, int ACC, int STAGES>
 cudaError_t moe_gate_up_w8(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int BN = kMoeChunk;
-  constexpr int STAGES = 4;
-  PersistentGroupedSched<1, true> s{h->d_tok_maps, h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F,
+  PersistentGroupedSched<1, true> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F,
                                     2 * F / 128, BN, L.egu, 1, (F + 127) / 128, (d + 127) / 128};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-  return launch_gemm<BN, STAGES, 1, kSplitB>(h, dim3(h->num_sms), L.tm_wgu8, h->tm_xg[3], d / 64, 1, s, e, nullptr,
-                                             &h->tm_xg_lo[3]);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu8, h->tm_xg[3], d / 64, 1, s, e, nullptr,
+                                               &h->tm_xg_lo[3], &h->tok_xg);
 }
 
+template <int BN, int ACC, int STAGES>
 cudaError_t moe_down_w8(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
   const int F = c.ffn_dim, d = c.d_model;
-  constexpr int BN = kMoeChunk;
-  constexpr int STAGES = 4;
-  PersistentGroupedSched<1, true> s{h->d_tok_maps + 8, h->offsets, h->routed, h->n_routed, h->chunk_prefix, d,
+  PersistentGroupedSched<1, true> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d,
                                     d / 128, BN, L.ed, 0, d / 128, (F + 127) / 128};
   EpiDown<BN> e{h->obuf, d};
-  return launch_gemm<BN, STAGES, 1, kSplitB>(h, dim3(h->num_sms), L.tm_wd8, h->tm_h[3], F / 64, 1, s, e, nullptr,
-                                             &h->tm_h_lo[3]);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd8, h->tm_h[3], F / 64, 1, s, e, nullptr,
+                                               &h->tm_h_lo[3], &h->tok_h);
 }
 
-// Grouped expert GEMMs of one layer. gate/up: one weight tile per item, two accumulator
-// buffers; down: two weight tiles per item sharing the token chunk (its 22 m tiles leave
-// enough items to spread over the SMs), or one with DLLM_MOE_PAIR=0.
-cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int l, uint32_t timed) {
+// Grouped expert GEMMs of one layer over chunks of `chunk` tokens (moe_chunk). gate/up:
+// one weight tile per item, two accumulator buffers; down at 64-token chunks: two weight
+// tiles per item sharing the token chunk (its 22 m tiles leave enough items to spread
+// over the SMs), or one with DLLM_MOE_PAIR=0.
+cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int l, int chunk, uint32_t timed) {
   cudaError_t r;
+  const bool wide = chunk == 128;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
-  r = h->w8 ? moe_gate_up_w8(h, L) : moe_gate_up<1, 2>(h, L);
+  if (h->w8)
+    r = wide ? moe_gate_up_w8<128, 1, 4>(h, L) : moe_gate_up_w8<64, 2, 6>(h, L);
+  else
+    r = wide ? moe_gate_up<128, 1, 2>(h, L) : moe_gate_up<64, 1, 2>(h, L);
   if (r != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
-  r = h->w8 ? moe_down_w8(h, L) : h->moe_pair ? moe_down<2, 1>(h, L) : moe_down<1, 2>(h, L);
+  if (h->w8)
+    r = wide ? moe_down_w8<128, 1, 4>(h, L) : moe_down_w8<64, 2, 6>(h, L);
+  else if (wide)
+    r = moe_down<128, 1, 2>(h, L);
+  else
+    r = h->moe_pair ? moe_down<64, 2, 2>(h, L) : moe_down<64, 1, 2>(h, L);
   if (r != cudaSuccess) return r;
   return tmark(h, timed, DLLM_TIMING_DOWN, l, 1);
 }
@@ -625,12 +643,13 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
   const int d = c.d_model;
   const int N = T * h->k;
   for (int l = 0; l < c.n_layers; ++l) {
+    NvtxRange nvtx_("layer");
     const LayerW& L = h->L[l];
     bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
     bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
     if (l == 0) {   // later layers get this norm from the previous layer's combine
       CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.attn_norm, d, c.rms_eps, h->y,
-                  h->y_lo, h->rstd));
+                  h->y_lo, h->y_lo2, h->rstd));
       h->launches++;
     }
     CK(tmark(h, timed, DLLM_TIMING_QKV, l, 0));
@@ -644,7 +663,7 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 0));
     CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo,
-                h->rstd));
+                (bf16_t*)nullptr, h->rstd));
     h->launches++;
     if (!h->dense) {
       if (h->router_tc) {
@@ -673,18 +692,19 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
       h->launches++;
     }
     CK(launch_k(h, permute_kernel, dim3(1), dim3(1024), 0, h->tk_idx, N, h->k, h->E, h->offsets, h->slot_of,
-                h->row_token, h->routed, h->n_routed, h->chunk_prefix, kMoeChunk,
+                h->row_token, h->routed, h->n_routed, h->chunk_prefix, moe_chunk(N, h->E),
                 timed ? h->routed_stat + l : nullptr));
     CK(launch_k(h, gather_rows_kernel, dim3(N), dim3(std::min(1024, (d / 8 + 31) / 32 * 32)), 0, h->y, h->y_lo,
                 h->row_token, N, d, h->xg, h->xg_lo));
     h->launches += 2;
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 1));
-    CK(moe_gemms(h, L, l, timed));
+    CK(moe_gemms(h, L, l, moe_chunk(N, h->E), timed));
     CK(tmark(h, timed, DLLM_TIMING_NORM, l, 0));
     const float* next_gain = l + 1 < c.n_layers ? h->L[l + 1].attn_norm : final_gain;
+    // the next layer's attention norm feeds the QKV projection: three bf16 terms
     if (next_gain)
       CK(launch_k(h, combine_norm_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k,
-                  d, next_gain, c.rms_eps, h->y, h->y_lo));
+                  d, next_gain, c.rms_eps, h->y, h->y_lo, l + 1 < c.n_layers ? h->y_lo2 : (bf16_t*)nullptr));
     else
       CK(launch_k(h, combine_kernel, dim3(T), dim3(256), 0, h->x, h->obuf, h->slot_of, h->tk_w, h->k, d));
     h->launches++;
@@ -861,8 +881,8 @@ int validate(const dllm_config* c, std::string* why) {
   if (c->max_batch < 1 || c->max_ctx < c->canvas + 1) return bad("max_batch >= 1 and max_ctx > canvas");
   if (c->weight_dtype != DLLM_WEIGHTS_F32 && c->weight_dtype != DLLM_WEIGHTS_BF16) return bad("weight_dtype");
   if (c->expert_format != DLLM_EXPERTS_BF16 && c->expert_format != DLLM_EXPERTS_FP8) return bad("expert_format");
-  if (c->expert_format == DLLM_EXPERTS_FP8 && c->n_experts > 0 && (c->ffn_dim % 128 || c->d_model % 128))
-    return bad("FP8 experts need ffn_dim and d_model multiples of 128");
+  if (c->expert_format == DLLM_EXPERTS_FP8 && c->ffn_dim > 128 * kConvMaxColBlocks)
+    return bad("FP8 experts: ffn_dim at most 8192");
   return DLLM_OK;
 }
 
@@ -932,15 +952,9 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   }
   // tensor-core attention for canvas passes when a query tile of 128 rows holds whole
   // GQA groups (DLLM_ATTN_LEGACY=1 keeps the warp-MMA kernel, for comparisons)
-  h->attn_tc = (128 % (H / Hkv) == 0) && !getenv("DLLM_ATTN_LEGACY");
-  if (const char* m = getenv("DLLM_OPROJ_SWAP")) h->oproj_swap = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_QKV_SPLITK")) h->qkv_splitk = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_PREFILL_TC")) h->prefill_tc = atoi(m) != 0;
+  h->attn_tc = 128 % (H / Hkv) == 0;
   if (const char* m = getenv("DLLM_MOE_PAIR")) h->moe_pair = atoi(m) != 0;
   h->router_tc = !h->dense && h->E % 32 == 0;
-  if (const char* m = getenv("DLLM_PDL")) h->pdl = atoi(m) != 0;
-  if (const char* m = getenv("DLLM_ROUTER_TC")) h->router_tc = h->router_tc && atoi(m) != 0;
-  if (const char* m = getenv("DLLM_ROUTER_KS")) h->router_ks = atoi(m);
   h->w8 = !h->dense && c.expert_format == DLLM_EXPERTS_FP8;
   const long qd = (long)H * hd, kvd = (long)Hkv * hd;
 
@@ -1045,6 +1059,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   DA(h->x, (size_t)T * d);
   DA(h->y, (size_t)T * d);
   DA(h->y_lo, (size_t)T * d);
+  DA(h->y_lo2, (size_t)T * d);
   DA(h->rstd, T);
   DA(h->q, (size_t)T * qd);
   DA(h->ao, (size_t)T * qd);
@@ -1114,8 +1129,7 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   bool ok = true;
   ok &= make_tmap(&h->tm_y, h->y, T, d, 128);
   ok &= make_tmap(&h->tm_y_lo, h->y_lo, T, d, 128);
-  ok &= make_tmap(&h->tm_ao, h->ao, T, qd, 128);
-  ok &= make_tmap(&h->tm_ao_lo, h->ao_lo, T, qd, 128);
+  ok &= make_tmap(&h->tm_y_lo2, h->y_lo2, T, d, 128);
   ok &= make_tmap(&h->tm_ao64, h->ao, T, qd, 64);
   ok &= make_tmap(&h->tm_ao64_lo, h->ao_lo, T, qd, 64);
   ok &= make_tmap(&h->tm_head, h->head, V, d, 256);
@@ -1146,17 +1160,11 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     }
   }
   if (!ok) return fail(h, DLLM_E_CUDA, "cuTensorMapEncodeTiled failed");
-  {
-    // the grouped GEMMs read their token-operand maps from device memory
-    CUtensorMap maps[16];
-    for (int i = 0; i < 4; ++i) {
-      maps[i] = h->tm_xg[i];
-      maps[4 + i] = h->tm_xg_lo[i];
-      maps[8 + i] = h->tm_h[i];
-      maps[12 + i] = h->tm_h_lo[i];
-    }
-    DA(h->d_tok_maps, 16);
-    CK(cudaMemcpy(h->d_tok_maps, maps, sizeof(maps), cudaMemcpyHostToDevice));
+  for (int i = 0; i < 4; ++i) {
+    h->tok_xg.m[i] = h->tm_xg[i];
+    h->tok_xg.m[4 + i] = h->tm_xg_lo[i];
+    h->tok_h.m[i] = h->tm_h[i];
+    h->tok_h.m[4 + i] = h->tm_h_lo[i];
   }
   CK(cudaFuncSetAttribute(reinterpret_cast<const void*>(router_kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
                           kRouterTok * d * (int)sizeof(float)));
@@ -1234,12 +1242,14 @@ int dllm_create(const dllm_config* cfg, const void* weights, size_t weight_bytes
 
 int dllm_prefill(dllm_handle* h, int req, const int32_t* prompt, int n) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_prefill");
   return prefill_impl(h, req, prompt, n, false);
 }
 
 int dllm_denoise_step(dllm_handle* h, int req_count, int32_t* canvas, uint8_t* mask, const dllm_policy* policy,
                       int step, int max_steps, float* conf_out, int32_t* argmax_out, int32_t* remaining_out) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_denoise_step");
   if (!canvas || !mask) return fail(h, DLLM_E_INVAL, "canvas/mask NULL");
   int r = check_requests(h, req_count);
   if (r) return r;
@@ -1265,6 +1275,7 @@ int dllm_denoise_step(dllm_handle* h, int req_count, int32_t* canvas, uint8_t* m
 int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm_policy* policy, int32_t* canvas_out,
                         int* steps_taken) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_generate_block");
   int r = check_requests(h, req_count);
   if (r) return r;
   if ((r = check_policy(h, policy, max_steps))) return r;
@@ -1306,6 +1317,7 @@ int dllm_generate_block(dllm_handle* h, int req_count, int max_steps, const dllm
 
 int dllm_append_kv(dllm_handle* h, int req_count, const int32_t* canvas) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_append_kv");
   int r = check_requests(h, req_count);
   if (r) return r;
   const int C = h->c.canvas, B = req_count;
@@ -1320,6 +1332,7 @@ int dllm_append_kv(dllm_handle* h, int req_count, const int32_t* canvas) {
 
 int dllm_append_kv_approx(dllm_handle* h, int req_count) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_append_kv_approx");
   int r = check_requests(h, req_count);
   if (r) return r;
   for (int b = 0; b < req_count; ++b)
@@ -1335,6 +1348,7 @@ int dllm_append_kv_approx(dllm_handle* h, int req_count) {
 int dllm_generate(dllm_handle* h, int req_count, const int32_t* prompts, int n_prompt, int n_canvases, int max_steps,
                   const dllm_policy* policy, int32_t* tokens_out, int* steps_out) {
   if (!h) return DLLM_E_INVAL;
+  NvtxRange nvtx_("dllm_generate");
   if (!prompts || !tokens_out || n_canvases < 1) return fail(h, DLLM_E_INVAL, "bad arguments");
   if (req_count < 1 || req_count > h->c.max_batch) return fail(h, DLLM_E_INVAL, "req_count out of range");
   const int C = h->c.canvas;

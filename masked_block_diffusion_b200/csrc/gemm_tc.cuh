@@ -96,9 +96,9 @@ struct DenseSplitKSched {
 //
 // The MMA width follows each chunk's token count (kDynN): a chunk of n tokens loads only
 // n16 = n rounded up to 16 rows of the token pair, composed from boxes of 128, 64, 32
-// and 16 rows (tok_maps: [hi 16, 32, 64, 128 | lo 16, 32, 64, 128], tensor maps in
-// global memory), stacked as [hi n16 rows | lo n16 rows], and one MMA of N = 2 n16 reads
-// both. An expert with few tokens then costs its weight bytes and little else.
+// and 16 rows (the kernel's TokMaps parameter), stacked as [hi n16 rows | lo n16 rows],
+// and one MMA of N = 2 n16 reads both. An expert with few tokens then costs its weight
+// bytes and little else.
 //
 // W8: the weights are FP8 E4M3 with one power-of-two scale 2^e per 128 x 128 tile of
 // each original expert matrix (exps, int8). Converter warps turn each staged FP8 tile
@@ -114,7 +114,6 @@ struct PersistentGroupedSched {
   static constexpr bool kDynN = true;
   static constexpr bool kW8 = W8;
   static constexpr int kMPerItem = MPI;
-  const CUtensorMap* tok_maps;   // 8 token-operand maps (see above), device memory
   const int* offsets;        // [E+1] token ranges per expert
   const int* routed;         // [E] experts with at least one token, ascending
   const int* n_routed;       // [1]
@@ -191,6 +190,12 @@ struct PersistentGroupedSched {
   }
 };
 
+// The token-operand tensor maps of a dynamic-width grouped GEMM, passed by value as a
+// kernel parameter: [hi boxes of 16, 32, 64, 128 rows | lo boxes of the same heights].
+struct alignas(64) TokMaps {
+  CUtensorMap m[8];
+};
+
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
 }
@@ -200,17 +205,22 @@ __host__ __device__ constexpr int tmem_alloc_cols(int n) {
   return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
 }
 
-// Threads of a GEMM CTA: producer, MMA, 4 epilogue warps, and for W8 4 converter warps.
+// Threads of a GEMM CTA: producer, MMA, 4 epilogue warps, and for W8 8 converter warps
+// (two per TMEM lane quarter, each on half of a row's 64 k values).
 template <class Sched>
-__host__ __device__ constexpr int gemm_threads() { return Sched::kW8 ? 320 : 192; }
+__host__ __device__ constexpr int gemm_threads() { return Sched::kW8 ? 448 : 192; }
+constexpr int kConvThreads = 256;
+constexpr int kConvMaxColBlocks = 64;   // W8: 128-column scale blocks per weight row (K <= 8192)
 
 // Operand splitting. Weights are bf16; an activation operand can be carried as a pair
 // of bf16 tensors (hi = bf16(v), lo = bf16(v - hi)) so that products keep about 16
 // mantissa bits of the activation. kSplitNone: plain. kSplitA: A is a (hi, lo) pair and
 // every k step issues two MMAs into the same accumulator. kSplitB: B is the pair; its
 // hi and lo rows sit next to each other in the stage, one MMA of width 2 BN reads both,
-// and the epilogue first adds the accumulator's two column halves.
-enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2 };
+// and the epilogue first adds the accumulator's two column halves. kSplitA3: A is a
+// triple (hi, mid, lo) carrying all 24 bits of an fp32 value, three MMAs per k step (the
+// third map travels in the TokMaps parameter's first slot).
+enum SplitMode : int { kSplitNone = 0, kSplitA = 1, kSplitB = 2, kSplitA3 = 3 };
 
 template <int BN, int STAGES, int SPLIT, class Epi, class Sched = DenseSched>
 struct GemmSmem {
@@ -218,11 +228,13 @@ struct GemmSmem {
   static constexpr int kAtile = Sched::kW8 ? 128 * 64 : 128 * 64 * 2;
   static constexpr int kA = Sched::kMPerItem * kAtile;     // the item's A tiles
   static constexpr int kB = BN * 64 * 2;
-  static constexpr int kA2 = SPLIT == kSplitA ? kA : 0;
+  static constexpr int kA2 = (SPLIT == kSplitA || SPLIT == kSplitA3) ? kA : 0;
+  static constexpr int kA3 = SPLIT == kSplitA3 ? kA : 0;
   static constexpr int kB2 = SPLIT == kSplitB ? kB : 0;
-  static constexpr int kStageBytes = kA + kA2 + kB + kB2;   // TMA bytes per stage
+  static constexpr int kStageBytes = kA + kA2 + kA3 + kB + kB2;   // TMA bytes per stage
   static constexpr int kOffA2 = STAGES * kA;
-  static constexpr int kOffB = kOffA2 + STAGES * kA2;
+  static constexpr int kOffA3 = kOffA2 + STAGES * kA2;
+  static constexpr int kOffB = kOffA3 + STAGES * kA3;
   // kSplitB keeps each stage's B pair adjacent ([hi rows | lo rows]), so that one MMA
   // with N = 2 BN reads both: the A tile is then read from shared memory once per k step
   // instead of once per half.
@@ -312,13 +324,14 @@ template <int BN, int STAGES, int ACC_BUFS, int SPLIT, class Sched, class Epi>
 __global__ void __launch_bounds__(gemm_threads<Sched>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_a2,
                const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_b2,
-               int k_blocks, int a_stream_first, Sched sched_in, Epi epi, int* err) {
+               const __grid_constant__ TokMaps tok, int k_blocks, int a_stream_first, Sched sched_in, Epi epi,
+               int* err) {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is a multiple of 16 in [16, 256]");
   using L = GemmSmem<BN, STAGES, SPLIT, Epi, Sched>;
   constexpr int kAccN = SPLIT == kSplitB ? 2 * BN : BN;   // kSplitB: columns [0, BN) hi, [BN, 2 BN) lo
   static_assert(kAccN <= 256, "UMMA N");
   constexpr int MPI = Sched::kMPerItem;                   // accumulators per work item
-  static_assert(MPI == 1 || SPLIT != kSplitA, "several m tiles per item share B only");
+  static_assert(MPI == 1 || (SPLIT != kSplitA && SPLIT != kSplitA3), "several m tiles per item share B only");
   constexpr int kCols = tmem_cols_for(kAccN);
   constexpr bool W8 = Sched::kW8;
   static_assert(!W8 || (SPLIT == kSplitB && Sched::kDynN), "FP8 weights: grouped expert tiles only");
@@ -334,6 +347,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sA2 = smem + L::kOffA2;
+  uint8_t* sA3 = smem + L::kOffA3;
   uint8_t* sB = smem + L::kOffB;
   uint8_t* sB2 = smem + L::kOffB2;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -363,12 +377,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     mbar_init(drain, 1);
     if (KS > 1) mbar_init(peer_ready, 128 * (KS - 1));
     if (W8)
-      for (int s = 0; s < STAGES; ++s) mbar_init(&conv_full[s], 128);
+      for (int s = 0; s < STAGES; ++s) mbar_init(&conv_full[s], kConvThreads);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tma_a);
     tma_prefetch_desc(&tma_b);
-    if (SPLIT == kSplitA) tma_prefetch_desc(&tma_a2);
+    if (SPLIT == kSplitA || SPLIT == kSplitA3) tma_prefetch_desc(&tma_a2);
+    if (SPLIT == kSplitA3) tma_prefetch_desc(&tok.m[0]);
     if (SPLIT == kSplitB) tma_prefetch_desc(&tma_b2);
   }
   if (warp == 1) {
@@ -394,7 +409,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
     if constexpr (Sched::kDynN)
-      for (int i = 0; i < 8; ++i) tma_prefetch_desc(sched.tok_maps + i);
+      for (int i = 0; i < 8; ++i) tma_prefetch_desc(&tok.m[i]);
     const uint64_t pol_first = policy_evict_first();
     const uint64_t pol_last = policy_evict_last();
     const uint64_t pol_a = a_stream_first ? pol_first : pol_last;
@@ -408,7 +423,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         if constexpr (Sched::kDynN) {
-          static_assert(SPLIT == kSplitB && BN == 128, "dynamic N: stacked token pair, up to 128 rows");
+          static_assert(SPLIT == kSplitB && BN <= 128 && BN % 16 == 0, "dynamic N: stacked token pair, <= 128 rows");
           const int n16 = t.n_cols;
           mbar_arrive_expect_tx(&full[stage], t.m_count * L::kAtile + 2 * n16 * 128);
           for (int u = 0; u < t.m_count; ++u)
@@ -422,7 +437,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
             for (int bi = 3; bi >= 0; --bi) {
               const int rows = 16 << bi;
               if ((n16 - off) & rows) {
-                tma_load_2d(dst + (half * n16 + off) * 128, sched.tok_maps + half * 4 + bi, &full[stage], kb * 64,
+                tma_load_2d(dst + (half * n16 + off) * 128, &tok.m[half * 4 + bi], &full[stage], kb * 64,
                             t.b_row + off, pol_b);
                 off += rows;
               }
@@ -432,7 +447,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes - (MPI - t.m_count) * L::kAtile);
           for (int u = 0; u < t.m_count; ++u)
             tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
-          if (SPLIT == kSplitA) tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
+          if (SPLIT == kSplitA || SPLIT == kSplitA3)
+            tma_load_2d(sA2 + stage * L::kA2, &tma_a2, &full[stage], kb * 64, t.a_row, pol_a);
+          if (SPLIT == kSplitA3) tma_load_2d(sA3 + stage * L::kA3, &tok.m[0], &full[stage], kb * 64, t.a_row, pol_a);
           tma_load_2d(sB + stage * L::kBStage, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
           if (SPLIT == kSplitB)
             tma_load_2d(sB2 + stage * L::kBStage, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
@@ -476,6 +493,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         const uint32_t a0 = smem_u32(sA + stage * L::kA);
         const uint32_t b0 = smem_u32(sB + stage * L::kBStage);
         const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
+        const uint32_t a2 = smem_u32(sA3 + stage * L::kA3);
         if constexpr (W8) {
           // A: the converted bf16 tile in tensor memory (8 columns per 16 k)
           const uint32_t at = tmem_base + kACol + stage * MPI * 32;
@@ -491,8 +509,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
           for (int kk = 0; kk < 4; ++kk) {
             umma_bf16(d_tmem, sdesc_k_sw128(a0 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc,
                       (kb != kb_begin || kk != 0) ? 1u : 0u);
-            if (SPLIT == kSplitA)
+            if (SPLIT == kSplitA || SPLIT == kSplitA3)
               umma_bf16(d_tmem, sdesc_k_sw128(a1 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc, 1);
+            if (SPLIT == kSplitA3)
+              umma_bf16(d_tmem, sdesc_k_sw128(a2 + kk * 32), sdesc_k_sw128(b0 + kk * 32), idesc, 1);
 #pragma unroll
             for (int u = 1; u < MPI; ++u)
               if (u < mc)
@@ -513,37 +533,47 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     umma_commit(drain);
     mbar_drain(drain, 0);
   } else if (W8 && warp >= 6) {
-    // ---------------- converters (W8): FP8 tile -> bf16 in tensor memory, one row per thread
+    // ---------------- converters (W8): FP8 tile -> bf16 in tensor memory. Warp 6 + w
+    // takes TMEM lane quarter w % 4 (row r = 32 (w % 4) + lane) and k values
+    // 32 (w / 4) .. 32 (w / 4) + 31 of the stage's 64.
     if constexpr (W8) {
+      static_assert(MPI == 1, "W8: one weight tile per item");
+      const int cw = warp - 6;
       const int q = warp & 3;
       const int r = q * 32 + lane;
+      const int kh = cw >> 2;                       // which 32 k values
+      const int ncb = sched.exp_ncb;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
         const Tile t = sched.tile(j);
+        // the scales of this warp's rows for the whole tile, one column block per lane
+        // (two registers: blocks lane and lane + 32), fetched once and shuffled per k block
+        const float sc_lo = lane < ncb ? ldexpf(1.0f, sched.exponent(t, 0, r, 2 * lane)) : 1.0f;
+        const float sc_hi = lane + 32 < ncb ? ldexpf(1.0f, sched.exponent(t, 0, r, 2 * (lane + 32))) : 1.0f;
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) { ok = false; break; }
-          for (int u = 0; u < t.m_count; ++u) {
-            // the FP8 tile was stored with the 64-byte swizzle: 16-byte chunk c of row r
-            // sits at chunk c ^ ((r >> 1) & 3) of its 64-byte row
-            const uint8_t* row = sA + stage * L::kA + u * L::kAtile + r * 64;
-            uint4 v[4];
-  #pragma unroll
-            for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + ((c ^ ((r >> 1) & 3)) << 4));
-            const float sc = ldexpf(1.0f, sched.exponent(t, u, r, kb));
-            uint32_t o[32];
-  #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-  #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                o[c * 8 + 2 * i] = e4m3x2_to_bf16x2((uint16_t)(w[i] & 0xFFFFu), sc);
-                o[c * 8 + 2 * i + 1] = e4m3x2_to_bf16x2((uint16_t)(w[i] >> 16), sc);
-              }
+          // the FP8 tile was stored with the 64-byte swizzle: 16-byte chunk c of row r sits
+          // at chunk c ^ ((r >> 1) & 3) of its 64-byte row
+          const uint8_t* row = sA + stage * L::kA + r * 64;
+          uint4 v[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            v[c] = *reinterpret_cast<const uint4*>(row + (((2 * kh + c) ^ ((r >> 1) & 3)) << 4));
+          const int cb = kb >> 1;
+          const float sc = __shfl_sync(0xffffffffu, cb < 32 ? sc_lo : sc_hi, cb & 31);
+          uint32_t o[16];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              o[c * 8 + 2 * i] = e4m3x2_to_bf16x2((uint16_t)(w[i] & 0xFFFFu), sc);
+              o[c * 8 + 2 * i + 1] = e4m3x2_to_bf16x2((uint16_t)(w[i] >> 16), sc);
             }
-            tmem_st32_nowait(tmem_at(tmem_base + kACol + (stage * MPI + u) * 32, q * 32, 0), o);
           }
+          tmem_st16_nowait(tmem_at(tmem_base + kACol + stage * 32 + kh * 16, q * 32, 0), o);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&conv_full[stage]);
@@ -722,43 +752,6 @@ struct EpiQKV {
           *reinterpret_cast<uint4*>(dst + c) = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
                                                           pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
         }
-      }
-    }
-  }
-};
-
-// x[row][col] += D: the attention output projection with its residual add.
-template <int BN>
-struct EpiResidual {
-  static constexpr int kSmemBytes = 0;
-  float* x;
-  int ldx;
-  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
-    static_assert(BN % 64 == 0, "64-column groups");
-    float* row = x + (long)(t.a_row + r) * ldx + t.b_row;
-    const bool valid = r < t.m_valid;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 64) {
-      // the row's 64 residual values are loaded together, then the accumulator
-      float4 o[16];
-      float4* p = reinterpret_cast<float4*>(row + c0);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = valid ? p[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[16];
-        tmem_ld16(taddr + c0 + 16 * q, v);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          o[4 * q + i].x += v[4 * i + 0];
-          o[4 * q + i].y += v[4 * i + 1];
-          o[4 * q + i].z += v[4 * i + 2];
-          o[4 * q + i].w += v[4 * i + 3];
-        }
-      }
-      if (valid) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) p[i] = o[i];
       }
     }
   }

@@ -34,10 +34,31 @@ __global__ void embed_kernel(const bf16_t* __restrict__ emb, const int32_t* __re
 
 // ---------------------------------------------------------------- a2/a6/a12: RMSNorm
 
-// v = x * rsqrt(mean(x^2) + eps) * g, written as the bf16 pair y = bf16(v),
-// y_lo = bf16(v - y) (y_lo may be NULL); rstd[t] kept for the fp32 router.
+// Writes v as bf16 terms: y = bf16(v), y_lo = bf16(v - y) and, when y_lo2 is given, the
+// third term y_lo2 = bf16(v - y - y_lo), so that y + y_lo + y_lo2 carries all of v's fp32
+// bits (the QKV projection's operand; the other GEMMs read the (y, y_lo) pair).
+DLLM_DEV void store_norm_terms(bf16_t* y, bf16_t* y_lo, bf16_t* y_lo2, long t, int d, int c, float4 v) {
+  uint32_t h0, l0, h1, l1;
+  if (y_lo2) {
+    uint32_t m0, m1;
+    split3_bf16x2(v.x, v.y, h0, m0, l0);
+    split3_bf16x2(v.z, v.w, h1, m1, l1);
+    reinterpret_cast<uint2*>(y + t * d)[c] = make_uint2(h0, h1);
+    reinterpret_cast<uint2*>(y_lo + t * d)[c] = make_uint2(m0, m1);
+    reinterpret_cast<uint2*>(y_lo2 + t * d)[c] = make_uint2(l0, l1);
+    return;
+  }
+  split_bf16x2(v.x, v.y, h0, l0);
+  split_bf16x2(v.z, v.w, h1, l1);
+  reinterpret_cast<uint2*>(y + t * d)[c] = make_uint2(h0, h1);
+  reinterpret_cast<uint2*>(y_lo + t * d)[c] = make_uint2(l0, l1);
+}
+
+// v = x * rsqrt(mean(x^2) + eps) * g, written as bf16 terms (store_norm_terms); rstd[t]
+// kept for the fp32 router.
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
-                               bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo, float* __restrict__ rstd) {
+                               bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo, bf16_t* __restrict__ y_lo2,
+                               float* __restrict__ rstd) {
   pdl_begin();
   const int t = blockIdx.x;
   const float4* xr = reinterpret_cast<const float4*>(x + (long)t * d);
@@ -59,15 +80,9 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
   const float r = rsqrtf(red[0] / (float)d + eps);
   if (threadIdx.x == 0 && rstd != nullptr) rstd[t] = r;
   const float4* gr = reinterpret_cast<const float4*>(g);
-  uint2* yr = reinterpret_cast<uint2*>(y + (long)t * d);
-  uint2* yl = y_lo ? reinterpret_cast<uint2*>(y_lo + (long)t * d) : nullptr;
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    float4 v = xr[c], gg = gr[c];
-    uint32_t h0, l0, h1, l1;
-    split_bf16x2(v.x * r * gg.x, v.y * r * gg.y, h0, l0);
-    split_bf16x2(v.z * r * gg.z, v.w * r * gg.w, h1, l1);
-    yr[c] = make_uint2(h0, h1);
-    if (yl) yl[c] = make_uint2(l0, l1);
+    const float4 v = xr[c], gg = gr[c];
+    store_norm_terms(y, y_lo, y_lo2, t, d, c, make_float4(v.x * r * gg.x, v.y * r * gg.y, v.z * r * gg.z, v.w * r * gg.w));
   }
 }
 
@@ -387,7 +402,8 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x
                                                            const int32_t* __restrict__ slot_of,
                                                            const float* __restrict__ gate, int k, int d,
                                                            const float* __restrict__ g, float eps,
-                                                           bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo) {
+                                                           bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo,
+                                                           bf16_t* __restrict__ y_lo2) {
   pdl_begin();
   const int t = blockIdx.x;
   float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
@@ -415,15 +431,9 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x
   __syncthreads();
   const float r = rsqrtf(red[0] / (float)d + eps);
   const float4* gr = reinterpret_cast<const float4*>(g);
-  uint2* yr = reinterpret_cast<uint2*>(y + (long)t * d);
-  uint2* yl = reinterpret_cast<uint2*>(y_lo + (long)t * d);
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     const float4 v = xr[c], gg = gr[c];   // this thread's own writes above
-    uint32_t h0, l0, h1, l1;
-    split_bf16x2(v.x * r * gg.x, v.y * r * gg.y, h0, l0);
-    split_bf16x2(v.z * r * gg.z, v.w * r * gg.w, h1, l1);
-    yr[c] = make_uint2(h0, h1);
-    yl[c] = make_uint2(l0, l1);
+    store_norm_terms(y, y_lo, y_lo2, t, d, c, make_float4(v.x * r * gg.x, v.y * r * gg.y, v.z * r * gg.z, v.w * r * gg.w));
   }
 }
 

@@ -50,7 +50,8 @@ Readings where the pages are silent (all listed in the design notes):
    and V also stay in the KV cache from pass to pass). The operands formed inside an
    operation from fp32 arithmetic (normalised activations, softmax probabilities,
    attention output, SwiGLU output) are kept exact here; the kernels carry them as a
-   bf16 (hi, lo) pair, more precisely than bf16 operands. Residual stream, router and
+   bf16 (hi, lo) pair, and the QKV projection's input as three bf16 terms, more
+   precisely than bf16 operands. Residual stream, router and
    softmax statistics are fp64; router and LM-head logits are rounded to fp32 before
    the top-k / argmax decision, and conf to fp32 before commit ranking;
 11. token-to-token editing (What changes, section 4.3, LLaDA2.1: the model may revise

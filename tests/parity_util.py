@@ -66,12 +66,19 @@ def commit_margin(conf: np.ndarray, mask: np.ndarray, n: int, policy: Policy) ->
     return m
 
 
-def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, stats=None):
-    """Replays every oracle step on the GPU and checks the decisions and values."""
+def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, stats=None, margin: float = MARGIN):
+    """Replays every oracle step on the GPU and checks the decisions and values.
+
+    Decisions whose oracle margin exceeds `margin` must agree. With a margin above 1e-3,
+    decisions with margins between 1e-3 and `margin` that differ are counted in
+    stats["near_flips"] instead (the caller bounds them).
+    """
     C = cfg.canvas
     stats = stats if stats is not None else {"route_pinned": 0, "route_total": 0, "arg_pinned": 0,
                                              "arg_total": 0, "commit_pinned": 0, "steps": 0, "edits": 0,
-                                             "edit_pinned": 0}
+                                             "edit_pinned": 0, "near_flips": 0, "near_total": 0}
+    stats.setdefault("near_flips", 0)
+    stats.setdefault("near_total", 0)
     pol = make_policy(policy.kind, policy.k, policy.tau, policy.floor, policy.t2t, policy.edit_tau)
     den.set_debug(True)
     for e in orc_trace:
@@ -101,23 +108,42 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
             for l in range(cfg.n_layers):
                 lg = rec["router_logits"][l]
                 srt = -np.sort(-lg, axis=1)
-                margin = srt[:, k - 1] - srt[:, k]
-                sel = margin > MARGIN
+                rmargin = srt[:, k - 1] - srt[:, k]
+                sel = rmargin > margin
+                near = (rmargin > MARGIN) & ~sel
                 gi = den.debug_read(2, l, (C, k), np.int32)
                 ri = rec["topk_idx"][l]
                 same = np.array([set(gi[t]) == set(ri[t]) for t in range(C)])
                 bad = np.nonzero(sel & ~same)[0]
-                assert bad.size == 0, f"step {e['step']} layer {l}: routing differs at tokens {bad[:8]}"
+                if bad.size:
+                    gl = den.debug_read(1, l, (C, cfg.n_experts), np.float32)
+                    xl = den.debug_read(5, l - 1, (C, cfg.d_model), np.float32) if l > 0 else None
+                    lines = []
+                    for t in bad[:4]:
+                        order = np.argsort(-lg[t], kind="stable")[:k + 1]
+                        lines.append(f"token {t}: margin {margin[t]:.3e}; oracle logits {lg[t][order]} "
+                                     f"gpu logits {gl[t][order]} (experts {order}); gpu picked {sorted(gi[t])}")
+                        if xl is not None:
+                            xr = rec["x"][l - 1][t]
+                            lines.append(f"  input row rel err {np.abs(xl[t] - xr).max() / np.abs(xr).max():.3e}")
+                    raise AssertionError(f"step {e['step']} layer {l}: routing differs at tokens {bad[:8]}\n"
+                                         + "\n".join(lines))
                 stats["route_pinned"] += int(sel.sum())
                 stats["route_total"] += C
+                stats["near_flips"] += int((near & ~same).sum())
+                stats["near_total"] += int(near.sum())
                 gl = den.debug_read(1, l, (C, cfg.n_experts), np.float32)
                 assert np.abs(gl - lg).max() <= REL * np.abs(lg).max()
 
         # LM head: conf and argmax
         assert np.all(np.abs(conf / e["conf"] - 1.0) <= REL), f"step {e['step']}: conf"
-        lm_sel = rec["logit_margin"] > MARGIN
+        lm_sel = rec["logit_margin"] > margin
+        lm_near = (rec["logit_margin"] > MARGIN) & ~lm_sel
         bad = np.nonzero(lm_sel & (arg != e["argmax"]))[0]
-        assert bad.size == 0, f"step {e['step']}: argmax differs at {bad[:8]}"
+        assert bad.size == 0, (f"step {e['step']}: argmax differs at {bad[:8]} (margins "
+                               f"{rec['logit_margin'][bad[:8]]}, conf rel err {(conf / e['conf'] - 1)[bad[:8]]})")
+        stats["near_flips"] += int((lm_near & (arg != e["argmax"])).sum())
+        stats["near_total"] += int(lm_near.sum())
         stats["arg_pinned"] += int(lm_sel.sum())
         stats["arg_total"] += C
 
@@ -126,9 +152,13 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
         n = int(e["commit"].sum())
         assert int(gpu_commit.sum()) == n, f"step {e['step']}: commit count {gpu_commit.sum()} vs {n}"
         assert int(rem.cpu().numpy()[0]) == int(old_mask.sum()) - n
-        if commit_margin(e["conf"], old_mask, n, policy) > MARGIN:
+        cm = commit_margin(e["conf"], old_mask, n, policy)
+        if cm > margin:
             assert np.array_equal(gpu_commit, e["commit"]), f"step {e['step']}: commit set differs"
             stats["commit_pinned"] += 1
+        elif cm > MARGIN:
+            stats["near_flips"] += int(not np.array_equal(gpu_commit, e["commit"]))
+            stats["near_total"] += 1
         # newly committed positions hold the pass's argmax
         assert np.array_equal(new_canvas[gpu_commit], arg[gpu_commit])
         # earlier commits: untouched (M2T); with T2T, re-written exactly where the oracle
@@ -138,7 +168,7 @@ def compare_trace(cfg, orc_trace, den: Denoiser, policy: Policy, s_max: int, sta
         gpu_edit = committed & (new_canvas != e["canvas"])
         if policy.t2t:
             pinned = committed & lm_sel & (np.abs(np.log(e["conf"].astype(np.float64))
-                                                  - math.log(policy.edit_tau)) > MARGIN)
+                                                  - math.log(policy.edit_tau)) > margin)
             bad = np.nonzero(pinned & (gpu_edit != e["edit"]))[0]
             assert bad.size == 0, f"step {e['step']}: edit set differs at {bad[:8]}"
             assert np.array_equal(new_canvas[gpu_edit], arg[gpu_edit])

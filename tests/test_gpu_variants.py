@@ -4,19 +4,13 @@ test_gpu_parity.py covers the default selections. Here each alternative is switc
 through the environment variable the engine reads when a handle is created, and the
 same step-by-step comparison with the oracle runs on a two-layer model:
 
-- DLLM_OPROJ_SWAP=0: O projection with tokens as M (weights as N) instead of swapped;
 - DLLM_MOE_PAIR=0: one weight tile per grouped down work item instead of two;
-- DLLM_ROUTER_TC=0: SIMT fp32 router instead of the tensor-core GEMM;
-- DLLM_QKV_SPLITK=0 with DLLM_PDL=0: QKV without the split-K cluster, launches without
-  programmatic dependent launch;
-- DLLM_PREFILL_TC=0: causal prefill on the mma.sync flash kernel;
-- DLLM_ROUTER_KS=2: router K split over 2 CTAs instead of 8;
-- DLLM_ATTN_LEGACY=1: canvas attention on the mma.sync flash kernel too;
 - DLLM_NO_GRAPH=1: every pass launched eagerly instead of replaying its CUDA graph.
 
 A GQA group of 3 (6 query heads over 2 KV heads) does not divide the 128-row query tile
 of the tensor-core attention, so that model runs both its prefill and its canvas passes
-on the mma.sync kernel.
+on the mma.sync attention kernel; its 16 experts (not a multiple of 32) run the SIMT
+router instead of the tensor-core router GEMM.
 """
 
 from dataclasses import replace
@@ -42,13 +36,7 @@ def _run(cfg, prefix, policy, s_max, prompt_seed):
 
 
 VARIANTS = {
-    "oproj-tokens-as-m": {"DLLM_OPROJ_SWAP": "0"},
     "down-one-tile-per-item": {"DLLM_MOE_PAIR": "0"},
-    "simt-router": {"DLLM_ROUTER_TC": "0"},
-    "qkv-no-splitk-no-pdl": {"DLLM_QKV_SPLITK": "0", "DLLM_PDL": "0"},
-    "prefill-mma-sync": {"DLLM_PREFILL_TC": "0"},
-    "router-ks2": {"DLLM_ROUTER_KS": "2"},
-    "attention-mma-sync": {"DLLM_ATTN_LEGACY": "1"},
     "no-graph": {"DLLM_NO_GRAPH": "1"},
 }
 
