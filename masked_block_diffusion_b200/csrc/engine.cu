@@ -559,9 +559,8 @@ cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
                                         nullptr, &h->tm_ao64_lo);
 }
 
-// One grouped gate/up (or down) GEMM over chunks of up to BN tokens, with MPI weight
-// tiles per work item and ACC accumulator buffers (MPI * ACC * 2 * BN TMEM columns <= 512).
-// The MMA width of each chunk follows its token count.
+// One grouped gate/up (or down) GEMM over chunks of BN tokens, with MPI weight tiles per
+// work item and ACC accumulator buffers (MPI * ACC * 2 * BN TMEM columns <= 512).
 template <int BN, int MPI, int ACC>
 cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
@@ -570,8 +569,8 @@ cudaError_t moe_gate_up(dllm_handle* h, const LayerW& L) {
   PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F, 2 * F / 128,
                                 BN};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[3], d / 64, 1, s, e, nullptr,
-                                               &h->tm_xg_lo[3], &h->tok_xg);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu, h->tm_xg[BN == 64 ? 2 : 3], d / 64, 1, s, e,
+                                               nullptr, &h->tm_xg_lo[BN == 64 ? 2 : 3]);
 }
 
 template <int BN, int MPI, int ACC>
@@ -582,12 +581,12 @@ cudaError_t moe_down(dllm_handle* h, const LayerW& L) {
   PersistentGroupedSched<MPI> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d, d / 128,
                                 BN};
   EpiDown<BN> e{h->obuf, d};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[3], F / 64, 1, s, e, nullptr,
-                                               &h->tm_h_lo[3], &h->tok_h);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd, h->tm_h[BN == 64 ? 2 : 3], F / 64, 1, s, e,
+                                               nullptr, &h->tm_h_lo[BN == 64 ? 2 : 3]);
 }
 
-// The FP8-weight variants: one weight tile per item; tensor memory holds the accumulators
-// and the converted bf16 A stages (32 columns each).
+// The FP8-weight variants: one weight tile per item; each stage holds the FP8 tile, the
+// token chunk and the converted bf16 tile.
 template <int BN, int ACC, int STAGES>
 cudaError_t moe_gate_up_w8(dllm_handle* h, const LayerW& L) {
   const auto& c = h->c;
@@ -595,8 +594,8 @@ cudaError_t moe_gate_up_w8(dllm_handle* h, const LayerW& L) {
   PersistentGroupedSched<1, true> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, 2 * F,
                                     2 * F / 128, BN, L.egu, 1, (F + 127) / 128, (d + 127) / 128};
   EpiSwiGLU<BN> e{h->hbuf, h->hbuf_lo, F};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu8, h->tm_xg[3], d / 64, 1, s, e, nullptr,
-                                               &h->tm_xg_lo[3], &h->tok_xg);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wgu8, h->tm_xg[BN == 64 ? 2 : 3], d / 64, 1, s, e,
+                                               nullptr, &h->tm_xg_lo[BN == 64 ? 2 : 3], &h->tok_xg);
 }
 
 template <int BN, int ACC, int STAGES>
@@ -606,8 +605,8 @@ cudaError_t moe_down_w8(dllm_handle* h, const LayerW& L) {
   PersistentGroupedSched<1, true> s{h->offsets, h->routed, h->n_routed, h->chunk_prefix, d,
                                     d / 128, BN, L.ed, 0, d / 128, (F + 127) / 128};
   EpiDown<BN> e{h->obuf, d};
-  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd8, h->tm_h[3], F / 64, 1, s, e, nullptr,
-                                               &h->tm_h_lo[3], &h->tok_h);
+  return launch_gemm<BN, STAGES, ACC, kSplitB>(h, dim3(h->num_sms), L.tm_wd8, h->tm_h[BN == 64 ? 2 : 3], F / 64, 1, s, e,
+                                               nullptr, &h->tm_h_lo[BN == 64 ? 2 : 3], &h->tok_h);
 }
 
 // Grouped expert GEMMs of one layer over chunks of `chunk` tokens (moe_chunk). gate/up:
@@ -619,14 +618,14 @@ cudaError_t moe_gemms(dllm_handle* h, const LayerW& L, int l, int chunk, uint32_
   const bool wide = chunk == 128;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 0)) != cudaSuccess) return r;
   if (h->w8)
-    r = wide ? moe_gate_up_w8<128, 1, 4>(h, L) : moe_gate_up_w8<64, 2, 6>(h, L);
+    r = wide ? moe_gate_up_w8<128, 2, 3>(h, L) : moe_gate_up_w8<64, 2, 4>(h, L);
   else
     r = wide ? moe_gate_up<128, 1, 2>(h, L) : moe_gate_up<64, 1, 2>(h, L);
   if (r != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_GATE_UP, l, 1)) != cudaSuccess) return r;
   if ((r = tmark(h, timed, DLLM_TIMING_DOWN, l, 0)) != cudaSuccess) return r;
   if (h->w8)
-    r = wide ? moe_down_w8<128, 1, 4>(h, L) : moe_down_w8<64, 2, 6>(h, L);
+    r = wide ? moe_down_w8<128, 2, 3>(h, L) : moe_down_w8<64, 2, 4>(h, L);
   else if (wide)
     r = moe_down<128, 1, 2>(h, L);
   else

@@ -94,11 +94,15 @@ struct DenseSplitKSched {
 // thread before the roles split), so that finding an item's expert is a short search in
 // shared memory instead of a chain of dependent global loads on the producer's path.
 //
-// The MMA width follows each chunk's token count (kDynN): a chunk of n tokens loads only
-// n16 = n rounded up to 16 rows of the token pair, composed from boxes of 128, 64, 32
-// and 16 rows (the kernel's TokMaps parameter), stacked as [hi n16 rows | lo n16 rows],
-// and one MMA of N = 2 n16 reads both. An expert with few tokens then costs its weight
-// bytes and little else.
+// With DYN (kDynN) the MMA width follows each chunk's token count: a chunk of n tokens
+// loads only n16 = n rounded up to 16 rows of the token pair (a full chunk with the
+// BN-row boxes of tma_b / tma_b2, a partial one composed from the kernel's TokMaps boxes
+// of 64, 32 and 16 rows), stacked as [hi n16 rows | lo n16 rows], and one MMA of N = 2 n16
+// reads both. Without it every chunk loads and multiplies BN token rows (the rows past
+// the chunk's end belong to the next expert and are dropped by the epilogue); measured
+// faster at batch 1 both at random-init routing (gate/up 64 vs 80 us per 26B canvas
+// launch) and with every expert routed (187 vs 229 us), so the engine runs the fixed
+// width; the dynamic one stays available to the schedules.
 //
 // W8: the weights are FP8 E4M3 with one power-of-two scale 2^e per 128 x 128 tile of
 // each original expert matrix (exps, int8). Converter warps turn each staged FP8 tile
@@ -106,12 +110,12 @@ struct DenseSplitKSched {
 // the bf16 copy never touches shared memory. exp_interleave = 1 for the gate/up layout
 // (each 128-row tile: 64 gate rows, then the matching 64 up rows), 0 for down; exps is
 // [E][2 if interleaved][exp_nrb][exp_ncb].
-template <int MPI, bool W8 = false>
+template <int MPI, bool W8 = false, bool DYN = false>
 struct PersistentGroupedSched {
   static constexpr int kMaxRouted = 256;
   static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
   static constexpr int kKSplit = 1;
-  static constexpr bool kDynN = true;
+  static constexpr bool kDynN = DYN;
   static constexpr bool kW8 = W8;
   static constexpr int kMPerItem = MPI;
   const int* offsets;        // [E+1] token ranges per expert
@@ -185,7 +189,7 @@ struct PersistentGroupedSched {
     t.b_row = off + chunk * BN;
     t.m_valid = 128;
     t.n_valid = min(BN, cnt - chunk * BN);
-    t.n_cols = (t.n_valid + 15) & ~15;
+    t.n_cols = kDynN ? (t.n_valid + 15) & ~15 : 0;
     return t;
   }
 };
@@ -240,7 +244,10 @@ struct GemmSmem {
   // instead of once per half.
   static constexpr int kBStage = kB + kB2;
   static constexpr int kOffB2 = kOffB + kB;   // the lo half of stage 0 (stage s: + s * kBStage)
-  static constexpr int kBarOff = STAGES * kStageBytes;
+  // W8: the converted bf16 A tiles, one per stage, 128-byte swizzled like a TMA-loaded tile
+  static constexpr int kAbf = Sched::kW8 ? Sched::kMPerItem * 128 * 64 * 2 : 0;
+  static constexpr int kOffAbf = STAGES * kStageBytes;
+  static constexpr int kBarOff = kOffAbf + STAGES * kAbf;
   static constexpr int kEpiOff = kBarOff + 256;
   static constexpr int kSchedOff = kEpiOff + Epi::kSmemBytes;
   static constexpr int kTotal = kSchedOff + Sched::kSmemBytes + 1024;   // + alignment slack
@@ -334,11 +341,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   static_assert(MPI == 1 || (SPLIT != kSplitA && SPLIT != kSplitA3), "several m tiles per item share B only");
   constexpr int kCols = tmem_cols_for(kAccN);
   constexpr bool W8 = Sched::kW8;
-  static_assert(!W8 || (SPLIT == kSplitB && Sched::kDynN), "FP8 weights: grouped expert tiles only");
+  static_assert(!W8 || SPLIT == kSplitB, "FP8 weights: grouped expert tiles only");
   constexpr int kAccCols = kCols * ACC_BUFS * MPI;
-  constexpr int kACol = kAccCols;                        // W8: bf16 A stages, 32 columns per tile
-  constexpr int kTmemCols = tmem_alloc_cols(kAccCols + (W8 ? STAGES * MPI * 32 : 0));
-  static_assert(kAccCols + (W8 ? STAGES * MPI * 32 : 0) <= 512, "TMEM has 512 columns");
+  constexpr int kTmemCols = tmem_alloc_cols(kAccCols);
+  static_assert(kAccCols <= 512, "TMEM has 512 columns");
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, kAccN);
   constexpr int KS = Sched::kKSplit;
   static_assert(KS == 1 || BN * 128 * 4 <= STAGES * L::kStageBytes, "split-K partial fits the stage buffers");
@@ -356,7 +362,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   uint64_t* acc_empty = acc_full + ACC_BUFS;
   uint64_t* drain = acc_empty + ACC_BUFS;
   uint64_t* peer_ready = drain + 1;   // split-K: rank 0 learns that the peers' partials are in place
-  uint64_t* conv_full = drain + 2;    // W8: the stage's bf16 A tiles are in tensor memory
+  uint64_t* conv_full = drain + 2;    // W8: the stage's bf16 A tiles are in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv_full + (W8 ? STAGES : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* epi_smem = smem + L::kEpiOff;
@@ -408,8 +414,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    if constexpr (Sched::kDynN)
-      for (int i = 0; i < 8; ++i) tma_prefetch_desc(&tok.m[i]);
     const uint64_t pol_first = policy_evict_first();
     const uint64_t pol_last = policy_evict_last();
     const uint64_t pol_a = a_stream_first ? pol_first : pol_last;
@@ -428,18 +432,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
           mbar_arrive_expect_tx(&full[stage], t.m_count * L::kAtile + 2 * n16 * 128);
           for (int u = 0; u < t.m_count; ++u)
             tma_load_2d(sA + stage * L::kA + u * L::kAtile, &tma_a, &full[stage], kb * 64, t.a_row + u * 128, pol_a);
-          // [hi n16 rows | lo n16 rows], each half from boxes of 128 / 64 / 32 / 16 rows
+          // [hi n16 rows | lo n16 rows]: a full chunk with the BN-row boxes of tma_b / tma_b2,
+          // a partial one composed from boxes of 64 / 32 / 16 rows
           uint8_t* dst = sB + stage * L::kBStage;
+          if (n16 == BN) {
+            tma_load_2d(dst, &tma_b, &full[stage], kb * 64, t.b_row, pol_b);
+            tma_load_2d(dst + BN * 128, &tma_b2, &full[stage], kb * 64, t.b_row, pol_b);
+          } else {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            int off = 0;
+            for (int half = 0; half < 2; ++half) {
+              int off = 0;
 #pragma unroll
-            for (int bi = 3; bi >= 0; --bi) {
-              const int rows = 16 << bi;
-              if ((n16 - off) & rows) {
-                tma_load_2d(dst + (half * n16 + off) * 128, &tok.m[half * 4 + bi], &full[stage], kb * 64,
-                            t.b_row + off, pol_b);
-                off += rows;
+              for (int bi = 2; bi >= 0; --bi) {
+                const int rows = 16 << bi;
+                if ((n16 - off) & rows) {
+                  tma_load_2d(dst + (half * n16 + off) * 128, &tok.m[half * 4 + bi], &full[stage], kb * 64,
+                              t.b_row + off, pol_b);
+                  off += rows;
+                }
               }
             }
           }
@@ -495,15 +505,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
         const uint32_t a1 = smem_u32(sA2 + stage * L::kA2);
         const uint32_t a2 = smem_u32(sA3 + stage * L::kA3);
         if constexpr (W8) {
-          // A: the converted bf16 tile in tensor memory (8 columns per 16 k)
-          const uint32_t at = tmem_base + kACol + stage * MPI * 32;
+          // A: the converted bf16 tile the converter warps wrote into shared memory
+          const uint32_t ab = smem_u32(smem + L::kOffAbf + stage * L::kAbf);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
             for (int u = 0; u < MPI; ++u)
               if (u < mc)
-                umma_bf16_ts(d_tmem + u * kCols, at + u * 32 + kk * 8, sdesc_k_sw128(b0 + kk * 32), idesc,
-                             (kb != kb_begin || kk != 0) ? 1u : 0u);
+                umma_bf16(d_tmem + u * kCols, sdesc_k_sw128(ab + u * 128 * 128 + kk * 32), sdesc_k_sw128(b0 + kk * 32),
+                          idesc, (kb != kb_begin || kk != 0) ? 1u : 0u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -533,9 +543,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
     umma_commit(drain);
     mbar_drain(drain, 0);
   } else if (W8 && warp >= 6) {
-    // ---------------- converters (W8): FP8 tile -> bf16 in tensor memory. Warp 6 + w
-    // takes TMEM lane quarter w % 4 (row r = 32 (w % 4) + lane) and k values
-    // 32 (w / 4) .. 32 (w / 4) + 31 of the stage's 64.
+    // ---------------- converters (W8): FP8 tile -> bf16 tile in shared memory, laid out
+    // with the 128-byte swizzle the MMA's descriptor expects. Warp 6 + w takes rows
+    // 32 (w % 4) .. + 31 (one per lane) and k values 32 (w / 4) .. + 31 of the stage's 64.
     if constexpr (W8) {
       static_assert(MPI == 1, "W8: one weight tile per item");
       const int cw = warp - 6;
@@ -573,9 +583,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
               o[c * 8 + 2 * i + 1] = e4m3x2_to_bf16x2((uint16_t)(w[i] >> 16), sc);
             }
           }
-          tmem_st16_nowait(tmem_at(tmem_base + kACol + stage * 32 + kh * 16, q * 32, 0), o);
-          tmem_wait_st();
-          tc_fence_before();
+          // 16-byte chunk c (8 k values) of row r goes to chunk c ^ (r & 7) of its 128-byte row
+          uint8_t* out_row = smem + L::kOffAbf + stage * L::kAbf + r * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = kh * 4 + i;
+            *reinterpret_cast<uint4*>(out_row + ((c ^ (r & 7)) << 4)) =
+                make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+          fence_proxy_async_smem();   // the writes above are read by the tensor core
           mbar_arrive(&conv_full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
