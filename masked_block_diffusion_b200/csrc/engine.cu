@@ -173,6 +173,9 @@ struct dllm_handle {
   float* apart = nullptr;
   float* alse = nullptr;
   float* rlogits = nullptr;
+  float* rpart = nullptr;     // router GEMM split-K partials, summed by the top-k kernel
+  float* opart = nullptr;     // O projection split-K partials, summed by the FFN norm
+  long rpart_elems = 0, opart_elems = 0;
   int32_t* tk_idx = nullptr;
   float* tk_w = nullptr;
   int32_t* offsets = nullptr;
@@ -196,6 +199,7 @@ struct dllm_handle {
   CUtensorMap tm_y_lo, tm_y_lo2, tm_xg_lo[4], tm_h_lo[4];
   TokMaps tok_xg, tok_h;     // the grouped GEMMs' token-operand maps: boxes of 16..128 rows, hi then lo
   CUtensorMap tm_ao64, tm_ao64_lo;   // attention output as 64-row boxes (swapped O projection)
+  CUtensorMap tm_ao128, tm_ao128_lo; // 128-row boxes (the O projection's split-K tiles)
   CUtensorMap tm_q3;        // q buffer [T][H][hd], box = 64 dims x group heads x 128/group queries
   bool attn_tc = false;     // attention on the tensor cores (the GQA group divides a 128-row query tile)
   bool moe_pair = true;     // grouped down GEMM at BN = 64: two weight tiles per work item
@@ -520,39 +524,47 @@ cudaError_t tmark(dllm_handle* h, uint32_t tmask, int kind, int layer, int which
 // Router logits on the tensor cores: logits[T][E] = y W_r^T with the normalised
 // activations as their (hi, lo) bf16 pair, so each product keeps about 16 mantissa bits
 // of y and the sum is fp32. Experts form 32-column tiles; with few tiles (one canvas:
-// 2 x 4) the K loop is split over clusters of up to 8 CTAs.
-template <int KS>
-cudaError_t router_gemm_ks(dllm_handle* h, const LayerW& L, int T, int mt, int tiles) {
-  EpiStoreF32<32> e{h->rlogits, h->E, h->E};
-  const int kb = h->c.d_model / 64;
-  if constexpr (KS == 1) {
-    DenseSched s{T, mt, 32};
-    return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
-  } else {
-    DenseSplitKSched<KS> s{T, mt, 32};
-    return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles * KS), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
-  }
-}
-
-cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T) {
+// 2 x 4) the K loop is split over up to 8 independent CTAs (slices x tiles <= 2 x the
+// SM count) whose partial logits the top-k kernel adds (*nparts > 0); otherwise the GEMM
+// writes the logits itself.
+cudaError_t router_gemm(dllm_handle* h, const LayerW& L, int T, int* nparts) {
   const int mt = ceil_div(T, 128);
   const int tiles = mt * (h->E / 32);
   const int kb = h->c.d_model / 64;
-  if (tiles * 8 <= 2 * h->num_sms && kb >= 8) return router_gemm_ks<8>(h, L, T, mt, tiles);
-  if (tiles * 4 <= 2 * h->num_sms && kb >= 4) return router_gemm_ks<4>(h, L, T, mt, tiles);
-  if (tiles * 2 <= 2 * h->num_sms && kb >= 2) return router_gemm_ks<2>(h, L, T, mt, tiles);
-  return router_gemm_ks<1>(h, L, T, mt, tiles);
+  const int ks = std::min({8, kb / 2, 2 * h->num_sms / tiles});
+  *nparts = 0;
+  if (ks >= 2 && (long)ks * T * h->E <= h->rpart_elems) {
+    EpiStoreF32<32> e{h->rpart, h->E, h->E, (long)T * h->E};
+    DensePartKSched s{T, mt, 32, ks};
+    *nparts = ks;
+    return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles * ks), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
+  }
+  EpiStoreF32<32> e{h->rlogits, h->E, h->E};
+  DenseSched s{T, mt, 32};
+  return launch_gemm<32, 6, 1, kSplitA>(h, dim3(tiles), h->tm_y, L.tm_wr, kb, 0, s, e, &h->tm_y_lo);
 }
 
 // Attention output projection with the residual add, x += ao * Wo^T, operands swapped:
-// weight rows (output features) are M and 64-token chunks N, with the token operand's
-// (hi, lo) halves stacked into one N = 128 MMA, so each weight tile is read from shared
-// memory once per k step (measured faster than tokens as M with two MMAs per k step:
-// 0.73 vs 0.91 ms per 26B canvas pass).
-cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T) {
+// weight rows (output features) are M and token chunks N, with the token operand's
+// (hi, lo) halves stacked into one MMA of width 2 BN, so each weight tile is read from
+// shared memory once per k step (measured faster than tokens as M with two MMAs per k
+// step: 0.73 vs 0.91 ms per 26B canvas pass). With few tiles (one canvas) the K loop is
+// split over ks independent CTAs on 128-token chunks and the FFN norm that follows adds
+// their partials into x (*nparts = ks); otherwise 64-token chunks add into x directly.
+cudaError_t o_proj(dllm_handle* h, const LayerW& L, int T, int* nparts) {
   const auto& c = h->c;
   const int d = c.d_model;
   const int kb = c.n_heads * c.head_dim / 64;
+  const int tiles128 = (d / 128) * ceil_div(T, 128);
+  const int ks = std::min({4, kb, h->num_sms / tiles128});
+  *nparts = 0;
+  if (ks >= 2 && (long)ks * T * d <= h->opart_elems) {
+    EpiPartialT<128> e{h->opart, d, T, (long)T * d};
+    DensePartKSched s{d, d / 128, 128, ks};
+    *nparts = ks;
+    return launch_gemm<128, 4, 1, kSplitB>(h, dim3(tiles128 * ks), L.tm_wo128, h->tm_ao128, kb, 1, s, e, nullptr,
+                                           &h->tm_ao128_lo);
+  }
   EpiResidualT<64> et{h->x, d, T};
   DenseSched s{d, d / 128, 64};
   return launch_gemm<64, 6, 1, kSplitB>(h, dim3((d / 128) * ceil_div(T, 64)), L.tm_wo128, h->tm_ao64, kb, 1, s, et,
@@ -647,8 +659,8 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     bf16_t* kc = h->kcache + (size_t)l * h->kv_layer;
     bf16_t* vc = h->vcache + (size_t)l * h->kv_layer;
     if (l == 0) {   // later layers get this norm from the previous layer's combine
-      CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.attn_norm, d, c.rms_eps, h->y,
-                  h->y_lo, h->y_lo2, h->rstd));
+      CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, (const float*)nullptr, 0, 0L,
+                  L.attn_norm, d, c.rms_eps, h->y, h->y_lo, h->y_lo2, h->rstd));
       h->launches++;
     }
     CK(tmark(h, timed, DLLM_TIMING_QKV, l, 0));
@@ -658,22 +670,24 @@ int run_layers(dllm_handle* h, int T, int nreq, int tok_per_req, const int* pos0
     CK(attention(h, kc, vc, T, nreq, tok_per_req, pos0, slot, causal, splits, &L));
     CK(tmark(h, timed, DLLM_TIMING_ATTN, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 0));
-    CK(o_proj(h, L, T));
+    int o_parts = 0;
+    CK(o_proj(h, L, T, &o_parts));
     CK(tmark(h, timed, DLLM_TIMING_OPROJ, l, 1));
     CK(tmark(h, timed, DLLM_TIMING_ROUTE, l, 0));
-    CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo,
-                (bf16_t*)nullptr, h->rstd));
+    CK(launch_k(h, rmsnorm_kernel, dim3(T), dim3(row_threads(d)), 0, h->x, (const float*)h->opart, o_parts,
+                (long)T * d, L.ffn_norm, d, c.rms_eps, h->y, h->y_lo, (bf16_t*)nullptr, h->rstd));
     h->launches++;
     if (!h->dense) {
+      int r_parts = 0;
       if (h->router_tc) {
-        CK(router_gemm(h, L, T));
+        CK(router_gemm(h, L, T, &r_parts));
       } else {
         CK(launch_k(h, router_kernel, dim3(ceil_div(T, kRouterTok), ceil_div(h->E, kRouterExp)), dim3(256),
                     kRouterTok * d * sizeof(float), h->x, h->rstd, L.ffn_norm, L.wr, T, d, h->E, h->rlogits));
         h->launches++;
       }
       CK(launch_k(h, topk_kernel, dim3(ceil_div((long)T * 32, 256)), dim3(256), 0, h->rlogits, T, h->E, h->k,
-                  h->tk_idx, h->tk_w));
+                  h->tk_idx, h->tk_w, (const float*)h->rpart, r_parts, (long)T * h->E));
       h->launches++;
       if (record) {
         CK(cudaMemcpyAsync(h->dbg_logits + (size_t)l * h->T_canvas_max * h->E, h->rlogits,
@@ -1073,6 +1087,13 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
     DA(h->alse, mx * c.canvas * H + 1);
   }
   DA(h->rlogits, (size_t)T * h->E);
+  // split-K partials exist only while slices x tiles <= 2 x the SM count (router:
+  // 32-expert tiles of 128 rows) or <= the SM count (O projection: 128 x 128 tiles),
+  // which bounds their size
+  h->rpart_elems = 2L * h->num_sms * 128 * 32;
+  h->opart_elems = (long)h->num_sms * 128 * 128;
+  DA(h->rpart, (size_t)h->rpart_elems);
+  DA(h->opart, (size_t)h->opart_elems);
   DA(h->tk_idx, (size_t)N);
   DA(h->tk_w, (size_t)N);
   DA(h->offsets, h->E + 1);
@@ -1131,6 +1152,8 @@ int create_impl(dllm_handle* h, const void* weights, size_t weight_bytes, int on
   ok &= make_tmap(&h->tm_y_lo2, h->y_lo2, T, d, 128);
   ok &= make_tmap(&h->tm_ao64, h->ao, T, qd, 64);
   ok &= make_tmap(&h->tm_ao64_lo, h->ao_lo, T, qd, 64);
+  ok &= make_tmap(&h->tm_ao128, h->ao, T, qd, 128);
+  ok &= make_tmap(&h->tm_ao128_lo, h->ao_lo, T, qd, 128);
   ok &= make_tmap(&h->tm_head, h->head, V, d, 256);
   if (h->attn_tc) ok &= make_tmap3(&h->tm_q3, h->q, hd, H, T, H / Hkv, 128 / (H / Hkv));
   for (int i = 0; i < 4; ++i) {

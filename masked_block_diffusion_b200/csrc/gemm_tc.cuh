@@ -22,6 +22,7 @@ struct Tile {
   int mt, nt;    // dense: (m tile, n tile); grouped: (m tile inside the expert, expert)
   int m_count = 1;   // m tiles of this work item (128 rows apart, sharing the B tile)
   int n_cols = 0;    // accumulator columns computed (per operand half); 0 = the full BN
+  int ks = 0;        // K slice of a DensePartKSched tile (its epilogue writes partial ks)
 };
 
 // Columns of the tile an epilogue reads: the full BN, or the rounded-up valid columns
@@ -34,6 +35,7 @@ DLLM_DEV int tile_cols(const Tile& t) { return t.n_cols > 0 ? t.n_cols : BN; }
 struct DenseSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = 1;
+  static constexpr bool kPartK = false;
   static constexpr bool kDynN = false;
   static constexpr bool kW8 = false;
   static constexpr int kMPerItem = 1;
@@ -61,6 +63,7 @@ template <int KS>
 struct DenseSplitKSched {
   static constexpr int kSmemBytes = 0;
   static constexpr int kKSplit = KS;
+  static constexpr bool kPartK = false;
   static constexpr bool kDynN = false;
   static constexpr bool kW8 = false;
   static constexpr int kMPerItem = 1;
@@ -70,6 +73,35 @@ struct DenseSplitKSched {
   DLLM_DEV Tile tile(int) const {
     Tile t;
     int id = blockIdx.x / KS;
+    t.mt = id % n_mtiles;
+    t.nt = id / n_mtiles;
+    t.a_row = t.mt * 128;
+    t.b_row = t.nt * BN;
+    t.m_valid = min(128, M - t.a_row);
+    t.n_valid = BN;
+    return t;
+  }
+};
+
+// Dense tiles with the K loop split over `ks` independent CTAs (consecutive blockIdx.x,
+// no cluster): slice r accumulates k blocks [r*kb/ks, (r+1)*kb/ks) and its epilogue
+// writes partial sum r of the tile (Tile::ks) to global memory, where the consumer kernel
+// adds the ks partials in slice order. No CTA waits on another, so the slices need not be
+// co-resident and nothing stalls at the end of the K loop.
+struct DensePartKSched {
+  static constexpr int kSmemBytes = 0;
+  static constexpr int kKSplit = 1;
+  static constexpr bool kPartK = true;
+  static constexpr bool kDynN = false;
+  static constexpr bool kW8 = false;
+  static constexpr int kMPerItem = 1;
+  int M, n_mtiles, BN, ks;
+  DLLM_DEV void stage(int*) {}
+  DLLM_DEV int count() const { return 1; }
+  DLLM_DEV Tile tile(int) const {
+    Tile t;
+    int id = blockIdx.x / ks;
+    t.ks = blockIdx.x % ks;
     t.mt = id % n_mtiles;
     t.nt = id / n_mtiles;
     t.a_row = t.mt * 128;
@@ -115,6 +147,7 @@ struct PersistentGroupedSched {
   static constexpr int kMaxRouted = 256;
   static constexpr int kSmemBytes = (4 * kMaxRouted + 8) * 4;
   static constexpr int kKSplit = 1;
+  static constexpr bool kPartK = false;
   static constexpr bool kDynN = DYN;
   static constexpr bool kW8 = W8;
   static constexpr int kMPerItem = MPI;
@@ -409,8 +442,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant_
   const uint32_t tmem_base = *tmem_slot;
   const int ntiles = sched.count();
   const int krank = KS > 1 ? (int)cluster_ctarank() : 0;
-  const int kb_begin = krank * k_blocks / KS;
-  const int kb_end = (krank + 1) * k_blocks / KS;
+  int kb_begin = krank * k_blocks / KS;
+  int kb_end = (krank + 1) * k_blocks / KS;
+  if constexpr (Sched::kPartK) {
+    const int sl = (int)blockIdx.x % sched.ks;
+    kb_begin = sl * k_blocks / sched.ks;
+    kb_end = (sl + 1) * k_blocks / sched.ks;
+  }
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -670,8 +708,10 @@ struct EpiStoreF32 {
   float* out;
   int ldo;
   int N;
+  long part_stride = 0;   // DensePartKSched: partial sum t.ks goes to out + t.ks * part_stride
   DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
     const long row = t.a_row + r;
+    float* out = this->out + t.ks * part_stride;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 16) {
       float v[16];
@@ -842,6 +882,32 @@ struct EpiResidualT {
       for (int i = 0; i < 16; ++i) {
         const int tok = t.b_row + c0 + i;
         if (tok < T && r < t.m_valid) x[(long)tok * ldx + f] = old[i] + v[i];
+      }
+    }
+  }
+};
+
+// Split-K partial of the swapped-operand O projection: partial t.ks of D^T, stored as
+// part[t.ks][token][feature] in fp32 (coalesced across the feature lanes like
+// EpiResidualT); the RMSNorm kernel that follows adds the partials into x in slice order.
+template <int BN>
+struct EpiPartialT {
+  static constexpr int kSmemBytes = 0;
+  float* part;
+  int ldp;      // features per row (d)
+  int T;        // token rows
+  long stride;  // elements per partial (T_max * d)
+  DLLM_DEV void operator()(const Tile& t, uint32_t taddr, int r, uint8_t*) const {
+    const int f = t.a_row + r;
+    float* p = part + t.ks * stride;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int tok = t.b_row + c0 + i;
+        if (tok < T && r < t.m_valid) p[(long)tok * ldp + f] = v[i];
       }
     }
   }

@@ -56,15 +56,31 @@ DLLM_DEV void store_norm_terms(bf16_t* y, bf16_t* y_lo, bf16_t* y_lo2, long t, i
 
 // v = x * rsqrt(mean(x^2) + eps) * g, written as bf16 terms (store_norm_terms); rstd[t]
 // kept for the fp32 router.
-__global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g, int d, float eps,
+//
+// With nparts > 0 the row first takes the split-K partial sums of the GEMM before it:
+// x[t] += part[0][t] + part[1][t] + ... (slice order, partial s at part + s * pstride),
+// written back to x, and the norm is taken of the updated row.
+__global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ part, int nparts, long pstride,
+                               const float* __restrict__ g, int d, float eps,
                                bf16_t* __restrict__ y, bf16_t* __restrict__ y_lo, bf16_t* __restrict__ y_lo2,
                                float* __restrict__ rstd) {
   pdl_begin();
   const int t = blockIdx.x;
-  const float4* xr = reinterpret_cast<const float4*>(x + (long)t * d);
+  float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
   float ss = 0.f;
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
     float4 v = xr[c];
+    if (nparts > 0) {
+      const float4* pr = reinterpret_cast<const float4*>(part + (long)t * d) + c;
+      for (int s = 0; s < nparts; ++s) {
+        const float4 a = pr[s * (pstride / 4)];
+        v.x += a.x;
+        v.y += a.y;
+        v.z += a.z;
+        v.w += a.w;
+      }
+      xr[c] = v;
+    }
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
   }
   __shared__ float red[32];
@@ -81,7 +97,7 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
   if (threadIdx.x == 0 && rstd != nullptr) rstd[t] = r;
   const float4* gr = reinterpret_cast<const float4*>(g);
   for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    const float4 v = xr[c], gg = gr[c];
+    const float4 v = xr[c], gg = gr[c];   // with partials: this thread's own writes above
     store_norm_terms(y, y_lo, y_lo2, t, d, c, make_float4(v.x * r * gg.x, v.y * r * gg.y, v.z * r * gg.z, v.w * r * gg.w));
   }
 }
@@ -208,12 +224,29 @@ DLLM_DEV void topk_token(const float* logits, int t, int E, int k, int32_t* idx,
   }
 }
 
-__global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
-                            float* __restrict__ gate) {
+// With nparts > 0 the router GEMM left split-K partial sums (partial s at
+// part + s * pstride): each lane first adds, in slice order, the partials of the logits it
+// reads and stores them in `logits` (the full logits stay available to the debug copies).
+__global__ void topk_kernel(float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ idx,
+                            float* __restrict__ gate, const float* __restrict__ part, int nparts, long pstride) {
   pdl_begin();
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
+  if (nparts > 0) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    for (int s = 0; s < nparts; ++s) {
+      const float* ps = part + s * pstride + (long)t * E;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (lane + 32 * j < E) v[j] += ps[lane + 32 * j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (lane + 32 * j < E) logits[(long)t * E + lane + 32 * j] = v[j];
+  }
   topk_token(logits, t, E, k, idx, gate, lane);
 }
 
