@@ -8,21 +8,29 @@
 // One CTA = one 128-row query tile of one KV head over one split of the key range. The
 // tile holds the GQA group's heads for 128 / group queries (row r = query r / group,
 // head r % group), so each K/V block is loaded once for all heads that read it.
+//
+// The split's key blocks are dealt to two independent online-softmax streams: stream 0
+// takes the even blocks, stream 1 the odd ones, each with its own running maximum and
+// sum, its own O accumulator and its own S buffer in TMEM. While one stream's softmax
+// warps turn its scores into probabilities, the tensor pipe runs the other stream's
+// S = Q K^T and O += P V, so neither the MMAs nor the softmax wait on each other's whole
+// chain. At the end the two streams are merged in log-sum-exp fashion.
+//
 // Roles (320 threads):
-//   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys into two
-//                  three-stage rings (a K stage is refilled once the S = Q K^T that read
+//   warp 0 lane 0  TMA: the Q tile once, then K and V blocks of BK keys, in block order,
+//                  into two three-stage rings (a K stage is refilled once the S that read
 //                  it completes, a V stage once its P V does);
-//   warp 1         TMEM allocation; lane 0 issues S = Q K^T into one of three TMEM S
-//                  buffers two blocks ahead of O += P_hi V + P_lo V, so the scores of the
-//                  next blocks are ready while the softmax works on the current one;
-//   warps 2..9     two warpgroups, each on one half (32 keys) of a block, one query row
-//                  per thread in each: read S from TMEM, scale and mask, running
-//                  maximum, P = exp2(s - m_ref) as a bf16 (hi, lo) pair written back into
-//                  TMEM with tcgen05.st (the P V MMA reads its A operand from TMEM, so P
-//                  needs no shared memory), running sum; O in TMEM is rescaled only when
-//                  the maximum grows by more than 2^8 (P stays below 256, exact enough,
-//                  and rescales are rare). At the end they read O, divide by the sum and
-//                  write the output (or a split partial).
+//   warp 1         TMEM allocation; lane 0 issues the MMAs: S(j) into stream j&1's S
+//                  buffer, O_(j&1) += P_hi V + P_lo V once the softmax has written P(j)
+//                  over S(j), and S(j+2) into the same buffer once that P V completed;
+//   warps 2..5     stream 0's softmax, warps 6..9 stream 1's: one query row per thread
+//                  (TMEM lane r), all BK keys of the row per block: read S, scale and
+//                  mask, running maximum, P = exp2(s - m_ref) as a bf16 (hi, lo) pair
+//                  written back into the S columns with tcgen05.st (the P V MMA reads its
+//                  A operand from TMEM), running sum. O is rescaled only when the maximum
+//                  grows by more than 2^8 (P stays below 256, exact enough, and rescales
+//                  are rare). At the end both streams read O_0 and O_1, merge them and
+//                  write the output (or a split partial), each on half of the columns.
 // Every wait is bounded, as in gemm_tc.cuh.
 #pragma once
 
@@ -76,24 +84,46 @@ DLLM_DEV float ex2_approx(float x) {
   return y;
 }
 
-// True on both warps of a lane-quarter pair (the two softmax halves of the same rows)
-// iff true on each of their 64 threads (named barrier `id`). The pairs agree on leaving
-// the loop together without holding the other pairs back.
-DLLM_DEV bool pair_all(bool ok, int id) {
+// Maximum and sum of N register values as a balanced tree (depth log2 N instead of a
+// chain of N dependent operations on the softmax's critical path). tree_sum overwrites v.
+template <int N>
+DLLM_DEV float tree_max(const float (&v)[N]) {
+  float a[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) a[i] = fmaxf(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+  for (int w = N / 4; w >= 1; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) a[i] = fmaxf(a[2 * i], a[2 * i + 1]);
+  return a[0];
+}
+
+template <int N>
+DLLM_DEV float tree_sum(float (&v)[N]) {
+#pragma unroll
+  for (int w = N / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) v[i] = v[2 * i] + v[2 * i + 1];
+  return v[0];
+}
+
+// True on every softmax thread (both streams, 256 threads, named barrier 1) iff true on
+// each of them.
+DLLM_DEV bool softmax_all(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 64, p;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
-      : "r"((uint32_t)ok), "r"(id)
+      : "r"((uint32_t)ok)
       : "memory");
   return r != 0;
 }
 
-// TMEM columns: S buffers at 0, 64 and 128; P buffer pb at 192 + 64 pb (hi in the first 32
-// columns, lo in the next 32, two bf16 per column); O from column 320.
+// TMEM columns: stream s's S buffer at 64 s (P(j) is written over S(j): hi pairs of the
+// 64 keys in its first 32 columns, lo pairs in the next 32), O of stream s at 128 + HD s.
 template <int HD>
 struct AttnTcCfg {
   static constexpr int BK = 64;
@@ -105,152 +135,132 @@ struct AttnTcCfg {
   static constexpr int kOffK = kQ;
   static constexpr int kOffV = kOffK + STAGES * kKV;
   static constexpr int kOffBar = kOffV + STAGES * kKV;
-  static constexpr int kOffRed = kOffBar + 256;          // softmax halves: maxima [2][2][128], sums [2][128]
-  static constexpr int kTotal = kOffRed + 768 * 4 + 1024;
-  static constexpr int kOSplit = ((HD / 2 + 15) / 16) * 16;   // O columns of the first softmax half
-  static constexpr int kSBufs = 3;                       // S buffers: S(j+2) is issued before P V(j)
-  static constexpr int kSCols = BK;
-  static constexpr int kPCol = kSBufs * BK;
-  static constexpr int kOCol = kPCol + 2 * BK;
+  static constexpr int kOffRed = kOffBar + 256;          // per stream: (max, sum) of each row, for the merge
+  static constexpr int kTotal = kOffRed + 512 * 4 + 1024;
+  static constexpr int kSCol = 0;                        // + 64 * stream
+  static constexpr int kOCol = 2 * BK;                   // + HD * stream
+  static constexpr int kOHalf = ((HD / 2 + 15) / 16) * 16;   // O columns the first stream writes out
   static constexpr int kTmemCols = 512;
-  static_assert(kPCol + 2 * BK <= kOCol && kOCol + HD <= kTmemCols, "TMEM");
+  static_assert(kOCol + 2 * HD <= kTmemCols, "TMEM");
   static_assert(kTotal <= 232448, "shared memory");
 };
 
-// Warps 2..9: two warpgroups, the first on keys 0..31 of each block, the second on keys
-// 32..63; thread (warp w, lane) owns query row r = 32 (w % 4) + lane (TMEM lane r) in
-// both, so each row's exponentials are split over two warps of the same SM sub-partition
-// pair. The halves agree on the row maximum through shared memory (red[parity][half][r],
-// one 64-thread named barrier per lane quarter), so they take the same rescaling
-// decisions; each rescales and finally writes its own column range of O, and the row sum
-// is combined once at the end.
+// Warps 2..9: stream st = (warp - 2) / 4; thread (warp w, lane) owns query row
+// r = 32 (w % 4) + lane (TMEM lane r) of its stream, all BK keys of each of the stream's
+// blocks j = st, st + 2, ...
 template <int HD>
-DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* s_empty,
-                           uint64_t* p_full, uint64_t* p_empty, uint64_t* o_final, float* red,
-                           volatile int* abort_flag, int warp, int lane, int q0, int b, int sp, int ks, int ke,
-                           int nblk) {
+DLLM_DEV void softmax_stream(const AttnTcParams& p, uint32_t tmem_base, uint64_t* s_full, uint64_t* p_full,
+                             uint64_t* o_final, float* red, volatile int* abort_flag, int warp, int lane, int q0,
+                             int b, int sp, int ks, int ke, int nblk) {
   using G = AttnTcCfg<HD>;
-  constexpr int BK = G::BK, HB = BK / 2;   // keys per half
-  static_assert(BK == 64, "two 32-key halves per block");
+  constexpr int BK = G::BK;
   const int q = warp & 3;
-  const int half = (warp - 2) >> 2;
+  const int st = (warp - 2) >> 2;
   const int r = q * 32 + lane;
   const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-  const int o_lo = half == 0 ? 0 : G::kOSplit, o_hi = half == 0 ? G::kOSplit : HD;   // this half's O columns
-  const int pair_bar = 3 + q;   // named barrier of the two warps sharing lane quarter q
+  const uint32_t s_col = lane_base + G::kSCol + st * BK;
+  const uint32_t o_own = lane_base + G::kOCol + st * HD;
   // keys this row may see end at row_ke: the tile's end, or (causal) the row's own query
   // position + 1; rows past the last query take the last query's limit (output dropped)
   int row_ke = ke;
   if (p.causal) row_ke = min(ke, p.pos0[b] + min(q0 + r / p.group, p.tok_per_req - 1) + 1);
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
-  for (int j = 0; j < nblk; ++j) {
-    const int sb = j % G::kSBufs;
-    if (!pair_all(mbar_wait(&s_full[sb], (j / G::kSBufs) & 1, abort_flag), pair_bar)) { ok = false; break; }
+  const int nb = (nblk - st + 1) / 2;
+  for (int i = 0; i < nb; ++i) {
+    const int j = 2 * i + st;
+    if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], i & 1, abort_flag))) { ok = false; break; }
     tc_fence_after();
-    float s[HB];
-    tmem_ld32(lane_base + sb * G::kSCols + half * HB, s);
-    tc_fence_before();
-    mbar_arrive(&s_empty[sb]);
-    // the maximum is taken on the raw scores (scaling by a positive constant commutes
-    // with it, rounding included); keys past the row's end are masked only in the
-    // blocks that have some
-    const int nvis = row_ke - (ks + j * BK + half * HB);
-    float mx_raw = -INFINITY;
-    if (nvis >= HB) {
+    float s[BK];
+    tmem_ld64(s_col, s);
+    const int nvis = row_ke - (ks + j * BK);
+    if (nvis < BK) {
 #pragma unroll
-      for (int c = 0; c < HB; ++c) mx_raw = fmaxf(mx_raw, s[c]);
-    } else {
-#pragma unroll
-      for (int c = 0; c < HB; ++c) {
+      for (int c = 0; c < BK; ++c)
         if (c >= nvis) s[c] = -INFINITY;
-        mx_raw = fmaxf(mx_raw, s[c]);
-      }
     }
-    float* slot = red + (j & 1) * 256;
-    slot[half * 128 + r] = mx_raw;
-    named_bar_sync(pair_bar, 64);
-    mx_raw = fmaxf(mx_raw, slot[(half ^ 1) * 128 + r]);
-    const float mx = mx_raw * p.scale_log2;
-    if (j == 0) {
-      m_ref = mx;   // block 0 always holds a visible key of every row
+    // the maximum is taken on the raw scores (scaling by a positive constant commutes
+    // with it, rounding included)
+    const float mx = tree_max<BK>(s) * p.scale_log2;
+    if (i == 0) {
+      m_ref = mx;
     } else {
       const bool need = mx > m_ref + 8.0f;
       if (__any_sync(0xffffffffu, need)) {
-        // O is rescaled once P V(j-1) has landed: its completion is the commit on P buffer
-        // (j-1)&1 (with S issued ahead of P V, S(j) being ready no longer implies it)
-        const bool got =
-            __all_sync(0xffffffffu, mbar_wait(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag));
-        if (got) {
-          tc_fence_after();
-          const float f = need ? exp2f(m_ref - mx) : 1.0f;
+        // this stream's O is stable here: S(j) was issued only after P V(j - 2) completed
+        const float f = need ? exp2f(m_ref - mx) : 1.0f;
 #pragma unroll 1
-          for (int c = o_lo; c < o_hi; c += 16) {
-            float v[16];
-            tmem_ld16(lane_base + G::kOCol + c, v);
+        for (int c = 0; c < HD; c += 16) {
+          float v[16];
+          tmem_ld16(o_own + c, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= f;
-            tmem_st16(lane_base + G::kOCol + c, v);
-          }
-          tc_fence_before();
-          if (need) {
-            l *= f;
-            m_ref = mx;
-          }
-        } else {
-          ok = false;
+          for (int e = 0; e < 16; ++e) v[e] *= f;
+          tmem_st16(o_own + c, v);
+        }
+        if (need) {
+          l *= f;
+          m_ref = mx;
         }
       }
     }
-    uint32_t hi[HB / 2], lo[HB / 2];
-    float psum = 0.f;
+    // a causal row whose keys so far are all masked has m_ref = -inf: every p is 0
+    const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+    uint32_t hi[BK / 2], lo[BK / 2];
 #pragma unroll
-    for (int c = 0; c < HB; c += 2) {
-      const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_ref));
-      const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_ref));
-      psum += p0 + p1;
-      split_bf16x2(p0, p1, hi[c / 2], lo[c / 2]);
+    for (int c = 0; c < BK; c += 2) {
+      s[c] = ex2_approx(fmaf(s[c], p.scale_log2, -mb));
+      s[c + 1] = ex2_approx(fmaf(s[c + 1], p.scale_log2, -mb));
+      split_bf16x2(s[c], s[c + 1], hi[c / 2], lo[c / 2]);
     }
-    l += psum;
-    const int pb = j & 1;
-    if (!pair_all(ok && mbar_wait(&p_empty[pb], ((j >> 1) & 1) ^ 1, abort_flag), pair_bar)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    // P buffer pb: hi pairs of keys 0..63 in columns 0..31, lo pairs in 32..63
-    const uint32_t pcol = lane_base + G::kPCol + pb * BK + half * (HB / 2);
-    tmem_st16_nowait(pcol, hi);
-    tmem_st16_nowait(pcol + BK / 2, lo);
+    l += tree_sum<BK>(s);
+    // P(j) over S(j): hi pairs of the 64 keys in the buffer's columns 0..31, lo in 32..63
+    tmem_st32_nowait(s_col, hi);
+    tmem_st32_nowait(s_col + BK / 2, lo);
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&p_full[pb]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&p_full[st]);
   }
-  if (ok) ok = pair_all(mbar_wait(o_final, 0, abort_flag), pair_bar);
-  if (!ok) {
-    atomicExch(p.err, kDevTimeoutEpilogue);
+  if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, abort_flag));
+  if (!softmax_all(ok)) {
+    if (!ok) atomicExch(p.err, kDevTimeoutEpilogue);
     *abort_flag = 1;
     return;
   }
-  // row sum of both halves
-  red[512 + half * 128 + r] = l;
-  named_bar_sync(pair_bar, 64);
-  l += red[512 + (half ^ 1) * 128 + r];
+  // merge the two streams per row: each hands its (max, sum) to the other's thread of the
+  // same row, then both scale their O by 2^(m_s - m) and each writes half of the columns
+  red[st * 256 + r] = m_ref;
+  red[st * 256 + 128 + r] = l;
+  named_bar_sync(1, 256);
+  const float mo = red[(st ^ 1) * 256 + r], lo_other = red[(st ^ 1) * 256 + 128 + r];
+  const float m0 = st == 0 ? m_ref : mo, m1 = st == 0 ? mo : m_ref;
+  const float l0 = st == 0 ? l : lo_other, l1 = st == 0 ? lo_other : l;
+  const float m = fmaxf(m0, m1);
+  // a stream that saw no key of this row (or had no block) has m = -inf and adds nothing;
+  // its O columns may never have been written, so they are not read into the sum
+  const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - m);
+  const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - m);
+  const float lt = l0 * f0 + l1 * f1;
   tc_fence_after();
   const int i = r / p.group;
   const int h = blockIdx.y * p.group + r % p.group;
   const bool valid = q0 + i < p.tok_per_req;
   const long t = (long)b * p.tok_per_req + q0 + i;
-  const float inv = 1.0f / l;
+  const float inv = 1.0f / lt;
+  const int c_lo = st == 0 ? 0 : G::kOHalf, c_hi = st == 0 ? G::kOHalf : HD;
+  const uint32_t o0 = lane_base + G::kOCol, o1 = o0 + HD;
 #pragma unroll 1
-  for (int c = o_lo; c < o_hi; c += 16) {
-    float v[16];
-    tmem_ld16(lane_base + G::kOCol + c, v);
+  for (int c = c_lo; c < c_hi; c += 16) {
+    float v[16], w[16];
+    tmem_ld16(o0 + c, v);
+    tmem_ld16(o1 + c, w);
     if (!valid) continue;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = ((f0 != 0.f ? v[e] * f0 : 0.f) + (f1 != 0.f ? w[e] * f1 : 0.f)) * inv;
     if (p.n_splits == 1) {
       uint32_t hw[8], lw[8];
 #pragma unroll
-      for (int e = 0; e < 16; e += 2) split_bf16x2(v[e] * inv, v[e + 1] * inv, hw[e / 2], lw[e / 2]);
+      for (int e = 0; e < 16; e += 2) split_bf16x2(v[e], v[e + 1], hw[e / 2], lw[e / 2]);
       bf16_t* oh = p.out + (t * p.H + h) * HD + c;
       bf16_t* ol = p.out_lo + (t * p.H + h) * HD + c;
       reinterpret_cast<uint4*>(oh)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -260,11 +270,10 @@ DLLM_DEV void softmax_rows(const AttnTcParams& p, uint32_t tmem_base, uint64_t* 
     } else {
       float4* po = reinterpret_cast<float4*>(p.part_o + (((long)sp * p.T + t) * p.H + h) * HD + c);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        po[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv, v[4 * e + 3] * inv);
+      for (int e = 0; e < 4; ++e) po[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     }
   }
-  if (valid && half == 0 && p.n_splits > 1) p.part_lse[((long)sp * p.T + t) * p.H + h] = m_ref + __log2f(l);
+  if (valid && st == 0 && p.n_splits > 1) p.part_lse[((long)sp * p.T + t) * p.H + h] = m + __log2f(lt);
 }
 
 template <int HD>
@@ -286,11 +295,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* k_empty = k_full + ST;
   uint64_t* v_full = k_empty + ST;
   uint64_t* v_empty = v_full + ST;
-  uint64_t* s_full = v_empty + ST;
-  uint64_t* s_empty = s_full + G::kSBufs;
-  uint64_t* p_full = s_empty + G::kSBufs;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* o_final = p_empty + 2;
+  uint64_t* s_full = v_empty + ST;     // [2]: stream s's S(j) is in its buffer
+  uint64_t* p_full = s_full + 2;       // [2]: stream s's P(j) is written over it
+  uint64_t* pv_done = p_full + 2;      // [2]: stream s's P V(j) completed (its buffer is free)
+  uint64_t* o_final = pv_done + 2;
   uint64_t* drain = o_final + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -319,13 +327,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int i = 0; i < G::kSBufs; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 256);
-    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&p_full[i], 256);
-      mbar_init(&p_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);   // one arrival per softmax warp of the stream
+      mbar_init(&pv_done[i], 1);
     }
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
@@ -377,33 +382,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     bool ok = mbar_wait(q_full, 0, abort_flag);
-    const uint32_t d_o = tmem_base + G::kOCol;
-    auto issue_pv = [&](int jj) -> bool {
-      const int pb = jj & 1, st = jj % ST;
-      if (!mbar_wait(&v_full[st], (jj / ST) & 1, abort_flag)) return false;
-      if (!mbar_wait(&p_full[pb], (jj >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t p_hi = tmem_base + G::kPCol + pb * BK;
-      const uint32_t p_lo = p_hi + BK / 2;
-      const uint32_t v0 = smem_u32(sV + st * G::kKV);
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t bdesc = sdesc_mn_sw128(v0 + kk * 16 * 128, G::kKatom);
-        umma_bf16_ts(d_o, p_hi + kk * 8, bdesc, kIdPV, (jj | kk) != 0);
-        umma_bf16_ts(d_o, p_lo + kk * 8, bdesc, kIdPV, 1);
-      }
-      umma_commit(&p_empty[pb]);
-      umma_commit(&v_empty[st]);
-      return true;
-    };
-    // S = Q K^T for block jj into S buffer jj % kSBufs
+    // S(jj) = Q K(jj)^T into stream jj&1's buffer
     auto issue_s = [&](int jj) -> bool {
-      const int st = jj % ST, sb = jj % G::kSBufs;
-      if (!mbar_wait(&k_full[st], (jj / ST) & 1, abort_flag)) return false;
-      if (!mbar_wait(&s_empty[sb], ((jj / G::kSBufs) & 1) ^ 1, abort_flag)) return false;
+      const int kst = jj % ST, sb = jj & 1;
+      if (!mbar_wait(&k_full[kst], (jj / ST) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t d_s = tmem_base + sb * G::kSCols;
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK + st * G::kKV);
+      const uint32_t d_s = tmem_base + G::kSCol + sb * BK;
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK + kst * G::kKV);
 #pragma unroll
       for (int a = 0; a < AT; ++a)
 #pragma unroll
@@ -411,16 +396,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           umma_bf16(d_s, sdesc_k_sw128(q_base + a * 128 * 128 + kk * 32),
                     sdesc_k_sw128(k_base + a * G::kKatom + kk * 32), kIdQK, (a | kk) != 0);
       umma_commit(&s_full[sb]);
-      umma_commit(&k_empty[st]);
+      umma_commit(&k_empty[kst]);
       return true;
     };
-    // S runs kSBufs - 1 blocks ahead of P V, so the tensor pipe always has the next
-    // scores queued while the softmax warps work on the current block
-    constexpr int kAhead = G::kSBufs - 1;
-    for (int j = 0; j < kAhead && j < nblk && ok; ++j) ok = issue_s(j);
+    // O_(jj&1) += P_hi(jj) V(jj) + P_lo(jj) V(jj); the stream's first block overwrites O
+    auto issue_pv = [&](int jj) -> bool {
+      const int vst = jj % ST, sb = jj & 1, i = jj >> 1;
+      if (!mbar_wait(&v_full[vst], (jj / ST) & 1, abort_flag)) return false;
+      if (!mbar_wait(&p_full[sb], i & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t p_hi = tmem_base + G::kSCol + sb * BK;
+      const uint32_t p_lo = p_hi + BK / 2;
+      const uint32_t d_o = tmem_base + G::kOCol + sb * HD;
+      const uint32_t v0 = smem_u32(sV + vst * G::kKV);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint64_t bdesc = sdesc_mn_sw128(v0 + kk * 16 * 128, G::kKatom);
+        umma_bf16_ts(d_o, p_hi + kk * 8, bdesc, kIdPV, (i | kk) != 0);
+        umma_bf16_ts(d_o, p_lo + kk * 8, bdesc, kIdPV, 1);
+      }
+      umma_commit(&v_empty[vst]);
+      umma_commit(&pv_done[sb]);
+      return true;
+    };
+    if (ok && nblk > 0) ok = issue_s(0);
+    if (ok && nblk > 1) ok = issue_s(1);
     for (int j = 0; j < nblk && ok; ++j) {
-      if (j + kAhead < nblk && !issue_s(j + kAhead)) { ok = false; break; }
       if (!issue_pv(j)) { ok = false; break; }
+      if (j + 2 < nblk) {
+        // S(j+2) goes into the columns P V(j) reads: wait until that MMA has completed
+        if (!mbar_wait(&pv_done[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!issue_s(j + 2)) { ok = false; break; }
+      }
     }
     if (ok) umma_commit(o_final);
     if (!ok) {
@@ -430,8 +437,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     umma_commit(drain);
     mbar_drain(drain, 0);
   } else if (warp >= 2) {
-    softmax_rows<HD>(p, tmem_base, s_full, s_empty, p_full, p_empty, o_final,
-                     reinterpret_cast<float*>(smem + G::kOffRed), abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);
+    softmax_stream<HD>(p, tmem_base, s_full, p_full, o_final, reinterpret_cast<float*>(smem + G::kOffRed),
+                       abort_flag, warp, lane, q0, b, sp, ks, ke, nblk);
   }
   __syncwarp();
   tc_fence_before();

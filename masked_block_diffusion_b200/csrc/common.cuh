@@ -118,14 +118,30 @@ DLLM_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint of 256 ns: the waiting thread re-checks the phase at
+// least that often instead of after the hardware's default suspend interval. Measured on
+// the grouped expert GEMMs' pipelines (26B canvas pass): gate/up 1.80 vs 1.94 ms per pass,
+// down 0.94 vs 0.96; 32 ns measured the same as 256, a test_wait spin slower than either.
+DLLM_DEV bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(256u)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `parity` to complete. Gives up after g_wait_limit_ns, or as
 // soon as another role of the CTA has raised *abort; returns false then.
 DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_hint(bar, parity)) return true;
   const unsigned long long limit = g_wait_limit_ns;
   unsigned long long t0 = global_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity)) return true;
     if (*abort) return false;
     if (global_ns() - t0 > limit) return false;
   }
