@@ -165,10 +165,10 @@ def parse_ncu_csv(path):
 
 
 def ingest_ncu(path, workload, routing, command):
-    """Writes TRAFFIC_FILE from an ncu capture of the gate/up GEMM's canvas-pass launches
-    of `workload` under `routing`: mean DRAM bytes and duration per launch, with the hash
+    """Records in TRAFFIC_FILE, under (workload, routing), an ncu capture of the gate/up
+    GEMM's canvas-pass launches: mean DRAM bytes and duration per launch, with the hash
     of the kernel's sources so that the benchmark reports the figure only while those
-    sources are unchanged."""
+    sources are unchanged. Entries of other (workload, routing) pairs are kept."""
     rows, names = parse_ncu_csv(path)
     ids = sorted(i for i in rows if "EpiSwiGLU" in names[i])
     if not ids:
@@ -179,21 +179,29 @@ def ingest_ncu(path, workload, routing, command):
            "dram_bytes_per_launch": statistics.mean(dram), "ns_per_launch_cold": statistics.mean(dur),
            "workload": workload, "routing": routing, "sources_sha256": sources_sha256(), "command": command,
            "csv": os.path.basename(path)}
+    records = _traffic_records()
+    records[f"{workload}|{routing}"] = rec
     os.makedirs(os.path.dirname(TRAFFIC_FILE), exist_ok=True)
     with open(TRAFFIC_FILE, "w") as f:
-        json.dump(rec, f, indent=1)
+        json.dump(records, f, indent=1, sort_keys=True)
         f.write("\n")
     print(json.dumps(rec))
 
 
-def recorded_traffic(workload, routing):
-    """Mean DRAM bytes per gate/up launch from the recorded ncu capture, if it was taken
-    on this workload and routing with the kernel sources unchanged since; else None."""
+def _traffic_records():
     if not os.path.exists(TRAFFIC_FILE):
-        return None
-    rec = json.load(open(TRAFFIC_FILE))
-    if (rec.get("sources_sha256") != sources_sha256() or rec.get("workload") != workload
-            or rec.get("routing") != routing):
+        return {}
+    data = json.load(open(TRAFFIC_FILE))
+    if "workload" in data:   # a single record
+        return {f"{data['workload']}|{data['routing']}": data}
+    return data
+
+
+def recorded_traffic(workload, routing):
+    """Mean DRAM bytes per gate/up launch from the recorded ncu capture of this workload
+    and routing, if the kernel sources are unchanged since; else None."""
+    rec = _traffic_records().get(f"{workload}|{routing}")
+    if rec is None or rec.get("sources_sha256") != sources_sha256():
         return None
     return float(rec["dram_bytes_per_launch"])
 

@@ -185,7 +185,9 @@ long long dllm_launch_count(const dllm_handle* h);
 
 /* Limit, in nanoseconds, of the pipeline waits inside the kernels (a stage waiting for
  * its TMA copy, an MMA for its operands, an epilogue for its accumulator, a split-K
- * rank for its peers); ns <= 0 restores the default of 2 s. The waits that let copies
+ * rank for its peers); ns <= 0 restores the default of 2 s. A wait first suspends for up
+ * to 256 ns and counts the limit from there, so a wait that completes within that
+ * window never gives up, whatever the limit. The waits that let copies
  * and MMAs already in flight land before a kernel exits keep the default. The limit is
  * one value per device, shared by every handle on it; it exists so that the timeout
  * path (DLLM_E_TIMEOUT, context intact) can be exercised. Synchronises the stream. */

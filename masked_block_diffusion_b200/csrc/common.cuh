@@ -134,8 +134,10 @@ DLLM_DEV bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete. Gives up after g_wait_limit_ns, or as
-// soon as another role of the CTA has raised *abort; returns false then.
+// Waits for the phase of `parity` to complete. Gives up once g_wait_limit_ns has passed
+// after a first wait of up to the 256 ns hint, or as soon as another role of the CTA has
+// raised *abort; returns false then. (Reading the limit before the first try measured
+// slower: gate/up 2.07 vs 1.80 ms per pass.)
 DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait_hint(bar, parity)) return true;
   const unsigned long long limit = g_wait_limit_ns;

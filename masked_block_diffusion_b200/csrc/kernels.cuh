@@ -184,14 +184,16 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ x
 }
 
 // Top-k of token t's E logits (ties to the lower expert) and the softmax of the k
-// selected logits as gates, by one warp (E <= 256, k <= 32).
+// selected logits as gates, by one warp (E <= 256, k <= 32). A NaN logit counts as -inf,
+// so every selected index is a valid expert whatever the hidden state holds.
 DLLM_DEV void topk_token(const float* logits, int t, int E, int k, int32_t* idx, float* gate, int lane) {
   float v[8];
   bool taken[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
-    v[j] = (e < E) ? logits[(long)t * E + e] : -INFINITY;
+    const float x = (e < E) ? logits[(long)t * E + e] : -INFINITY;
+    v[j] = x != x ? -INFINITY : x;
     taken[j] = (e >= E);
   }
   float sel_v = 0.f, top = 0.f;

@@ -1,0 +1,62 @@
+"""Host logic of bench.py: the ncu traffic record the roofline line reads."""
+
+import importlib.util
+import json
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture()
+def bench(tmp_path, monkeypatch):
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(mod, "TRAFFIC_FILE", str(tmp_path / "traffic.json"))
+    return mod
+
+
+def _csv(path, launches):
+    """An `ncu --csv` metrics log: one row per (launch, metric)."""
+    hdr = '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+    rows = []
+    for i, (name, rd, wr, ns) in enumerate(launches):
+        rows.append(f'"{i}","{name}","dram__bytes_read.sum","byte","{rd}"\n')
+        rows.append(f'"{i}","{name}","dram__bytes_write.sum","byte","{wr}"\n')
+        rows.append(f'"{i}","{name}","gpu__time_duration.sum","nsecond","{ns}"\n')
+    path.write_text("==PROF== noise line\n" + hdr + "".join(rows))
+
+
+def test_traffic_is_recorded_per_workload_and_routing(bench, tmp_path):
+    gu = "void gemm_tc_kernel<64, 6, 2, 2, PersistentGroupedSched<1>, EpiSwiGLU<64>>(...)"
+    other = "void gemm_tc_kernel<64, 6, 1, 2, DenseSched, EpiResidualT<64>>(...)"
+    a = tmp_path / "a.csv"
+    _csv(a, [(gu, "100", "10", "5000"), (other, "999", "999", "1"), (gu, "300", "30", "7000")])
+    bench.ingest_ncu(str(a), "w", "model", "cmd a")
+    b = tmp_path / "b.csv"
+    _csv(b, [(gu, "1000", "0", "9000")])
+    bench.ingest_ncu(str(b), "w", "uniform", "cmd b")
+    assert bench.recorded_traffic("w", "model") == pytest.approx((110 + 330) / 2)
+    assert bench.recorded_traffic("w", "uniform") == pytest.approx(1000)
+    assert bench.recorded_traffic("other", "model") is None
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    assert rec["w|model"]["launches"] == 2 and rec["w|model"]["command"] == "cmd a"
+
+
+def test_traffic_is_dropped_once_the_kernel_sources_change(bench, tmp_path, monkeypatch):
+    gu = "gemm_tc_kernel<...EpiSwiGLU<128>>"
+    a = tmp_path / "a.csv"
+    _csv(a, [(gu, "5", "5", "1")])
+    bench.ingest_ncu(str(a), "w", "model", "")
+    assert bench.recorded_traffic("w", "model") == pytest.approx(10)
+    monkeypatch.setattr(bench, "sources_sha256", lambda: "changed")
+    assert bench.recorded_traffic("w", "model") is None
+
+
+def test_a_capture_without_the_gate_up_kernel_is_refused(bench, tmp_path):
+    a = tmp_path / "a.csv"
+    _csv(a, [("attn_tc_kernel<176>", "1", "1", "1")])
+    with pytest.raises(SystemExit):
+        bench.ingest_ncu(str(a), "w", "model", "")

@@ -138,8 +138,10 @@ def test_timeout_path_reports_and_keeps_the_context_usable():
 
 
 def test_single_ops_poison_their_outputs_on_timeout():
+    # a wait first suspends for up to 256 ns before the limit counts, so the shapes are
+    # large enough (44 k blocks per tile) that some wait of each launch takes longer
     from synth import bf16_bits_to_f32, f32_to_bf16_bits, normal_f32, uniform_f32
-    T, d, V = 64, 256, 1024
+    T, d, V = 64, 2816, 4096
     y = bf16_bits_to_f32(f32_to_bf16_bits(uniform_f32(5, 1, T * d, -2, 2)))
     hd = bf16_bits_to_f32(f32_to_bf16_bits(normal_f32(5, 2, V * d)))
     Y = torch.from_numpy(f32_to_bf16_bits(y).view(np.int16)).cuda()
