@@ -164,11 +164,11 @@ def parse_ncu_csv(path):
     return rows, names
 
 
-def ingest_ncu(path, workload, routing, command):
-    """Records in TRAFFIC_FILE, under (workload, routing), an ncu capture of the gate/up
+def ingest_ncu(path, workload, routing, experts, command):
+    """Records in TRAFFIC_FILE, under (workload, routing, expert format), an ncu capture of the gate/up
     GEMM's canvas-pass launches: mean DRAM bytes and duration per launch, with the hash
     of the kernel's sources so that the benchmark reports the figure only while those
-    sources are unchanged. Entries of other (workload, routing) pairs are kept."""
+    sources are unchanged. Entries of other (workload, routing, format) keys are kept."""
     rows, names = parse_ncu_csv(path)
     ids = sorted(i for i in rows if "EpiSwiGLU" in names[i])
     if not ids:
@@ -177,10 +177,11 @@ def ingest_ncu(path, workload, routing, command):
     dur = [rows[i].get("gpu__time_duration.sum", 0.0) for i in ids]
     rec = {"kernel": "grouped expert gate/up GEMM + SwiGLU", "launches": len(ids),
            "dram_bytes_per_launch": statistics.mean(dram), "ns_per_launch_cold": statistics.mean(dur),
-           "workload": workload, "routing": routing, "sources_sha256": sources_sha256(), "command": command,
+           "workload": workload, "routing": routing, "experts": experts, "sources_sha256": sources_sha256(),
+           "command": command,
            "csv": os.path.basename(path)}
     records = _traffic_records()
-    records[f"{workload}|{routing}"] = rec
+    records[f"{workload}|{routing}|{experts}"] = rec
     os.makedirs(os.path.dirname(TRAFFIC_FILE), exist_ok=True)
     with open(TRAFFIC_FILE, "w") as f:
         json.dump(records, f, indent=1, sort_keys=True)
@@ -192,15 +193,13 @@ def _traffic_records():
     if not os.path.exists(TRAFFIC_FILE):
         return {}
     data = json.load(open(TRAFFIC_FILE))
-    if "workload" in data:   # a single record
-        return {f"{data['workload']}|{data['routing']}": data}
     return data
 
 
-def recorded_traffic(workload, routing):
-    """Mean DRAM bytes per gate/up launch from the recorded ncu capture of this workload
-    and routing, if the kernel sources are unchanged since; else None."""
-    rec = _traffic_records().get(f"{workload}|{routing}")
+def recorded_traffic(workload, routing, experts):
+    """Mean DRAM bytes per gate/up launch from the recorded ncu capture of this workload,
+    routing and expert format, if the kernel sources are unchanged since; else None."""
+    rec = _traffic_records().get(f"{workload}|{routing}|{experts}")
     if rec is None or rec.get("sources_sha256") != sources_sha256():
         return None
     return float(rec["dram_bytes_per_launch"])
@@ -494,7 +493,7 @@ def run_ours(args):
     act = Bq * C * cfg.top_k * (cfg.d_model + cfg.ffn_dim) * 2
     wbytes = 1 if args.experts == "fp8" else 2
     routed = (gu_bytes - act) / (2 * cfg.ffn_dim * cfg.d_model * wbytes)
-    traffic = recorded_traffic(w.name, args.routing)
+    traffic = recorded_traffic(w.name, args.routing, args.experts)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak_hbm, "unit": "GB/s",
                 "frac": round(achieved / peak_hbm, 4), "traffic": round(traffic) if traffic else None,
                 "kernel": "grouped expert gate/up GEMM + SwiGLU (tcgen05, one launch per layer)",
@@ -666,7 +665,8 @@ def run_reference(args):
 def main():
     args = parse_args()
     if args.ingest_ncu:
-        ingest_ncu(args.ingest_ncu, resolve_workload(args).name, args.routing, os.environ.get("NCU_COMMAND", ""))
+        ingest_ncu(args.ingest_ncu, resolve_workload(args).name, args.routing, args.experts,
+                   os.environ.get("NCU_COMMAND", ""))
         return
     if args.impl == "reference":
         run_reference(args)

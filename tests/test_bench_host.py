@@ -34,29 +34,30 @@ def test_traffic_is_recorded_per_workload_and_routing(bench, tmp_path):
     other = "void gemm_tc_kernel<64, 6, 1, 2, DenseSched, EpiResidualT<64>>(...)"
     a = tmp_path / "a.csv"
     _csv(a, [(gu, "100", "10", "5000"), (other, "999", "999", "1"), (gu, "300", "30", "7000")])
-    bench.ingest_ncu(str(a), "w", "model", "cmd a")
+    bench.ingest_ncu(str(a), "w", "model", "bf16", "cmd a")
     b = tmp_path / "b.csv"
     _csv(b, [(gu, "1000", "0", "9000")])
-    bench.ingest_ncu(str(b), "w", "uniform", "cmd b")
-    assert bench.recorded_traffic("w", "model") == pytest.approx((110 + 330) / 2)
-    assert bench.recorded_traffic("w", "uniform") == pytest.approx(1000)
-    assert bench.recorded_traffic("other", "model") is None
+    bench.ingest_ncu(str(b), "w", "uniform", "bf16", "cmd b")
+    assert bench.recorded_traffic("w", "model", "bf16") == pytest.approx((110 + 330) / 2)
+    assert bench.recorded_traffic("w", "uniform", "bf16") == pytest.approx(1000)
+    assert bench.recorded_traffic("other", "model", "bf16") is None
+    assert bench.recorded_traffic("w", "model", "fp8") is None   # another weight format
     rec = json.load(open(bench.TRAFFIC_FILE))
-    assert rec["w|model"]["launches"] == 2 and rec["w|model"]["command"] == "cmd a"
+    assert rec["w|model|bf16"]["launches"] == 2 and rec["w|model|bf16"]["command"] == "cmd a"
 
 
 def test_traffic_is_dropped_once_the_kernel_sources_change(bench, tmp_path, monkeypatch):
     gu = "gemm_tc_kernel<...EpiSwiGLU<128>>"
     a = tmp_path / "a.csv"
     _csv(a, [(gu, "5", "5", "1")])
-    bench.ingest_ncu(str(a), "w", "model", "")
-    assert bench.recorded_traffic("w", "model") == pytest.approx(10)
+    bench.ingest_ncu(str(a), "w", "model", "bf16", "")
+    assert bench.recorded_traffic("w", "model", "bf16") == pytest.approx(10)
     monkeypatch.setattr(bench, "sources_sha256", lambda: "changed")
-    assert bench.recorded_traffic("w", "model") is None
+    assert bench.recorded_traffic("w", "model", "bf16") is None
 
 
 def test_a_capture_without_the_gate_up_kernel_is_refused(bench, tmp_path):
     a = tmp_path / "a.csv"
     _csv(a, [("attn_tc_kernel<176>", "1", "1", "1")])
     with pytest.raises(SystemExit):
-        bench.ingest_ncu(str(a), "w", "model", "")
+        bench.ingest_ncu(str(a), "w", "model", "bf16", "")
