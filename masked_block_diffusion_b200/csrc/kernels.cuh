@@ -72,12 +72,20 @@ __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ 
     float4 v = xr[c];
     if (nparts > 0) {
       const float4* pr = reinterpret_cast<const float4*>(part + (long)t * d) + c;
-      for (int s = 0; s < nparts; ++s) {
-        const float4 a = pr[s * (pstride / 4)];
-        v.x += a.x;
-        v.y += a.y;
-        v.z += a.z;
-        v.w += a.w;
+      // four partials' loads at a time, all in flight before they are added (in slice order)
+      for (int s0 = 0; s0 < nparts; s0 += 4) {
+        float4 a[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = s0 + u < nparts ? pr[(s0 + u) * (pstride / 4)] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (s0 + u < nparts) {
+            v.x += a[u].x;
+            v.y += a[u].y;
+            v.z += a[u].z;
+            v.w += a[u].w;
+          }
+        }
       }
       xr[c] = v;
     }
@@ -239,11 +247,20 @@ __global__ void topk_kernel(float* __restrict__ logits, int T, int E, int k, int
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = 0.f;
-    for (int s = 0; s < nparts; ++s) {
-      const float* ps = part + s * pstride + (long)t * E;
+    // four partials' loads at a time, all in flight before they are added (in slice order)
+    for (int s0 = 0; s0 < nparts; s0 += 4) {
+      float pv[4][8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (lane + 32 * j < E) v[j] += ps[lane + 32 * j];
+      for (int u = 0; u < 4; ++u) {
+        const float* ps = part + (s0 + u) * pstride + (long)t * E;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pv[u][j] = (s0 + u < nparts && lane + 32 * j < E) ? ps[lane + 32 * j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (s0 + u < nparts) v[j] += pv[u][j];
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -433,7 +450,12 @@ __global__ void combine_kernel(float* __restrict__ x, const float* __restrict__ 
 // norm, or the final norm before the LM head): x is updated in place, then
 // v = x * rsqrt(mean(x^2) + eps) * g is written as the (hi, lo) bf16 pair. One block per
 // token; the same per-row arithmetic as combine_kernel and rmsnorm_kernel.
-__global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x, const float* __restrict__ o,
+constexpr int kCombineChunks = 3;   // float4 columns per thread: d / 4 <= 3 * blockDim
+
+// Two 256-thread blocks per SM (at most 128 registers a thread): all 256 tokens of a canvas
+// stay resident with their loads in flight (measured 0.31 vs 0.36 ms per 26B canvas pass
+// with one block per SM, 0.47 before the loads were issued together).
+__global__ void __launch_bounds__(256, 2) combine_norm_kernel(float* __restrict__ x, const float* __restrict__ o,
                                                            const int32_t* __restrict__ slot_of,
                                                            const float* __restrict__ gate, int k, int d,
                                                            const float* __restrict__ g, float eps,
@@ -442,33 +464,78 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(float* __restrict__ x
   pdl_begin();
   const int t = blockIdx.x;
   float4* xr = reinterpret_cast<float4*>(x + (long)t * d);
-  float ss = 0.f;
+  const float4* gr = reinterpret_cast<const float4*>(g);
+  const int n4 = d / 4;
   const CombineRow cr(o, slot_of, gate, t, k, d);
-  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+  // every load of this thread's first kCombineChunks float4 columns is issued before any
+  // is used: the k routed rows, x and the gains (a 256-thread block covers d <= 3072 this
+  // way; wider rows finish column by column below)
+  float4 v[kCombineChunks][kMaxK], xv[kCombineChunks], gv[kCombineChunks];
+#pragma unroll
+  for (int i = 0; i < kCombineChunks; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    const bool on = c < n4;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) v[i][j] = (on && j < k) ? cr.row[j][c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    xv[i] = on ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    gv[i] = on ? gr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kCombineChunks; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c >= n4) continue;
+    // the same per-column arithmetic as combine_kernel: sum_j w_j o_j in j order, then + x
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j < k) {
+        acc.x = fmaf(cr.w[j], v[i][j].x, acc.x);
+        acc.y = fmaf(cr.w[j], v[i][j].y, acc.y);
+        acc.z = fmaf(cr.w[j], v[i][j].z, acc.z);
+        acc.w = fmaf(cr.w[j], v[i][j].w, acc.w);
+      }
+    }
+    xv[i].x += acc.x;
+    xv[i].y += acc.y;
+    xv[i].z += acc.z;
+    xv[i].w += acc.w;
+    xr[c] = xv[i];
+    ss += xv[i].x * xv[i].x + xv[i].y * xv[i].y + xv[i].z * xv[i].z + xv[i].w * xv[i].w;
+  }
+  // rows wider than kCombineChunks * blockDim float4s: the rest column by column
+  for (int c = threadIdx.x + kCombineChunks * blockDim.x; c < n4; c += blockDim.x) {
     const float4 acc = cr.at(c);
-    float4 xv = xr[c];
-    xv.x += acc.x;
-    xv.y += acc.y;
-    xv.z += acc.z;
-    xv.w += acc.w;
-    xr[c] = xv;
-    ss += xv.x * xv.x + xv.y * xv.y + xv.z * xv.z + xv.w * xv.w;
+    float4 a = xr[c];
+    a.x += acc.x;
+    a.y += acc.y;
+    a.z += acc.z;
+    a.w += acc.w;
+    xr[c] = a;
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
   }
   __shared__ float red[32];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-    v = warp_sum(v);
-    if (threadIdx.x == 0) red[0] = v;
+    float a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    a = warp_sum(a);
+    if (threadIdx.x == 0) red[0] = a;
   }
   __syncthreads();
   const float r = rsqrtf(red[0] / (float)d + eps);
-  const float4* gr = reinterpret_cast<const float4*>(g);
-  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
-    const float4 v = xr[c], gg = gr[c];   // this thread's own writes above
-    store_norm_terms(y, y_lo, y_lo2, t, d, c, make_float4(v.x * r * gg.x, v.y * r * gg.y, v.z * r * gg.z, v.w * r * gg.w));
+#pragma unroll
+  for (int i = 0; i < kCombineChunks; ++i) {
+    const int c = threadIdx.x + i * blockDim.x;
+    if (c >= n4) continue;
+    store_norm_terms(y, y_lo, y_lo2, t, d, c,
+                     make_float4(xv[i].x * r * gv[i].x, xv[i].y * r * gv[i].y, xv[i].z * r * gv[i].z,
+                                 xv[i].w * r * gv[i].w));
+  }
+  for (int c = threadIdx.x + kCombineChunks * blockDim.x; c < n4; c += blockDim.x) {
+    const float4 a = xr[c], gg = gr[c];   // this thread's own writes above
+    store_norm_terms(y, y_lo, y_lo2, t, d, c, make_float4(a.x * r * gg.x, a.y * r * gg.y, a.z * r * gg.z, a.w * r * gg.w));
   }
 }
 
