@@ -68,7 +68,7 @@ extern "C" {
 
 typedef struct dllm_handle dllm_handle;
 
-/* Model and capacity. Requirements of this build: d_model % 256 == 0, d_model <= 4096,
+/* Model and capacity. Requirements of this library: d_model % 256 == 0, d_model <= 4096,
  * head_dim in {64, 176}, n_heads * head_dim % 64 == 0, ffn_dim % 64 == 0,
  * vocab % 256 == 0, n_experts <= 256, top_k <= 8 (dense: n_experts = 0, top_k = 1),
  * canvas <= 1024, mask_id = vocab - 1. */
