@@ -80,10 +80,11 @@ sigmoid(ln 3) = 3/4; MoE top-k against brute force over all subsets and the k = 
 reduction; LM-head confidence against a zero-gain closed form and log-sum-exp; commit
 schedule, strict threshold, T2T edit rule and sampler invariants; the KV-cache pass
 against an uncached block-causal sequence forward; the approximate append against the
-last pass's own K/V and the exact append at a canvas without a final commit. tests/test_oracle_mutations.py plants a
-plausible mistake in each function in turn and checks that a pin fails. Values
-produced for random weights beyond those properties are "parity unpinned": no page
-prints a worked example.
+last pass's own K/V and the exact append at a canvas without a final commit; FP8 E4M3
+rounding against the format's value set, its ties and torch's float8_e4m3fn, and the
+tile scales against their round trip. tests/test_oracle_mutations.py plants a plausible
+mistake in each function in turn and checks that a pin fails. Values produced for random
+weights beyond those properties are "parity unpinned": no page prints a worked example.
 """
 
 from __future__ import annotations
