@@ -61,3 +61,31 @@ def test_a_capture_without_the_gate_up_kernel_is_refused(bench, tmp_path):
     _csv(a, [("attn_tc_kernel<176>", "1", "1", "1")])
     with pytest.raises(SystemExit):
         bench.ingest_ncu(str(a), "w", "model", "bf16", "")
+
+
+def test_design_point_routing_gives_every_expert_the_same_load(bench):
+    from synth import WORKLOADS
+    cfg = WORKLOADS["c3-moe26b-canvas"].model
+    T = cfg.canvas
+    idx = bench.uniform_routing(cfg, T)
+    assert idx.shape == (cfg.n_layers, T, cfg.top_k)
+    import numpy as np
+    for l in (0, cfg.n_layers - 1):
+        counts = np.bincount(idx[l].ravel(), minlength=cfg.n_experts)
+        assert np.all(counts == T * cfg.top_k // cfg.n_experts)          # 16 each at one canvas
+        assert all(len(set(row)) == cfg.top_k for row in idx[l].tolist())  # k distinct experts per token
+
+
+def test_gate_up_bytes_and_pass_flops_follow_the_shapes(bench):
+    from synth import WORKLOADS
+    cfg = WORKLOADS["c3-moe26b-canvas"].model
+    T, d, F, k = cfg.canvas, cfg.d_model, cfg.ffn_dim, cfg.top_k
+    # all experts: 128 x (gate + up) x F x d bf16 + the gathered rows in + the SwiGLU rows out
+    assert bench.gate_up_bytes(cfg, T) == cfg.n_experts * 2 * F * d * 2 + T * k * d * 2 + T * k * F * 2
+    assert bench.gate_up_bytes(cfg, T, routed=14) - bench.gate_up_bytes(cfg, T, routed=13) == 2 * F * d * 2
+    # one canvas pass with no LM-head rows: per layer QKV + O + experts + router + attention
+    P = 4096
+    per_layer = (2 * T * d * (cfg.q_dim + 2 * cfg.kv_dim) + 2 * T * cfg.q_dim * d + 2 * T * k * 3 * F * d
+                 + 2 * T * d * cfg.n_experts + 4 * T * (P + T) * cfg.n_heads * cfg.head_dim)
+    assert bench.pass_flops(cfg, T, P, 0) == cfg.n_layers * per_layer
+    assert bench.pass_flops(cfg, T, P, T) - bench.pass_flops(cfg, T, P, 0) == 2 * T * d * cfg.vocab
